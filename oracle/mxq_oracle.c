@@ -1,0 +1,410 @@
+/*
+ * mxq_oracle.c -- plain, slow, scalar CPU oracle for block-scaled quantization
+ * (MXFP8 rowwise with E8M0 group scales, NVFP4 two-level with E4M3 block scales).
+ *
+ * TEST INFRASTRUCTURE. This file is the reference the CUDA path is checked
+ * against. Only the test suite, the package's smoke check and the benchmark's
+ * CPU-baseline leg may load it. It shares no code, header, table or constant
+ * with the CUDA library, and the CUDA library never loads it.
+ *
+ * Every function writes out the plain definition of what it computes, one
+ * element at a time, in double precision (exact for every MXFP8 step), except
+ * the NVFP4 scale arithmetic, which the pages fix as fp32 (global FP32 scale,
+ * "effective = block_scale * global_scale") and is therefore done in IEEE
+ * binary32 with round-to-nearest-even, subnormals kept, no contraction.
+ * Build: gcc -O2 -std=c11 -fno-fast-math -ffp-contract=off -fPIC -shared.
+ *
+ * Sources (page title, section):
+ *  [P4]  "PR #1935 完整报告 -- Use TransformerEngine for MXFP8 quantization",
+ *        实现拆解 item 1: group size 32, rowwise only, flatten, zero-pad rows
+ *        to a multiple of 32, quantize, crop back, compact non-swizzled
+ *        qweight + scale; 关键源码片段: qweight, scale = mxfp8_quantize(weight),
+ *        scale stored as "<name>_scale_inv" (a dequantisation multiplier).
+ *  [P3]  "V4 mxfp4 #1372", description: power-of-two scales on Blackwell,
+ *        float8_e8m0fnu scale dtype; review: E2M1 packed two per byte
+ *        (float4_e2m1fn_x2, last dim N//2), N % block_size == 0.
+ *  [P2]  "Add FP8, NVFP4, and QARL training and export", review "What looked
+ *        solid": NVFP4 two-level global + FP8-block scaling, "effective =
+ *        block_scale * global_scale", zero blocks guarded (safe_eff).
+ *  The E8M0 rule (scale = 2^(floor(log2 amax) - 8), biased byte clamped to
+ *  [0,254], all-zero group -> 127), the E4M3 cast (RNE, saturate to +-448,
+ *  NaN propagated) and the NVFP4 global scale amax/(448*6) are the statement
+ *  of the problem these pages turn on; readings where the pages are silent
+ *  are listed beside each function.
+ *
+ * Parity status: every function below is pinned by tests in tests/ against
+ * independent formulations (brute-force nearest-code search, library casts,
+ * closed forms, invariants). orc_swizzle_scales follows NVIDIA's public
+ * block-scaled-MMA scale-factor layout, which the pages do not describe: its
+ * layout is pinned to that document's index formula only (parity unpinned by
+ * the pages).
+ */
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#define ORC_BF16 0
+#define ORC_FP32 1
+
+#define ORC_OK 0
+#define ORC_ERR_SHAPE 2
+#define ORC_ERR_DTYPE 3
+
+/* ---------------------------------------------------------------- inputs */
+
+/* Value of element k of x as a double (exact: bf16 and fp32 are subsets). */
+static double load_elem(const void* x, int dt, int64_t k) {
+  if (dt == ORC_BF16) {
+    uint16_t h;
+    memcpy(&h, (const uint8_t*)x + 2 * k, 2);
+    uint32_t u = (uint32_t)h << 16; /* bf16 is the top half of an fp32 */
+    float f;
+    memcpy(&f, &u, 4);
+    return (double)f;
+  } else {
+    float f;
+    memcpy(&f, (const uint8_t*)x + 4 * k, 4);
+    return (double)f;
+  }
+}
+
+/* ------------------------------------------------------------- E8M0 scale */
+
+/* Biased E8M0 byte of a group with absolute maximum `amax` (amax >= 0, NaN
+ * already excluded). scale = 2^(floor(log2 amax) - 8), byte = 127 + that
+ * exponent, clamped to [0, 254]; an all-zero group gives 127 (scale 1).
+ * 8 is emax of E4M3 (largest normal 448 = 1.75 * 2^8).
+ * Reading: an infinite amax has floor(log2) = +inf, which clamps to 254. */
+uint8_t orc_e8m0_from_amax(double amax) {
+  if (amax == 0.0) return 127;
+  if (isinf(amax)) return 254;
+  int e;
+  frexp(amax, &e);           /* amax = f * 2^e with f in [0.5, 1) */
+  long fl = (long)e - 1;     /* floor(log2 amax) */
+  long b = 127 + fl - 8;
+  if (b < 0) b = 0;
+  if (b > 254) b = 254;
+  return (uint8_t)b;
+}
+
+/* Value of an E8M0 byte: 2^(b - 127); 0xFF is NaN (float8_e8m0fnu). */
+double orc_e8m0_value(uint8_t b) {
+  if (b == 255) return NAN;
+  return ldexp(1.0, (int)b - 127);
+}
+
+/* ----------------------------------------------------------------- E4M3 */
+
+/* OCP FP8 E4M3 ("fn"): bias 7, normals (1 + m/8) * 2^(e-7) for e = 1..15
+ * except (e,m) = (15,7) which is NaN, subnormals m * 2^-9, no infinity,
+ * largest finite 448. */
+double orc_e4m3_decode(uint8_t c) {
+  int s = c >> 7, e = (c >> 3) & 15, m = c & 7;
+  if (e == 15 && m == 7) return NAN;
+  double v = (e == 0) ? ldexp((double)m, -9) : ldexp((double)(8 + m), e - 10);
+  return s ? -v : v;
+}
+
+/* Round-to-nearest-even of the exact value v onto the E4M3 grid, saturating
+ * every |v| > 448 (infinity included) to 448.
+ * Readings: NaN -> 0x7F (canonical positive NaN; the pages do not say which
+ * NaN); the sign of a zero result is kept (-0 and negatives that round to 0
+ * give 0x80). */
+uint8_t orc_e4m3_encode(double v) {
+  if (isnan(v)) return 0x7F;
+  uint8_t sign = signbit(v) ? 0x80 : 0x00;
+  double a = fabs(v);
+  if (a > 448.0) return sign | 0x7E;
+  /* exponent of the binade holding a; below the normal range the spacing
+   * stays that of the lowest binade (2^-6), i.e. the subnormal step 2^-9 */
+  int e;
+  if (a < ldexp(1.0, -6)) {
+    e = -6;
+  } else {
+    frexp(a, &e);
+    e -= 1;
+  }
+  double step = ldexp(1.0, e - 3);       /* 3 mantissa bits */
+  double r = nearbyint(a / step);        /* ties to even (default mode) */
+  double rv = r * step;                  /* <= 448: 448 lies on the grid */
+  if (rv == 0.0) return sign;
+  int E;
+  frexp(rv, &E);
+  int ex = E - 1;                        /* rv = 1.f * 2^ex */
+  if (ex < -6) {                         /* subnormal: rv = m * 2^-9 */
+    int m = (int)(rv / ldexp(1.0, -9));
+    return sign | (uint8_t)m;
+  }
+  int m = (int)((rv / ldexp(1.0, ex) - 1.0) * 8.0);
+  return sign | (uint8_t)(((ex + 7) << 3) | m);
+}
+
+/* ----------------------------------------------------------------- E2M1 */
+
+/* FP4 E2M1: codes 0..7 = {0, 0.5, 1, 1.5, 2, 3, 4, 6}, bit 3 = sign. */
+double orc_e2m1_decode(uint8_t c) {
+  int s = (c >> 3) & 1, e = (c >> 1) & 3, m = c & 1;
+  double v = (e == 0) ? 0.5 * m : ldexp(1.0 + 0.5 * m, e - 1);
+  return s ? -v : v;
+}
+
+/* Round-to-nearest-even onto the E2M1 grid, saturating |u| > 6 to 6.
+ * Readings: the sign of a zero result is kept (0x8); E2M1 has no NaN, and a
+ * NaN quotient is mapped to +6 (0x7), the largest finite code, as for the
+ * infinities. */
+uint8_t orc_e2m1_encode(double u) {
+  if (isnan(u)) return 0x7;
+  uint8_t sign = signbit(u) ? 0x8 : 0x0;
+  double a = fabs(u);
+  if (a > 6.0) return sign | 0x7;
+  int e;
+  if (a < 1.0) {
+    e = 0;                               /* subnormal step 0.5 */
+  } else {
+    frexp(a, &e);
+    e -= 1;
+  }
+  double step = ldexp(1.0, e - 1);       /* 1 mantissa bit */
+  double r = nearbyint(a / step);
+  double rv = r * step;                  /* <= 6 */
+  if (rv == 0.0) return sign;
+  if (rv < 1.0) return sign | 0x1;       /* 0.5 */
+  int E;
+  frexp(rv, &E);
+  int ex = E - 1;
+  int m = (int)((rv / ldexp(1.0, ex) - 1.0) * 2.0);
+  return sign | (uint8_t)(((ex + 1) << 1) | m);
+}
+
+/* --------------------------------------------------------- output roundings */
+
+/* bf16 bits of RNE(d): 8 significant bits, fp32 exponent range, subnormals
+ * kept (step 2^-133), overflow to infinity. Reading: NaN -> 0x7FC0. */
+uint16_t orc_bf16_round(double d) {
+  if (isnan(d)) return 0x7FC0;
+  uint16_t sign = signbit(d) ? 0x8000 : 0x0000;
+  double a = fabs(d);
+  if (isinf(a)) return sign | 0x7F80;
+  int e;
+  if (a < ldexp(1.0, -126)) {
+    e = -126;
+  } else {
+    frexp(a, &e);
+    e -= 1;
+  }
+  double step = ldexp(1.0, e - 7);       /* 7 stored mantissa bits */
+  double rv = nearbyint(a / step) * step;
+  if (rv >= ldexp(1.0, 128)) return sign | 0x7F80;
+  float f = (float)rv;                   /* exact: rv is a bf16 value */
+  uint32_t u;
+  memcpy(&u, &f, 4);
+  return sign | (uint16_t)(u >> 16);
+}
+
+/* fp32 bits of d, which the callers only pass when it is exactly
+ * representable or beyond the fp32 range (then +-inf). Reading: NaN ->
+ * 0x7FC00000. */
+static uint32_t f32_bits_of(double d) {
+  if (isnan(d)) return 0x7FC00000u;
+  float f = (float)d;
+  uint32_t u;
+  memcpy(&u, &f, 4);
+  return u;
+}
+
+static void store_out(void* y, int dt, int64_t k, double d) {
+  if (dt == ORC_BF16) {
+    uint16_t h = orc_bf16_round(d);
+    memcpy((uint8_t*)y + 2 * k, &h, 2);
+  } else {
+    uint32_t u = f32_bits_of(d);
+    memcpy((uint8_t*)y + 4 * k, &u, 4);
+  }
+}
+
+/* ----------------------------------------------------------------- MXFP8 */
+
+/* MXFP8 rowwise quantize of x [M, N] (row stride ld_x elements):
+ * for every row r and group j of 32 consecutive columns,
+ *   amax  = max |x| over the group's non-NaN elements (starting at +0),
+ *   b     = E8M0 byte of amax,             scale[r, j] = b,
+ *   q     = E4M3(x * 2^(127 - b)) exactly, qweight[r, c] = q.
+ * Outputs are compact: qweight [M, N] and scale [M, N/32], row-major.
+ * Reading: NaN never raises amax (a NaN scale byte would be 0xFF, which the
+ * [0,254] clamp excludes). N must be a multiple of 32. */
+int orc_mxfp8_quantize(const void* x, int dt, int64_t M, int64_t N, int64_t ld_x,
+                       uint8_t* qweight, uint8_t* scale) {
+  if (dt != ORC_BF16 && dt != ORC_FP32) return ORC_ERR_DTYPE;
+  if (M < 0 || N < 0 || N % 32 != 0 || ld_x < N) return ORC_ERR_SHAPE;
+  int64_t S = N / 32;
+  for (int64_t r = 0; r < M; r++) {
+    for (int64_t j = 0; j < S; j++) {
+      double amax = 0.0;
+      for (int i = 0; i < 32; i++) {
+        double v = load_elem(x, dt, r * ld_x + 32 * j + i);
+        if (!isnan(v) && fabs(v) > amax) amax = fabs(v);
+      }
+      uint8_t b = orc_e8m0_from_amax(amax);
+      scale[r * S + j] = b;
+      for (int i = 0; i < 32; i++) {
+        double v = load_elem(x, dt, r * ld_x + 32 * j + i);
+        qweight[r * N + 32 * j + i] = orc_e4m3_encode(ldexp(v, 127 - (int)b));
+      }
+    }
+  }
+  return ORC_OK;
+}
+
+/* MXFP8 dequantize: y[r, c] = decode_e4m3(q[r, c]) * 2^(scale[r, c/32] - 127),
+ * exact in double, then rounded to the output type (fp32: exact except
+ * overflow to inf; bf16: RNE). */
+int orc_mxfp8_dequantize(const uint8_t* qweight, const uint8_t* scale, int64_t M,
+                         int64_t N, void* y, int out_dt) {
+  if (out_dt != ORC_BF16 && out_dt != ORC_FP32) return ORC_ERR_DTYPE;
+  if (M < 0 || N < 0 || N % 32 != 0) return ORC_ERR_SHAPE;
+  int64_t S = N / 32;
+  for (int64_t r = 0; r < M; r++) {
+    for (int64_t c = 0; c < N; c++) {
+      double d = orc_e4m3_decode(qweight[r * N + c]) * orc_e8m0_value(scale[r * S + c / 32]);
+      store_out(y, out_dt, r * N + c, d);
+    }
+  }
+  return ORC_OK;
+}
+
+/* Scale bytes in the block-scaled MMA scale-factor layout (NVIDIA's public
+ * description of the 128x4 scale tiles): the [M, S] scale is padded with
+ * 0x00 to [ceil(M/128)*128, ceil(S/4)*4]; tile (i, j) holds rows 128i.. and
+ * scale columns 4j.. and starts at byte (i * ceil(S/4) + j) * 512; inside a
+ * tile, entry (r, c) lies at (r % 32) * 16 + ((r % 128) / 32) * 4 + c % 4.
+ * The pages do not describe this layout (parity unpinned by the pages). */
+int orc_swizzle_scales(const uint8_t* scale, int64_t M, int64_t S, uint8_t* out) {
+  if (M < 0 || S < 0) return ORC_ERR_SHAPE;
+  int64_t Mp = (M + 127) / 128 * 128, Sp = (S + 3) / 4 * 4;
+  memset(out, 0, (size_t)(Mp * Sp));
+  for (int64_t r = 0; r < M; r++) {
+    for (int64_t c = 0; c < S; c++) {
+      int64_t tile = (r / 128) * (Sp / 4) + c / 4;
+      int64_t off = tile * 512 + (r % 32) * 16 + ((r % 128) / 32) * 4 + c % 4;
+      out[off] = scale[r * S + c];
+    }
+  }
+  return ORC_OK;
+}
+
+/* ----------------------------------------------------------------- NVFP4 */
+
+/* Tensor absolute maximum over non-NaN elements, as an fp32 (exact: the max
+ * of fp32-representable magnitudes). */
+float orc_nvfp4_global_amax(const void* x, int dt, int64_t M, int64_t N, int64_t ld_x) {
+  double A = 0.0;
+  for (int64_t r = 0; r < M; r++)
+    for (int64_t c = 0; c < N; c++) {
+      double v = load_elem(x, dt, r * ld_x + c);
+      if (!isnan(v) && fabs(v) > A) A = fabs(v);
+    }
+  return (float)A;
+}
+
+/* NVFP4 two-level quantize of x [M, N] in fp32 arithmetic:
+ *   g     = A / 2688            (A = tensor amax; 2688 = 448 * 6), unless
+ *                               g_given, in which case *g is read;
+ *   per block of 16 consecutive columns:
+ *   amax_b = max |x| over its non-NaN elements,
+ *   s_b   = E4M3(amax_b / (6 * g))       (RNE, saturating),
+ *   eff   = decode(s_b) * g,
+ *   q_i   = E2M1(x_i / eff)              (correctly rounded fp32 quotient,
+ *                                         then RNE, saturating), or a zero
+ *                                         of x_i's sign when eff == 0;
+ *   packed[r, k] = q[r, 2k] | q[r, 2k+1] << 4.
+ * Readings: the order of the fp32 operations is the one written above (the
+ * pages give only "effective = block_scale * global_scale"); a zero global
+ * scale gives s_b = 0 and zero codes with no division; the zero-block guard
+ * writes sign-kept zero codes. Non-finite inputs are outside the method's
+ * contract: the same fp32 operations are applied, with no further meaning. */
+int orc_nvfp4_quantize(const void* x, int dt, int64_t M, int64_t N, int64_t ld_x,
+                       uint8_t* packed, uint8_t* block_scale, float* g_io, int g_given) {
+  if (dt != ORC_BF16 && dt != ORC_FP32) return ORC_ERR_DTYPE;
+  if (M < 0 || N < 0 || N % 16 != 0 || ld_x < N) return ORC_ERR_SHAPE;
+  float g;
+  if (g_given) {
+    g = *g_io;
+  } else {
+    float A = orc_nvfp4_global_amax(x, dt, M, N, ld_x);
+    g = A / 2688.0f;
+    *g_io = g;
+  }
+  int64_t B = N / 16;
+  for (int64_t r = 0; r < M; r++) {
+    for (int64_t j = 0; j < B; j++) {
+      float xs[16];
+      float amax_b = 0.0f;
+      for (int i = 0; i < 16; i++) {
+        xs[i] = (float)load_elem(x, dt, r * ld_x + 16 * j + i);
+        if (!isnan(xs[i]) && fabsf(xs[i]) > amax_b) amax_b = fabsf(xs[i]);
+      }
+      uint8_t sb;
+      float eff;
+      if (g == 0.0f) {
+        sb = 0x00;
+        eff = 0.0f;
+      } else {
+        float t = 6.0f * g;
+        float s = amax_b / t;
+        sb = orc_e4m3_encode((double)s);
+        eff = (float)orc_e4m3_decode(sb) * g;
+      }
+      block_scale[r * B + j] = sb;
+      uint8_t codes[16];
+      for (int i = 0; i < 16; i++) {
+        if (eff == 0.0f) {
+          codes[i] = signbit(xs[i]) ? 0x8 : 0x0;
+        } else {
+          float u = xs[i] / eff;
+          codes[i] = orc_e2m1_encode((double)u);
+        }
+      }
+      for (int k = 0; k < 8; k++)
+        packed[r * (N / 2) + 8 * j + k] = (uint8_t)(codes[2 * k] | (codes[2 * k + 1] << 4));
+    }
+  }
+  return ORC_OK;
+}
+
+/* NVFP4 dequantize: eff = decode_e4m3(s_b) * g and y = decode_e2m1(q) * eff,
+ * both fp32 products, then rounded to the output type. */
+int orc_nvfp4_dequantize(const uint8_t* packed, const uint8_t* block_scale, float g,
+                         int64_t M, int64_t N, void* y, int out_dt) {
+  if (out_dt != ORC_BF16 && out_dt != ORC_FP32) return ORC_ERR_DTYPE;
+  if (M < 0 || N < 0 || N % 16 != 0) return ORC_ERR_SHAPE;
+  int64_t B = N / 16;
+  for (int64_t r = 0; r < M; r++) {
+    for (int64_t c = 0; c < N; c++) {
+      uint8_t byte = packed[r * (N / 2) + c / 2];
+      uint8_t code = (c % 2 == 0) ? (byte & 0x0F) : (byte >> 4);
+      float eff = (float)orc_e4m3_decode(block_scale[r * B + c / 16]) * g;
+      float v = (float)orc_e2m1_decode(code) * eff;
+      store_out(y, out_dt, r * N + c, (double)v);
+    }
+  }
+  return ORC_OK;
+}
+
+/* ------------------------------------------------- element-wise batch loops */
+
+/* The scalar codecs above applied to n values (for exhaustive checks). */
+void orc_e4m3_encode_array(const double* v, int64_t n, uint8_t* out) {
+  for (int64_t i = 0; i < n; i++) out[i] = orc_e4m3_encode(v[i]);
+}
+
+void orc_e2m1_encode_array(const double* u, int64_t n, uint8_t* out) {
+  for (int64_t i = 0; i < n; i++) out[i] = orc_e2m1_encode(u[i]);
+}
+
+void orc_e8m0_from_amax_array(const double* a, int64_t n, uint8_t* out) {
+  for (int64_t i = 0; i < n; i++) out[i] = orc_e8m0_from_amax(a[i]);
+}
+
+void orc_bf16_round_array(const double* d, int64_t n, uint16_t* out) {
+  for (int64_t i = 0; i < n; i++) out[i] = orc_bf16_round(d[i]);
+}

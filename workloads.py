@@ -1,0 +1,140 @@
+"""Seeded synthetic inputs for block-scaled quantization.
+
+This module only draws random numbers and lays them out; it holds none of the
+quantization arithmetic. Both the CUDA path and the CPU oracle consume the
+bytes it returns. Every tensor is produced as float32 from
+``numpy.random.default_rng(seed)`` and rounded to bf16 (round-to-nearest-even,
+via torch's fp32 -> bf16 cast), and returned as bf16 bit patterns (uint16).
+
+Workloads (one per benchmark configuration; shapes are parameters so the
+tests can draw smaller instances of the same recipe):
+
+1. ``planted``      bf16 [256, 1024] N(0,1), seed 0, plus hand-planted groups
+                    in group 0 of rows 0-7 (all-zero, one 1e4 outlier, +-448,
+                    bf16 subnormals, one NaN, one +Inf, E4M3 rounding ties,
+                    largest bf16 magnitudes).
+2. ``linear_weight``  bf16 [4096, 4096] N(0, 0.02), 0.1 % of entries replaced
+                    by +-U(0.5, 4), seed 1.
+3. ``activation``   bf16 [16384, 7168] Student-t(df=3) * 0.5; 1 % of the
+                    32-element groups zeroed, a disjoint 0.5 % scaled by
+                    2^-120, seed 2.
+4. ``experts``      64 expert weights bf16 [2048, 7168], per-expert std from
+                    U(0.01, 0.05), values N(0, std), seed 3.
+5. ``nvfp4_tensor`` bf16 [8192, 8192] N(0,1) with 0.05 % of entries replaced
+                    by +-U(20, 100), seed 4.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+BF16_MAX_BITS = 0x7F7F            # largest finite bf16 (about 3.39e38)
+
+
+def to_bf16_bits(a: np.ndarray) -> np.ndarray:
+    """float32 array -> uint16 bf16 bit patterns, round-to-nearest-even."""
+    t = torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32))
+    return t.to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+
+
+def bits_of(values, dtype=np.float32) -> np.ndarray:
+    return to_bf16_bits(np.asarray(values, dtype=dtype))
+
+
+# -------------------------------------------------------------- workload 1
+
+# E4M3 rounding ties at scale byte 127 (the 448 entry pins the group's scale):
+# 1.0625 (between 1 and 1.125), 1.1875 (between 1.125 and 1.25), 17 (between
+# 16 and 18), 464 (between 448 and the nonexistent 480), 2^-10 (between 0 and
+# the smallest subnormal), 3 * 2^-10 (between 2^-9 and 2^-8).
+TIE_VALUES = [448.0, 1.0625, 1.1875, 17.0, 464.0, 2.0 ** -10, 3 * 2.0 ** -10,
+              -1.0625, -1.1875, -17.0, -464.0, -(2.0 ** -10), -(3 * 2.0 ** -10)]
+
+
+def planted(seed: int = 0, M: int = 256, N: int = 1024) -> np.ndarray:
+    """Workload 1: N(0,1) with hand-planted groups in group 0 of rows 0-7
+    (needs M >= 8, N >= 32)."""
+    rng = np.random.default_rng(seed)
+    x = to_bf16_bits(rng.standard_normal((M, N), dtype=np.float32))
+    # row 0: all-zero group
+    x[0, :32] = 0
+    # row 1: one outlier 1e4 (bf16 9984)
+    x[1, 5] = bits_of([1e4])[0]
+    # row 2: +-448
+    x[2, 0], x[2, 1] = bits_of([448.0, -448.0])
+    # row 3: 32 bf16 subnormals +-k * 2^-133, k in [1, 127]
+    k = rng.integers(1, 128, size=32).astype(np.uint16)
+    sign = rng.integers(0, 2, size=32).astype(np.uint16) << 15
+    x[3, :32] = k | sign
+    # row 4: one NaN
+    x[4, 7] = 0x7FC0
+    # row 5: one +Inf
+    x[5, 3] = 0x7F80
+    # row 6: E4M3 rounding ties at scale byte 127
+    x[6, :len(TIE_VALUES)] = bits_of(TIE_VALUES)
+    # row 7: largest finite bf16 magnitudes
+    x[7, 0], x[7, 1] = BF16_MAX_BITS, BF16_MAX_BITS | 0x8000
+    return x
+
+
+# -------------------------------------------------------------- workload 2
+
+def linear_weight(seed: int = 1, M: int = 4096, N: int = 4096) -> np.ndarray:
+    rng = np.random.default_rng(seed)
+    w = rng.standard_normal((M, N), dtype=np.float32) * np.float32(0.02)
+    n_out = (M * N) // 1000                      # 0.1 %
+    pos = rng.choice(M * N, size=n_out, replace=False)
+    mag = rng.uniform(0.5, 4.0, size=n_out).astype(np.float32)
+    sgn = np.where(rng.integers(0, 2, size=n_out) == 1, -1.0, 1.0).astype(np.float32)
+    w.reshape(-1)[pos] = mag * sgn
+    return to_bf16_bits(w)
+
+
+# -------------------------------------------------------------- workload 3
+
+def activation(seed: int = 2, M: int = 16384, N: int = 7168) -> np.ndarray:
+    rng = np.random.default_rng(seed)
+    a = (rng.standard_t(3.0, size=(M, N)) * 0.5).astype(np.float32)
+    G = M * N // 32
+    n_zero = G // 100                            # 1 %
+    n_tiny = G // 200                            # 0.5 %
+    idx = rng.choice(G, size=n_zero + n_tiny, replace=False)
+    groups = a.reshape(G, 32)
+    groups[idx[:n_zero]] = 0.0
+    groups[idx[n_zero:]] *= np.float32(2.0 ** -120)
+    return to_bf16_bits(a)
+
+
+# -------------------------------------------------------------- workload 4
+
+def experts(seed: int = 3, E: int = 64, M: int = 2048, N: int = 7168) -> np.ndarray:
+    """Stacked expert weights, uint16 [E, M, N]."""
+    rng = np.random.default_rng(seed)
+    std = rng.uniform(0.01, 0.05, size=E).astype(np.float32)
+    out = np.empty((E, M, N), np.uint16)
+    for e in range(E):
+        out[e] = to_bf16_bits(rng.standard_normal((M, N), dtype=np.float32) * std[e])
+    return out
+
+
+# -------------------------------------------------------------- workload 5
+
+def nvfp4_tensor(seed: int = 4, M: int = 8192, N: int = 8192) -> np.ndarray:
+    rng = np.random.default_rng(seed)
+    x = rng.standard_normal((M, N), dtype=np.float32)
+    n_out = (M * N) * 5 // 10000                 # 0.05 %
+    pos = rng.choice(M * N, size=n_out, replace=False)
+    mag = rng.uniform(20.0, 100.0, size=n_out).astype(np.float32)
+    sgn = np.where(rng.integers(0, 2, size=n_out) == 1, -1.0, 1.0).astype(np.float32)
+    x.reshape(-1)[pos] = mag * sgn
+    return to_bf16_bits(x)
+
+
+WORKLOADS = {
+    "planted": dict(fn=planted, shape=(256, 1024), op="mxfp8 quantize+dequantize"),
+    "linear_weight": dict(fn=linear_weight, shape=(4096, 4096), op="mxfp8 quantize"),
+    "activation": dict(fn=activation, shape=(16384, 7168),
+                       op="mxfp8 quantize (+swizzled scales) + dequantize"),
+    "experts": dict(fn=experts, shape=(64, 2048, 7168), op="grouped mxfp8 quantize"),
+    "nvfp4_tensor": dict(fn=nvfp4_tensor, shape=(8192, 8192), op="nvfp4 quantize"),
+}
