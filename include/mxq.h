@@ -1,0 +1,188 @@
+/*
+ * mxq.h -- C ABI of libmxq.so: block-scaled low-precision quantization of
+ * training tensors on NVIDIA B200 (sm_100a).
+ *
+ *   MXFP8 rowwise: groups of 32 consecutive elements along the last dim share
+ *   one power-of-two E8M0 scale; elements are FP8 E4M3.
+ *   NVFP4 two-level: an fp32 global scale times per-16-element E4M3 block
+ *   scales; elements are FP4 E2M1, packed two per byte.
+ *
+ * Sources (page title, section):
+ *  - "PR #1935 完整报告 -- Use TransformerEngine for MXFP8 quantization",
+ *    实现拆解 item 1 and 关键源码片段: `qweight, scale = mxfp8_quantize(weight)`,
+ *    group size 32, rowwise only, rows zero-padded to a multiple of 32 and
+ *    cropped back, compact non-swizzled (qweight, scale); the scale is stored
+ *    as "<name>_scale_inv", a dequantisation multiplier. 实现拆解 item 4:
+ *    grouped quantization of stacked expert weights (mxfp8_group_quantize).
+ *  - "V4 mxfp4 #1372": power-of-two (float8_e8m0fnu) scales on Blackwell;
+ *    E2M1 stored two per byte (float4_e2m1fn_x2, last dim N//2), with
+ *    N % block_size == 0.
+ *  - "Add FP8, NVFP4, and QARL training and export", review "What looked
+ *    solid": NVFP4 two-level global + FP8-block scaling, "effective =
+ *    block_scale * global_scale", zero blocks guarded.
+ *  - "feat(training): MXFP8 混合精度训练落地", and the same xorl review,
+ *    item 2: failures are visible, never a silent downgrade -- this library
+ *    has no fallback path; every error is a status code.
+ *
+ * Conventions (all entry points):
+ *  - Tensor pointers are DEVICE pointers owned by the caller (for example
+ *    PyTorch tensors); host pointers appear only where stated. The library
+ *    never allocates, frees or synchronizes, and keeps no state between
+ *    calls.
+ *  - Work is enqueued on `stream` (NULL = the legacy default stream) and runs
+ *    asynchronously; outputs are ready when the stream reaches that point.
+ *  - Arguments are checked on the host before anything is enqueued. A call
+ *    that returns anything other than MXQ_OK for an argument error has
+ *    enqueued nothing. MXQ_ERR_CUDA reports a failed launch
+ *    (cudaGetLastError after the launch); the CUDA error string is then
+ *    available from mxq_last_cuda_error() on the calling thread.
+ *  - Shapes are int64_t element counts, row-major; ld_x is the row stride of
+ *    the input in elements (ld_x >= N). M == 0 is valid and does nothing
+ *    (pointers may then be NULL).
+ *  - Alignment: inputs and ld_x * element size must be multiples of 16 bytes;
+ *    qweight / packed / outputs y must be 16-byte aligned; scale arrays have
+ *    no alignment requirement. Otherwise MXQ_ERR_ALIGN.
+ *  - Results are bit-exact functions of the input bits (no atomics on data,
+ *    no order-dependent arithmetic): repeated calls give identical bytes.
+ */
+#ifndef MXQ_H_
+#define MXQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same object as cudaStream_t; declared here so the header needs no CUDA
+ * include. */
+typedef struct CUstream_st* mxq_stream_t;
+
+typedef enum {
+  MXQ_OK = 0,
+  MXQ_ERR_NULL = 1,          /* a required pointer is NULL */
+  MXQ_ERR_SHAPE = 2,         /* negative size, N not a multiple of the group
+                                or block, ld_x < N, or a size limit exceeded */
+  MXQ_ERR_DTYPE = 3,         /* unknown mxq_dtype */
+  MXQ_ERR_ALIGN = 4,         /* pointer or row stride misaligned */
+  MXQ_ERR_WORKSPACE = 5,     /* workspace NULL or smaller than required */
+  MXQ_ERR_CUDA = 6,          /* a CUDA call or launch failed */
+  MXQ_ERR_ARG = 7            /* inconsistent flags or arguments */
+} mxq_status;
+
+typedef enum { MXQ_BF16 = 0, MXQ_FP32 = 1 } mxq_dtype;
+
+#define MXQ_ABI_VERSION 1
+#define MXQ_MXFP8_GROUP 32
+#define MXQ_NVFP4_BLOCK 16
+#define MXQ_GROUPED_MAX_EXPERTS 1024
+#define MXQ_NVFP4_GLOBAL_GIVEN 1u
+
+/* Version of this ABI (MXQ_ABI_VERSION of the built library). */
+int mxq_abi_version(void);
+
+/* Static, human-readable name of a status code. */
+const char* mxq_status_string(int status);
+
+/* Message of the last CUDA error seen by this thread's calls ("" if none). */
+const char* mxq_last_cuda_error(void);
+
+/* ------------------------------------------------------------------ MXFP8 */
+
+/* Bytes of the swizzled scale layout for an [M, S] scale (S = N/32):
+ * ceil(M/128)*128 * ceil(S/4)*4. Returns -1 for negative sizes. */
+int64_t mxq_swizzled_scale_bytes(int64_t M, int64_t S);
+
+/* MXFP8 rowwise quantize ("PR #1935 完整报告 ...", 实现拆解 item 1).
+ *  x        [M, N] bf16 or fp32 (dt), row stride ld_x elements.
+ *  qweight  [M, N] uint8, E4M3 codes, row-major, compact.
+ *  scale    [M, N/32] uint8, E8M0 biased exponents, row-major, compact:
+ *           byte (r, j) covers row r, columns 32j .. 32j+31.
+ *  scale_swz  NULL, or mxq_swizzled_scale_bytes(M, N/32) bytes that receive
+ *           the same scales in the 128x4-tile layout read by block-scaled
+ *           tensor-core MMA (tile (i, j) = rows 128i.., scale columns 4j..,
+ *           at byte (i*ceil(S/4) + j)*512; entry (r, c) inside it at
+ *           (r%32)*16 + ((r%128)/32)*4 + c%4; padding bytes are 0x00).
+ * Per group: amax = max |x| over non-NaN elements; byte = 127 if amax == 0,
+ * 254 if amax is infinite, else clamp(floor(log2 amax) - 8 + 127, 0, 254);
+ * q = E4M3(x * 2^(127 - byte)) rounded to nearest even, |.| > 448 saturating
+ * to 448, NaN -> 0x7F, zero results keeping the sign.
+ * Rows need no padding: groups never cross rows, so the result equals the
+ * pages' pad-to-32-rows-then-crop contract for any M.
+ * Errors: NULL x/qweight/scale (M > 0), N % 32 != 0, ld_x < N, M*N/32 >=
+ * 2^32, misalignment. */
+mxq_status mxfp8_quantize(const void* x, int dt, int64_t M, int64_t N, int64_t ld_x,
+                          uint8_t* qweight, uint8_t* scale, uint8_t* scale_swz,
+                          mxq_stream_t stream);
+
+/* MXFP8 dequantize: y[r, c] = decode_e4m3(q[r, c]) * 2^(scale[r, c/32] - 127)
+ * ("_scale_inv" is the dequantisation multiplier, "PR #1935 完整报告 ...",
+ * 关键源码片段). Computed exactly, then written as fp32 (exact; overflow to
+ * inf only for scale byte 254) or bf16 (round to nearest even, subnormals
+ * kept). NaN codes give 0x7FC0 / 0x7FC00000; scale byte 255 gives NaN.
+ *  qweight [M, N] uint8, scale [M, N/32] uint8, y [M, N] of out_dt. */
+mxq_status mxfp8_dequantize(const uint8_t* qweight, const uint8_t* scale, int64_t M,
+                            int64_t N, void* y, int out_dt, mxq_stream_t stream);
+
+/* Grouped MXFP8 quantize of E expert tensors in one launch ("PR #1935
+ * 完整报告 ...", 实现拆解 item 4).
+ *  xs    HOST array of E device pointers; expert e is a contiguous
+ *        [rows[e], N] tensor of dtype dt (16-byte aligned).
+ *  rows  HOST array of E row counts (>= 0).
+ *  qweight [sum rows, N] and scale [sum rows, N/32]: expert e's rows follow
+ *        expert e-1's, as if the experts were stacked and quantized by
+ *        mxfp8_quantize (identical bytes).
+ * 1 <= E <= MXQ_GROUPED_MAX_EXPERTS. The host arrays are read during the call
+ * only. */
+mxq_status mxfp8_quantize_grouped(int32_t E, const void* const* xs, const int64_t* rows,
+                                  int64_t N, int dt, uint8_t* qweight, uint8_t* scale,
+                                  mxq_stream_t stream);
+
+/* ------------------------------------------------------------------ NVFP4 */
+
+/* Workspace bytes nvfp4_quantize / nvfp4_amax need (per-CTA partial maxima of
+ * the tensor-amax pass); a constant independent of M and N. */
+size_t mxq_nvfp4_workspace_bytes(int64_t M, int64_t N);
+
+/* Tensor amax (max |x| over non-NaN elements, fp32) into *amax (device).
+ * The pass-1 reduction of nvfp4_quantize on its own, for a tensor sharded
+ * across ranks: all-reduce the per-rank amax with MAX, then pass it to
+ * nvfp4_quantize as amax_in. */
+mxq_status nvfp4_amax(const void* x, int dt, int64_t M, int64_t N, int64_t ld_x,
+                      float* amax, void* workspace, size_t ws_bytes, mxq_stream_t stream);
+
+/* NVFP4 two-level quantize ("Add FP8, NVFP4, and QARL training and export",
+ * review; "V4 mxfp4 #1372", review), all arithmetic in fp32:
+ *   g    = A / 2688 (A = tensor amax, 2688 = 448 * 6), written to
+ *          *global_scale; or, with flags & MXQ_NVFP4_GLOBAL_GIVEN, read from
+ *          *global_scale; or, with amax_in != NULL, A read from *amax_in;
+ *   per block of 16: s_b = E4M3(amax_b / (6 g)) (RNE, saturating),
+ *          eff = decode(s_b) * g, q_i = E2M1(x_i / eff) (correctly rounded
+ *          quotient, then RNE, |.| > 6 -> 6, NaN -> +6), or a zero of x_i's
+ *          sign when eff == 0 (zero-block guard); g == 0 gives s_b = 0.
+ *  packed      [M, N/2] uint8: element 2k in the low nibble, 2k+1 high.
+ *  block_scale [M, N/16] uint8 E4M3 codes.
+ *  global_scale device fp32 scalar (out, or in with GLOBAL_GIVEN).
+ *  amax_in     device fp32 scalar or NULL; must be NULL with GLOBAL_GIVEN.
+ *  workspace   device, >= mxq_nvfp4_workspace_bytes; needed only when the
+ *              tensor amax is computed here (no GLOBAL_GIVEN, no amax_in).
+ * N % 16 != 0 -> MXQ_ERR_SHAPE. Non-finite inputs are outside the method's
+ * contract: the same fp32 operations are applied to them. */
+mxq_status nvfp4_quantize(const void* x, int dt, int64_t M, int64_t N, int64_t ld_x,
+                          uint8_t* packed, uint8_t* block_scale, float* global_scale,
+                          const float* amax_in, uint32_t flags, void* workspace,
+                          size_t ws_bytes, mxq_stream_t stream);
+
+/* NVFP4 dequantize: eff = decode_e4m3(s_b) * g and y = decode_e2m1(q) * eff,
+ * both fp32 products, written as fp32 or bf16 (RNE). global_scale is a device
+ * pointer. */
+mxq_status nvfp4_dequantize(const uint8_t* packed, const uint8_t* block_scale,
+                            const float* global_scale, int64_t M, int64_t N, void* y,
+                            int out_dt, mxq_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MXQ_H_ */

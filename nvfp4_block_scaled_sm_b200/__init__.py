@@ -1,0 +1,292 @@
+"""Block-scaled low-precision quantization (MXFP8 / NVFP4) for NVIDIA B200.
+
+Python binding of ``libmxq.so`` (C ABI declared in ``include/mxq.h``). This
+module only marshals arguments: it allocates outputs with torch on the input's
+device, passes raw pointers and the current CUDA stream, and raises on any
+non-zero status. Every step of quantization runs in the library's sm_100a
+kernels; there is no fallback of any kind, and importing this package fails
+if the library has not been built (``python nvfp4_block_scaled_sm_b200/build.py``).
+
+The call ``qweight, scale = mxfp8_quantize(weight)`` follows "PR #1935 完整报告
+-- Use TransformerEngine for MXFP8 quantization" (关键源码片段): compact,
+non-swizzled qweight (E4M3 codes, same shape) and scale (E8M0 bytes, last dim
+N/32), the scale being the dequantization multiplier ("_scale_inv").
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Sequence
+
+import torch
+
+__all__ = [
+    "MxqError", "lib", "library_path",
+    "mxfp8_quantize", "mxfp8_dequantize", "mxfp8_quantize_grouped",
+    "nvfp4_amax", "nvfp4_quantize", "nvfp4_dequantize",
+    "swizzled_scale_bytes", "nvfp4_workspace_bytes",
+    "as_float8_e4m3", "as_float8_e8m0", "as_float4_e2m1x2",
+]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+library_path = os.path.join(_HERE, "libmxq.so")
+
+BF16, FP32 = 0, 1
+NVFP4_GLOBAL_GIVEN = 1
+
+
+class MxqError(RuntimeError):
+    """A libmxq call returned a non-zero status."""
+
+    def __init__(self, fn: str, status: int, message: str):
+        super().__init__(f"{fn}: status {status}: {message}")
+        self.status = status
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(library_path):
+        raise ImportError(
+            f"{library_path} is missing: build it with "
+            "`python nvfp4_block_scaled_sm_b200/build.py` (nvcc, sm_100a)")
+    L = ctypes.CDLL(library_path)
+    vp, i64, i32, u32, sz = (ctypes.c_void_p, ctypes.c_int64, ctypes.c_int,
+                             ctypes.c_uint32, ctypes.c_size_t)
+    L.mxq_abi_version.restype = i32
+    L.mxq_status_string.argtypes, L.mxq_status_string.restype = [i32], ctypes.c_char_p
+    L.mxq_last_cuda_error.restype = ctypes.c_char_p
+    L.mxq_swizzled_scale_bytes.argtypes, L.mxq_swizzled_scale_bytes.restype = [i64, i64], i64
+    L.mxq_nvfp4_workspace_bytes.argtypes, L.mxq_nvfp4_workspace_bytes.restype = [i64, i64], sz
+    L.mxfp8_quantize.argtypes = [vp, i32, i64, i64, i64, vp, vp, vp, vp]
+    L.mxfp8_dequantize.argtypes = [vp, vp, i64, i64, vp, i32, vp]
+    L.mxfp8_quantize_grouped.argtypes = [i32, vp, vp, i64, i32, vp, vp, vp]
+    L.nvfp4_amax.argtypes = [vp, i32, i64, i64, i64, vp, vp, sz, vp]
+    L.nvfp4_quantize.argtypes = [vp, i32, i64, i64, i64, vp, vp, vp, vp, u32, vp, sz, vp]
+    L.nvfp4_dequantize.argtypes = [vp, vp, vp, i64, i64, vp, i32, vp]
+    for f in ("mxfp8_quantize", "mxfp8_dequantize", "mxfp8_quantize_grouped", "nvfp4_amax",
+              "nvfp4_quantize", "nvfp4_dequantize"):
+        getattr(L, f).restype = i32
+    return L
+
+
+lib = _load()
+
+
+def _check(fn: str, status: int):
+    if status != 0:
+        msg = lib.mxq_status_string(status).decode()
+        if status == 6:
+            msg += f" ({lib.mxq_last_cuda_error().decode()})"
+        raise MxqError(fn, status, msg)
+
+
+def _dtype_code(dt: torch.dtype) -> int:
+    if dt == torch.bfloat16:
+        return BF16
+    if dt == torch.float32:
+        return FP32
+    raise TypeError(f"unsupported dtype {dt}: expected torch.bfloat16 or torch.float32")
+
+
+def _require_cuda(*ts: torch.Tensor):
+    for t in ts:
+        if not t.is_cuda:
+            raise ValueError("tensors must live on a CUDA device (no CPU path exists)")
+
+
+def _stream(t: torch.Tensor) -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream(t.device).cuda_stream)
+
+
+def _rows_view(x: torch.Tensor):
+    """(M, N, ld_x) of x seen as M rows of N contiguous elements with row
+    stride ld_x; raises if the leading dims do not collapse to one stride."""
+    if x.dim() == 0:
+        raise ValueError("expected at least one dimension")
+    N = x.shape[-1]
+    if x.dim() == 1:
+        return 1, N, N
+    if N > 1 and x.stride(-1) != 1:
+        raise ValueError("the last dimension must be contiguous")
+    M = 1
+    for s in x.shape[:-1]:
+        M *= s
+    lead = [(s, st) for s, st in zip(x.shape[:-1], x.stride()[:-1]) if s > 1]
+    if not lead:
+        return M, N, N
+    ld = lead[-1][1]
+    for (s0, st0), (s1, st1) in zip(lead[:-1], lead[1:]):
+        if st0 != st1 * s1:
+            raise ValueError("leading dimensions do not collapse to a single row stride")
+    return M, N, ld
+
+
+def _ptr(t: torch.Tensor | None):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def swizzled_scale_bytes(M: int, S: int) -> int:
+    return int(lib.mxq_swizzled_scale_bytes(M, S))
+
+
+def nvfp4_workspace_bytes(M: int = 0, N: int = 0) -> int:
+    return int(lib.mxq_nvfp4_workspace_bytes(M, N))
+
+
+# ------------------------------------------------------------------ MXFP8
+
+def mxfp8_quantize(x: torch.Tensor, *, swizzled: bool = False):
+    """MXFP8 rowwise quantize of a bf16/fp32 CUDA tensor.
+
+    Returns ``(qweight, scale)``: uint8 E4M3 codes shaped like ``x`` and uint8
+    E8M0 bytes shaped ``x.shape[:-1] + (N // 32,)``; with ``swizzled=True`` a
+    third flat uint8 tensor holds the scales in the 128x4-tile layout read by
+    block-scaled tensor-core MMA.
+    """
+    _require_cuda(x)
+    dt = _dtype_code(x.dtype)
+    M, N, ld = _rows_view(x)
+    q = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
+    s = torch.empty((*x.shape[:-1], N // 32), dtype=torch.uint8, device=x.device)
+    swz = None
+    if swizzled:
+        swz = torch.empty(max(swizzled_scale_bytes(M, N // 32), 0), dtype=torch.uint8,
+                          device=x.device)
+    _check("mxfp8_quantize", lib.mxfp8_quantize(_ptr(x), dt, M, N, ld, _ptr(q), _ptr(s),
+                                                _ptr(swz), _stream(x)))
+    return (q, s, swz) if swizzled else (q, s)
+
+
+def mxfp8_dequantize(qweight: torch.Tensor, scale: torch.Tensor,
+                     dtype: torch.dtype = torch.bfloat16) -> torch.Tensor:
+    """decode(q) * 2^(scale - 127), as bf16 (RNE) or fp32 (exact)."""
+    _require_cuda(qweight, scale)
+    if qweight.dtype != torch.uint8 or scale.dtype != torch.uint8:
+        raise TypeError("qweight and scale must be uint8")
+    if not (qweight.is_contiguous() and scale.is_contiguous()):
+        raise ValueError("qweight and scale must be contiguous")
+    N = qweight.shape[-1]
+    M = qweight.numel() // N if N else 0
+    if scale.numel() != M * (N // 32):
+        raise ValueError("scale does not match qweight")
+    y = torch.empty(qweight.shape, dtype=dtype, device=qweight.device)
+    _check("mxfp8_dequantize", lib.mxfp8_dequantize(_ptr(qweight), _ptr(scale), M, N, _ptr(y),
+                                                    _dtype_code(dtype), _stream(qweight)))
+    return y
+
+
+def mxfp8_quantize_grouped(xs: torch.Tensor | Sequence[torch.Tensor]):
+    """Grouped MXFP8 of expert tensors sharing N, in one launch.
+
+    ``xs`` is a stacked [E, M, N] tensor (results [E, M, N] and [E, M, N/32])
+    or a sequence of contiguous [M_e, N] tensors (results concatenated along
+    rows: [sum M_e, N] and [sum M_e, N/32])."""
+    stacked = isinstance(xs, torch.Tensor)
+    parts = list(xs.unbind(0)) if stacked else list(xs)
+    if not parts:
+        raise ValueError("no experts")
+    _require_cuda(*parts)
+    dt = _dtype_code(parts[0].dtype)
+    N = parts[0].shape[-1]
+    rows = []
+    for p in parts:
+        if p.dtype != parts[0].dtype or p.shape[-1] != N or p.device != parts[0].device:
+            raise ValueError("experts must share dtype, device and last dimension")
+        if not p.is_contiguous():
+            raise ValueError("expert tensors must be contiguous")
+        rows.append(p.numel() // N if N else 0)
+    E = len(parts)
+    total = sum(rows)
+    dev = parts[0].device
+    q = torch.empty((total, N), dtype=torch.uint8, device=dev)
+    s = torch.empty((total, N // 32), dtype=torch.uint8, device=dev)
+    ptrs = (ctypes.c_void_p * E)(*[p.data_ptr() for p in parts])
+    rws = (ctypes.c_int64 * E)(*rows)
+    _check("mxfp8_quantize_grouped",
+           lib.mxfp8_quantize_grouped(E, ctypes.cast(ptrs, ctypes.c_void_p),
+                                      ctypes.cast(rws, ctypes.c_void_p), N, dt, _ptr(q), _ptr(s),
+                                      _stream(parts[0])))
+    if stacked:
+        return q.view(xs.shape), s.view(*xs.shape[:-1], N // 32)
+    return q, s
+
+
+# ------------------------------------------------------------------ NVFP4
+
+def nvfp4_amax(x: torch.Tensor, workspace: torch.Tensor | None = None) -> torch.Tensor:
+    """Tensor amax (non-NaN max |x|) as a 0-d fp32 CUDA tensor."""
+    _require_cuda(x)
+    dt = _dtype_code(x.dtype)
+    M, N, ld = _rows_view(x)
+    out = torch.zeros((), dtype=torch.float32, device=x.device)
+    ws = workspace if workspace is not None else torch.empty(
+        nvfp4_workspace_bytes(M, N), dtype=torch.uint8, device=x.device)
+    _check("nvfp4_amax", lib.nvfp4_amax(_ptr(x), dt, M, N, ld, _ptr(out), _ptr(ws),
+                                        ws.numel() * ws.element_size(), _stream(x)))
+    return out
+
+
+def nvfp4_quantize(x: torch.Tensor, global_scale: torch.Tensor | None = None,
+                   amax: torch.Tensor | None = None, workspace: torch.Tensor | None = None):
+    """NVFP4 two-level quantize.
+
+    Returns ``(packed, block_scale, global_scale)``: uint8 [..., N/2] with two
+    E2M1 codes per byte (even element in the low nibble), uint8 E4M3 block
+    scales [..., N/16], and the fp32 global scale as a 0-d CUDA tensor.
+    ``global_scale`` (a given g) or ``amax`` (a given tensor amax, e.g. the
+    all-reduced amax of a sharded tensor) skip the amax pass."""
+    _require_cuda(x)
+    dt = _dtype_code(x.dtype)
+    M, N, ld = _rows_view(x)
+    dev = x.device
+    packed = torch.empty((*x.shape[:-1], N // 2), dtype=torch.uint8, device=dev)
+    bs = torch.empty((*x.shape[:-1], N // 16), dtype=torch.uint8, device=dev)
+    flags = 0
+    if global_scale is not None:
+        if global_scale.dtype != torch.float32 or global_scale.numel() != 1:
+            raise TypeError("global_scale must be a single fp32 value")
+        g = global_scale.to(dev)
+        flags = NVFP4_GLOBAL_GIVEN
+    else:
+        g = torch.empty((), dtype=torch.float32, device=dev)
+    if amax is not None and (amax.dtype != torch.float32 or amax.numel() != 1):
+        raise TypeError("amax must be a single fp32 value")
+    ws = None
+    if global_scale is None and amax is None:
+        ws = workspace if workspace is not None else torch.empty(
+            nvfp4_workspace_bytes(M, N), dtype=torch.uint8, device=dev)
+    _check("nvfp4_quantize",
+           lib.nvfp4_quantize(_ptr(x), dt, M, N, ld, _ptr(packed), _ptr(bs), _ptr(g), _ptr(amax),
+                              flags, _ptr(ws), 0 if ws is None else ws.numel() * ws.element_size(),
+                              _stream(x)))
+    return packed, bs, g
+
+
+def nvfp4_dequantize(packed: torch.Tensor, block_scale: torch.Tensor, global_scale: torch.Tensor,
+                     dtype: torch.dtype = torch.bfloat16) -> torch.Tensor:
+    """E2M1 code * (E4M3 block scale * g), as bf16 (RNE) or fp32."""
+    _require_cuda(packed, block_scale, global_scale)
+    if not (packed.is_contiguous() and block_scale.is_contiguous()):
+        raise ValueError("packed and block_scale must be contiguous")
+    N = packed.shape[-1] * 2
+    M = packed.numel() * 2 // N if N else 0
+    if block_scale.numel() != M * (N // 16):
+        raise ValueError("block_scale does not match packed")
+    y = torch.empty((*packed.shape[:-1], N), dtype=dtype, device=packed.device)
+    _check("nvfp4_dequantize",
+           lib.nvfp4_dequantize(_ptr(packed), _ptr(block_scale), _ptr(global_scale), M, N, _ptr(y),
+                                _dtype_code(dtype), _stream(packed)))
+    return y
+
+
+# ------------------------------------------------------------------ views
+
+def as_float8_e4m3(q: torch.Tensor) -> torch.Tensor:
+    return q.view(torch.float8_e4m3fn)
+
+
+def as_float8_e8m0(s: torch.Tensor) -> torch.Tensor:
+    return s.view(torch.float8_e8m0fnu)
+
+
+def as_float4_e2m1x2(p: torch.Tensor) -> torch.Tensor:
+    return p.view(torch.float4_e2m1fn_x2)

@@ -1,0 +1,234 @@
+// common.cuh -- device and host helpers shared by the libmxq kernels (sm_100a).
+//
+// Numerics: the library is compiled without fast math (-ftz=false,
+// -prec-div=true, -fmad=false), so fp32 multiplies and divides are IEEE
+// round-to-nearest-even with subnormals kept; the power-of-two scaling of the
+// MXFP8 path is therefore exact wherever the E4M3 / E8M0 definitions need it
+// to be (see mxfp8.cu).
+#pragma once
+
+#include <cstdint>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <algorithm>
+#include <cstring>
+
+#include "mxq.h"
+
+namespace mxq {
+
+constexpr int kThreads = 256;          // threads per CTA in every kernel
+constexpr unsigned kFull = 0xffffffffu;
+
+// ------------------------------------------------------------------ host
+
+// Records the message of a failed CUDA call for mxq_last_cuda_error().
+void record_cuda_error(cudaError_t e);
+
+// Status after a launch: MXQ_ERR_CUDA (and the message recorded) if the
+// launch failed.
+mxq_status check_launch();
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline int elem_size(int dt) { return dt == MXQ_BF16 ? 2 : 4; }
+
+inline bool valid_dtype(int dt) { return dt == MXQ_BF16 || dt == MXQ_FP32; }
+
+// n / d for 64-bit n and 32-bit d, as one multiply-high: with
+// magic = ceil(2^64 / d), floor(n * magic / 2^64) == floor(n / d) whenever
+// n * d < 2^64 (the rounding error n * (magic - 2^64/d) / 2^64 stays below
+// 1/d, the smallest possible distance of n/d to the next integer).
+struct FastDiv {
+  uint64_t magic;
+  uint32_t d;
+
+  static FastDiv make(uint32_t div) {
+    FastDiv f;
+    f.d = div;
+    f.magic = (div <= 1) ? 0 : (~0ull / div) + 1;
+    return f;
+  }
+  __device__ __forceinline__ uint64_t div(uint64_t n) const {
+    return d == 1 ? n : __umul64hi(n, magic);
+  }
+};
+
+// ---------------------------------------------------------------- device
+
+// 16-byte read-only load that does not allocate in L1 (streamed once).
+__device__ __forceinline__ uint4 ld_nc_v4(const void* p) {
+  uint4 r;
+  asm("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+      : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+      : "l"(p));
+  return r;
+}
+
+__device__ __forceinline__ uint2 ld_nc_v2(const void* p) {
+  uint2 r;
+  asm("ld.global.nc.L1::no_allocate.v2.u32 {%0, %1}, [%2];" : "=r"(r.x), "=r"(r.y) : "l"(p));
+  return r;
+}
+
+__device__ __forceinline__ uint32_t ld_nc_u32(const void* p) {
+  uint32_t r;
+  asm("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(r) : "l"(p));
+  return r;
+}
+
+__device__ __forceinline__ uint32_t ld_nc_u8(const void* p) {
+  uint32_t r;
+  asm("ld.global.nc.u8 %0, [%1];" : "=r"(r) : "l"(p));
+  return r;
+}
+
+__device__ __forceinline__ void st_v4(void* p, uint4 v) {
+  asm volatile("st.global.v4.u32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(v.x), "r"(v.y),
+               "r"(v.z), "r"(v.w)
+               : "memory");
+}
+
+__device__ __forceinline__ void st_v2(void* p, uint2 v) {
+  asm volatile("st.global.v2.u32 [%0], {%1, %2};" ::"l"(p), "r"(v.x), "r"(v.y) : "memory");
+}
+
+__device__ __forceinline__ void st_u32(void* p, uint32_t v) {
+  asm volatile("st.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ void st_u8(void* p, uint32_t v) {
+  asm volatile("st.global.u8 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// Elementwise max of two bf16 pairs. PTX max ignores a NaN operand (returns
+// the other one), which is the amax rule: NaN never raises the maximum.
+__device__ __forceinline__ uint32_t max_bf16x2(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("max.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+
+// fp32 value of the low / high bf16 of a packed pair (exact).
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+// Two fp32 -> E4M3 codes (round to nearest even, |v| > 448 -> 448, NaN ->
+// NaN); `lo` lands in the low byte.
+__device__ __forceinline__ uint32_t cvt_e4m3x2(float lo, float hi) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// Two E4M3 codes (low byte first) -> f16x2 (exact: E4M3 is a subset of f16).
+__device__ __forceinline__ uint32_t cvt_f16x2_from_e4m3x2(uint32_t codes) {
+  uint32_t r;
+  uint16_t c = static_cast<uint16_t>(codes);
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r) : "h"(c));
+  return r;
+}
+
+// fp32 values of a packed f16 pair (exact).
+__device__ __forceinline__ float2 f16x2_to_f32x2(uint32_t h) {
+  __half2 v;
+  memcpy(&v, &h, 4);
+  return __half22float2(v);
+}
+
+// Two fp32 -> packed bf16 pair, round to nearest even (lo in the low half).
+__device__ __forceinline__ uint32_t cvt_bf16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// Two fp32 -> E2M1 codes in one byte (round to nearest even, |u| > 6 -> 6);
+// `lo` lands in the low nibble.
+__device__ __forceinline__ uint32_t cvt_e2m1x2(float lo, float hi) {
+  uint32_t r;
+  asm("{ .reg .b8 t; cvt.rn.satfinite.e2m1x2.f32 t, %1, %2; cvt.u32.u8 %0, t; }"
+      : "=r"(r)
+      : "f"(hi), "f"(lo));
+  return r;
+}
+
+// One byte holding two E2M1 codes (low nibble first) -> f16x2 (exact).
+__device__ __forceinline__ uint32_t cvt_f16x2_from_e2m1x2(uint32_t byte) {
+  uint32_t r;
+  asm("{ .reg .b8 t; cvt.u8.u32 t, %1; cvt.rn.f16x2.e2m1x2 %0, t; }" : "=r"(r) : "r"(byte));
+  return r;
+}
+
+// Per-byte flag (0x80) for the E4M3 NaN codes 0x7F / 0xFF in a word of four
+// codes. Bytes are at most 0x7F after the mask, so the +1 never carries.
+__device__ __forceinline__ uint32_t e4m3_nan_bytes(uint32_t w) {
+  return ((w & 0x7f7f7f7fu) + 0x01010101u) & 0x80808080u;
+}
+
+// ------------------------------------------------------ 8-element lanes
+
+// Eight consecutive input elements held by one lane: one 16-byte load of
+// bf16 bit patterns, or two of fp32.
+template <typename InT>
+struct In8;
+
+template <>
+struct In8<uint16_t> {
+  uint32_t w[4];
+  __device__ __forceinline__ void load(const uint16_t* p) {
+    const uint4 t = ld_nc_v4(p);
+    w[0] = t.x; w[1] = t.y; w[2] = t.z; w[3] = t.w;
+  }
+  __device__ __forceinline__ void zero() { w[0] = w[1] = w[2] = w[3] = 0; }
+  // max |x| over the non-NaN elements (NaN if all are NaN)
+  __device__ __forceinline__ float absmax() const {
+    uint32_t m = max_bf16x2(w[0] & 0x7fff7fffu, w[1] & 0x7fff7fffu);
+    m = max_bf16x2(m, w[2] & 0x7fff7fffu);
+    m = max_bf16x2(m, w[3] & 0x7fff7fffu);
+    return fmaxf(bf16_lo(m), bf16_hi(m));
+  }
+  __device__ __forceinline__ float operator[](int i) const {
+    return (i & 1) ? bf16_hi(w[i >> 1]) : bf16_lo(w[i >> 1]);
+  }
+};
+
+template <>
+struct In8<float> {
+  uint32_t w[8];
+  __device__ __forceinline__ void load(const float* p) {
+    const uint4 a = ld_nc_v4(p), b = ld_nc_v4(p + 4);
+    w[0] = a.x; w[1] = a.y; w[2] = a.z; w[3] = a.w;
+    w[4] = b.x; w[5] = b.y; w[6] = b.z; w[7] = b.w;
+  }
+  __device__ __forceinline__ void zero() {
+#pragma unroll
+    for (int i = 0; i < 8; i++) w[i] = 0;
+  }
+  __device__ __forceinline__ float absmax() const {
+    float m = fabsf(__uint_as_float(w[0]));
+#pragma unroll
+    for (int i = 1; i < 8; i++) m = fmaxf(m, fabsf(__uint_as_float(w[i])));
+    return m;
+  }
+  __device__ __forceinline__ float operator[](int i) const { return __uint_as_float(w[i]); }
+};
+
+// ----------------------------------------------------------- block reduce
+
+// Max over the CTA of a non-negative float (NaN ignored); every thread gets
+// the result. `red` is kThreads/32 floats of shared memory.
+__device__ __forceinline__ float block_max(float v, float* red) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(kFull, v, o));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  __syncthreads();
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  float r = red[0];
+#pragma unroll
+  for (int w = 1; w < kThreads / 32; w++) r = fmaxf(r, red[w]);
+  return r;
+}
+
+}  // namespace mxq

@@ -1,0 +1,159 @@
+"""The C-ABI library loads without a GPU, exports every function that
+include/mxq.h declares, and rejects bad arguments on the host with the
+documented status before touching CUDA (no call below launches anything)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import nvfp4_block_scaled_sm_b200 as mxq
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "mxq.h")
+
+OK, NULL, SHAPE, DTYPE, ALIGN, WORKSPACE, CUDA, ARG = range(8)
+A = 0x10000          # a 16-byte-aligned fake device address (never dereferenced)
+
+# The argument checks below pass fake addresses: they only run where no GPU
+# is visible, so a check that wrongly let a call through could never launch
+# a kernel on real memory.
+if __import__("torch").cuda.is_available():
+    pytest.skip("host-validation tests with fake addresses run without a GPU only",
+                allow_module_level=True)
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b([a-z][a-z0-9_]*)\s*\(", text)) - {"sizeof"})
+
+
+def test_header_declares_expected_entry_points():
+    names = declared_functions()
+    for f in ("mxfp8_quantize", "mxfp8_dequantize", "mxfp8_quantize_grouped", "nvfp4_quantize",
+              "nvfp4_dequantize", "nvfp4_amax", "mxq_abi_version", "mxq_status_string"):
+        assert f in names
+
+
+def test_library_exports_every_declared_symbol():
+    raw = ctypes.CDLL(mxq.library_path)
+    missing = [f for f in declared_functions() if not hasattr(raw, f)]
+    assert not missing, missing
+
+
+def test_version_and_strings():
+    assert mxq.lib.mxq_abi_version() == 1
+    for s in range(8):
+        assert mxq.lib.mxq_status_string(s)
+    assert mxq.lib.mxq_status_string(99) == b"unknown status"
+
+
+def test_size_helpers():
+    assert mxq.swizzled_scale_bytes(16384, 224) == 16384 * 224
+    assert mxq.swizzled_scale_bytes(130, 7) == 256 * 8
+    assert mxq.swizzled_scale_bytes(1, 1) == 128 * 4
+    assert mxq.swizzled_scale_bytes(-1, 4) == -1
+    assert mxq.nvfp4_workspace_bytes(8192, 8192) >= 4
+
+
+def test_mxfp8_quantize_validation():
+    L = mxq.lib
+    assert L.mxfp8_quantize(A, 2, 4, 64, 64, A, A, None, None) == DTYPE
+    assert L.mxfp8_quantize(A, 0, 4, 48, 48, A, A, None, None) == SHAPE
+    assert L.mxfp8_quantize(A, 0, -1, 64, 64, A, A, None, None) == SHAPE
+    assert L.mxfp8_quantize(A, 0, 4, 64, 32, A, A, None, None) == SHAPE
+    assert L.mxfp8_quantize(None, 0, 4, 64, 64, A, A, None, None) == NULL
+    assert L.mxfp8_quantize(A, 0, 4, 64, 64, None, A, None, None) == NULL
+    assert L.mxfp8_quantize(A, 0, 4, 64, 64, A, None, None, None) == NULL
+    assert L.mxfp8_quantize(A + 2, 0, 4, 64, 64, A, A, None, None) == ALIGN
+    assert L.mxfp8_quantize(A, 0, 4, 64, 68, A, A, None, None) == ALIGN
+    assert L.mxfp8_quantize(A, 0, 4, 64, 64, A + 8, A, None, None) == ALIGN
+    # empty inputs succeed without touching any pointer
+    assert L.mxfp8_quantize(None, 0, 0, 64, 64, None, None, None, None) == OK
+    assert L.mxfp8_quantize(None, 1, 5, 0, 0, None, None, None, None) == OK
+
+
+def test_mxfp8_dequantize_validation():
+    L = mxq.lib
+    assert L.mxfp8_dequantize(A, A, 4, 64, A, 7, None) == DTYPE
+    assert L.mxfp8_dequantize(A, A, 4, 40, A, 0, None) == SHAPE
+    assert L.mxfp8_dequantize(None, A, 4, 64, A, 0, None) == NULL
+    assert L.mxfp8_dequantize(A, A, 4, 64, None, 0, None) == NULL
+    assert L.mxfp8_dequantize(A + 4, A, 4, 64, A, 0, None) == ALIGN
+    assert L.mxfp8_dequantize(A, A, 4, 64, A + 2, 1, None) == ALIGN
+    assert L.mxfp8_dequantize(None, None, 0, 64, None, 0, None) == OK
+
+
+def test_grouped_validation():
+    L = mxq.lib
+    ptrs = (ctypes.c_void_p * 3)(A, A, A)
+    rows = (ctypes.c_int64 * 3)(4, 0, 2)
+    P, R = ctypes.cast(ptrs, ctypes.c_void_p), ctypes.cast(rows, ctypes.c_void_p)
+    assert L.mxfp8_quantize_grouped(0, P, R, 64, 0, A, A, None) == SHAPE
+    assert L.mxfp8_quantize_grouped(1025, P, R, 64, 0, A, A, None) == SHAPE
+    assert L.mxfp8_quantize_grouped(3, P, R, 48, 0, A, A, None) == SHAPE
+    assert L.mxfp8_quantize_grouped(3, P, R, 64, 5, A, A, None) == DTYPE
+    assert L.mxfp8_quantize_grouped(3, None, R, 64, 0, A, A, None) == NULL
+    assert L.mxfp8_quantize_grouped(3, P, R, 64, 0, None, A, None) == NULL
+    assert L.mxfp8_quantize_grouped(3, P, R, 64, 0, A + 1, A, None) == ALIGN
+    bad_rows = (ctypes.c_int64 * 3)(4, -1, 2)
+    assert L.mxfp8_quantize_grouped(3, P, ctypes.cast(bad_rows, ctypes.c_void_p), 64, 0, A, A,
+                                    None) == SHAPE
+    mis = (ctypes.c_void_p * 3)(A, A, A + 8)
+    assert L.mxfp8_quantize_grouped(3, ctypes.cast(mis, ctypes.c_void_p), R, 64, 0, A, A,
+                                    None) == ALIGN
+    zero_rows = (ctypes.c_int64 * 3)(0, 0, 0)
+    assert L.mxfp8_quantize_grouped(3, P, ctypes.cast(zero_rows, ctypes.c_void_p), 64, 0, None,
+                                    None, None) == OK
+
+
+def test_grouped_null_pointer_only_matters_for_nonempty_expert():
+    L = mxq.lib
+    rows = (ctypes.c_int64 * 2)(4, 0)
+    ptrs = (ctypes.c_void_p * 2)(None, A)
+    assert L.mxfp8_quantize_grouped(2, ctypes.cast(ptrs, ctypes.c_void_p),
+                                    ctypes.cast(rows, ctypes.c_void_p), 64, 0, A, A, None) == NULL
+
+
+def test_nvfp4_validation():
+    L = mxq.lib
+    ws = mxq.nvfp4_workspace_bytes()
+    assert L.nvfp4_quantize(A, 0, 4, 64, 64, A, A, A, None, 2, A, ws, None) == ARG
+    assert L.nvfp4_quantize(A, 0, 4, 64, 64, A, A, A, A, 1, A, ws, None) == ARG
+    assert L.nvfp4_quantize(A, 3, 4, 64, 64, A, A, A, None, 0, A, ws, None) == DTYPE
+    assert L.nvfp4_quantize(A, 0, 4, 40, 40, A, A, A, None, 0, A, ws, None) == SHAPE
+    assert L.nvfp4_quantize(A, 0, 4, 64, 48, A, A, A, None, 0, A, ws, None) == SHAPE
+    assert L.nvfp4_quantize(None, 0, 4, 64, 64, A, A, A, None, 0, A, ws, None) == NULL
+    assert L.nvfp4_quantize(A, 0, 4, 64, 64, A, A, None, None, 0, A, ws, None) == NULL
+    assert L.nvfp4_quantize(A, 0, 4, 64, 64, A + 4, A, A, None, 0, A, ws, None) == ALIGN
+    assert L.nvfp4_quantize(A, 1, 4, 64, 66, A, A, A, None, 0, A, ws, None) == ALIGN
+    assert L.nvfp4_quantize(A, 0, 4, 64, 64, A, A, A, None, 0, None, ws, None) == WORKSPACE
+    assert L.nvfp4_quantize(A, 0, 4, 64, 64, A, A, A, None, 0, A, ws - 4, None) == WORKSPACE
+    assert L.nvfp4_quantize(None, 0, 0, 64, 64, None, None, None, None, 0, None, 0, None) == OK
+    assert L.nvfp4_amax(A, 0, 4, 64, 64, None, A, ws, None) == NULL
+    assert L.nvfp4_amax(A, 0, 4, 64, 64, A, A, 16, None) == WORKSPACE
+    assert L.nvfp4_dequantize(A, A, A, 4, 40, A, 0, None) == SHAPE
+    assert L.nvfp4_dequantize(A, A, None, 4, 64, A, 0, None) == NULL
+    assert L.nvfp4_dequantize(A, A, A, 4, 64, A + 2, 0, None) == ALIGN
+    assert L.nvfp4_dequantize(A, A, A, 4, 64, A, 9, None) == DTYPE
+
+
+def test_python_binding_rejects_cpu_tensors():
+    import torch
+    with pytest.raises(ValueError):
+        mxq.mxfp8_quantize(torch.zeros(4, 64, dtype=torch.bfloat16))
+    with pytest.raises(ValueError):
+        mxq.nvfp4_quantize(torch.zeros(4, 64, dtype=torch.bfloat16))
+
+
+def test_rows_view():
+    import torch
+    x = torch.zeros(6, 10, 64)
+    assert mxq._rows_view(x) == (60, 64, 64)
+    assert mxq._rows_view(torch.zeros(8, 96)[:, :64]) == (8, 64, 96)
+    assert mxq._rows_view(torch.zeros(4, 1, 96)[:, :, :64]) == (4, 64, 96)
+    with pytest.raises(ValueError):
+        mxq._rows_view(torch.zeros(4, 6, 96)[:, :, :64].transpose(0, 1))
+    with pytest.raises(ValueError):
+        mxq._rows_view(torch.zeros(64, 4).t())

@@ -138,3 +138,92 @@ WORKLOADS = {
     "experts": dict(fn=experts, shape=(64, 2048, 7168), op="grouped mxfp8 quantize"),
     "nvfp4_tensor": dict(fn=nvfp4_tensor, shape=(8192, 8192), op="nvfp4 quantize"),
 }
+
+
+# ------------------------------------------------------ structured sweeps
+
+def mxfp8_every_value_every_scale() -> np.ndarray:
+    """bf16 [M, 1024] covering every (bf16 value, E8M0 byte) pair that can
+    occur together: for each byte b in 0..246 the groups start with
+    1.5 * 2^(b - 119) (amax with floor(log2) = b - 119, i.e. byte b) followed
+    by every bf16 pattern of magnitude below 2^(b - 118) and every NaN
+    pattern; for byte 254 the groups start with +inf and hold every pattern.
+    Groups are 1 planted + 31 swept elements; the tail is zero-filled."""
+    allp = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    mag_e = (allp >> 7) & 0xFF                       # exponent field
+    is_nan = ((allp & 0x7FFF) > 0x7F80)
+    groups = []
+    for b in range(0, 247):
+        lead = to_bf16_bits(np.array([1.5 * 2.0 ** (b - 119)], np.float32))[0]
+        vals = allp[((mag_e <= b + 8) & ~is_nan) | is_nan]
+        n = (len(vals) + 30) // 31
+        g = np.zeros((n, 32), np.uint16)
+        g[:, 0] = lead
+        flat = np.zeros(n * 31, np.uint16)
+        flat[:len(vals)] = vals
+        g[:, 1:] = flat.reshape(n, 31)
+        groups.append(g)
+    n = (65536 + 30) // 31
+    g = np.zeros((n, 32), np.uint16)
+    g[:, 0] = 0x7F80
+    flat = np.zeros(n * 31, np.uint16)
+    flat[:65536] = allp
+    g[:, 1:] = flat.reshape(n, 31)
+    groups.append(g)
+    allg = np.concatenate(groups, 0)
+    per_row = 32
+    rows = (allg.shape[0] + per_row - 1) // per_row
+    out = np.zeros((rows * per_row, 32), np.uint16)
+    out[:allg.shape[0]] = allg
+    return out.reshape(rows, per_row * 32)
+
+
+def mxfp8_all_code_scale_pairs():
+    """(qweight [256, 8192], scale [256, 256]): row r carries scale byte r on
+    every group and the 256 E4M3 codes repeated, so every (code, byte) pair
+    is dequantized."""
+    q = np.tile(np.arange(256, dtype=np.uint8), (256, 32))
+    s = np.repeat(np.arange(256, dtype=np.uint8)[:, None], 256, axis=1)
+    return q, s
+
+
+def nvfp4_e2m1_sweep_fp32() -> np.ndarray:
+    """fp32 [M, 256] blocks of 16 whose first element is 6 (with a global
+    scale of 1 every block gets scale 1.0 and eff = 1) and whose other 15
+    elements sweep fp32 values in [-6, 6]: every 64th bit pattern in [0, 6]
+    plus +-512 ulp around each E2M1 value and midpoint, both signs."""
+    top = np.float32(6.0).view(np.int32)
+    dense = np.arange(0, top + 1, 64, dtype=np.int32)
+    pts = np.array([0, 0.25, 0.5, 0.75, 1, 1.25, 1.5, 1.75, 2, 2.5, 3, 3.5, 4, 5, 6], np.float32)
+    near = (pts.view(np.int32)[:, None] + np.arange(-512, 513, dtype=np.int32)[None, :]).reshape(-1)
+    near = near[(near >= 0) & (near <= top)]
+    v = np.concatenate([dense, near]).view(np.float32)
+    v = np.concatenate([v, -v])
+    nb = (v.size + 14) // 15
+    blocks = np.zeros((nb, 16), np.float32)
+    blocks[:, 0] = 6.0
+    flat = np.zeros(nb * 15, np.float32)
+    flat[:v.size] = v
+    blocks[:, 1:] = flat.reshape(nb, 15)
+    rows = (nb + 15) // 16
+    out = np.zeros((rows * 16, 16), np.float32)
+    out[:nb] = blocks
+    return out.reshape(rows, 256)
+
+
+def nvfp4_block_scale_sweep_fp32(seed: int = 5) -> np.ndarray:
+    """fp32 [M, 256] blocks whose amax sweeps the E4M3 block-scale range
+    (log-uniform over [2^-14, 2^12] plus values near 6 * every E4M3 value and
+    midpoint), the other elements uniform in [-amax, amax]."""
+    rng = np.random.default_rng(seed)
+    from_log = np.exp2(rng.uniform(-14, 12, 40000)).astype(np.float32)
+    codes = np.array([m * 2.0 ** e for e in range(-9, 9) for m in (1, 1.0625, 1.125, 1.1875, 1.25,
+                      1.375, 1.5, 1.625, 1.75, 1.875)], np.float32) * np.float32(6.0)
+    near = (codes.view(np.int32)[:, None] + np.arange(-3, 4, dtype=np.int32)[None, :]).reshape(-1)
+    amax = np.concatenate([from_log, near.view(np.float32)])
+    nb = amax.size
+    rows = (nb + 15) // 16
+    blocks = (rng.uniform(-1, 1, (rows * 16, 16)).astype(np.float32)
+              * np.resize(amax, rows * 16)[:, None])
+    blocks[:, 0] = np.resize(amax, rows * 16)
+    return blocks.reshape(rows, 256)
