@@ -12,6 +12,7 @@
 #include <cuda_runtime.h>
 #include <algorithm>
 #include <cstring>
+#include <utility>
 
 #include "mxq.h"
 
@@ -28,6 +29,16 @@ void record_cuda_error(cudaError_t e);
 // Status after a launch: MXQ_ERR_CUDA (and the message recorded) if the
 // launch failed.
 mxq_status check_launch();
+
+// Status of a launch call followed by the launch's own error state.
+inline mxq_status launched(cudaError_t e) {
+  if (e != cudaSuccess) {
+    record_cuda_error(e);
+    cudaGetLastError();
+    return MXQ_ERR_CUDA;
+  }
+  return check_launch();
+}
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -106,6 +117,41 @@ __device__ __forceinline__ void st_u8(void* p, uint32_t v) {
 __device__ __forceinline__ uint32_t max_bf16x2(uint32_t a, uint32_t b) {
   uint32_t r;
   asm("max.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+
+// Elementwise max of |a| and |b| for two bf16 pairs (the sign of each result
+// half is the xor of the input signs and is masked off by the caller); a NaN
+// operand is ignored.
+__device__ __forceinline__ uint32_t absmax_bf16x2(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+
+// 32-byte read-only load (sm_100 256-bit global load); p must be 32-byte aligned.
+__device__ __forceinline__ void ld_nc_v8(const void* p, uint32_t (&w)[8]) {
+  asm("ld.global.nc.L1::no_allocate.v8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+      : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3]), "=r"(w[4]), "=r"(w[5]), "=r"(w[6]),
+        "=r"(w[7])
+      : "l"(p));
+}
+
+// 32-byte store (sm_100 256-bit global store); p must be 32-byte aligned.
+__device__ __forceinline__ void st_v8(void* p, const uint32_t (&w)[8]) {
+  asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "r"(w[0]),
+               "r"(w[1]), "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7])
+               : "memory");
+}
+
+// Two independent IEEE fp32 products (a0*b, a1*b) in one packed instruction
+// (sm_100 mul.rn.f32x2; subnormals kept).
+__device__ __forceinline__ float2 mul2(float a0, float a1, float b) {
+  float2 r;
+  asm("{ .reg .b64 a, m, d; mov.b64 a, {%2, %3}; mov.b64 m, {%4, %4};\n\t"
+      "mul.rn.f32x2 d, a, m; mov.b64 {%0, %1}, d; }"
+      : "=f"(r.x), "=f"(r.y)
+      : "f"(a0), "f"(a1), "f"(b));
   return r;
 }
 
@@ -213,6 +259,115 @@ struct In8<float> {
   }
   __device__ __forceinline__ float operator[](int i) const { return __uint_as_float(w[i]); }
 };
+
+// Sixteen consecutive input elements held by one lane: 32 bytes of bf16 or 64
+// of fp32, read with 256-bit loads when V8 (32-byte aligned) or 128-bit ones.
+template <typename InT>
+struct In16;
+
+template <>
+struct In16<uint16_t> {
+  uint32_t w[8];
+  template <bool V8>
+  __device__ __forceinline__ void load(const uint16_t* p) {
+    if constexpr (V8) {
+      ld_nc_v8(p, w);
+    } else {
+      const uint4 a = ld_nc_v4(p), b = ld_nc_v4(p + 8);
+      w[0] = a.x; w[1] = a.y; w[2] = a.z; w[3] = a.w;
+      w[4] = b.x; w[5] = b.y; w[6] = b.z; w[7] = b.w;
+    }
+  }
+  __device__ __forceinline__ void zero() {
+#pragma unroll
+    for (int i = 0; i < 8; i++) w[i] = 0;
+  }
+  // max |x| over the non-NaN elements (NaN if all are NaN)
+  __device__ __forceinline__ float absmax() const {
+    uint32_t m = absmax_bf16x2(w[0], w[1]);
+    const uint32_t m2 = absmax_bf16x2(w[2], w[3]);
+    const uint32_t m3 = absmax_bf16x2(w[4], w[5]);
+    const uint32_t m4 = absmax_bf16x2(w[6], w[7]);
+    m = absmax_bf16x2(absmax_bf16x2(m, m2), absmax_bf16x2(m3, m4)) & 0x7fff7fffu;
+    return fmaxf(bf16_lo(m), bf16_hi(m));
+  }
+  __device__ __forceinline__ float lo(int k) const { return bf16_lo(w[k]); }  // element 2k
+  __device__ __forceinline__ float hi(int k) const { return bf16_hi(w[k]); }  // element 2k+1
+  __device__ __forceinline__ uint32_t signs() const {  // bit i = sign of element i
+    uint32_t r = 0;
+#pragma unroll
+    for (int k = 0; k < 8; k++) r |= ((w[k] >> 15) & 1u) << (2 * k) | (w[k] >> 31) << (2 * k + 1);
+    return r;
+  }
+};
+
+template <>
+struct In16<float> {
+  uint32_t w[16];
+  template <bool V8>
+  __device__ __forceinline__ void load(const float* p) {
+    if constexpr (V8) {
+      uint32_t (&a)[8] = *reinterpret_cast<uint32_t(*)[8]>(&w[0]);
+      uint32_t (&b)[8] = *reinterpret_cast<uint32_t(*)[8]>(&w[8]);
+      ld_nc_v8(p, a);
+      ld_nc_v8(p + 8, b);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 4; i++) {
+        const uint4 t = ld_nc_v4(p + 4 * i);
+        w[4 * i] = t.x; w[4 * i + 1] = t.y; w[4 * i + 2] = t.z; w[4 * i + 3] = t.w;
+      }
+    }
+  }
+  __device__ __forceinline__ void zero() {
+#pragma unroll
+    for (int i = 0; i < 16; i++) w[i] = 0;
+  }
+  __device__ __forceinline__ float absmax() const {
+    float m = fabsf(__uint_as_float(w[0]));
+#pragma unroll
+    for (int i = 1; i < 16; i++) m = fmaxf(m, fabsf(__uint_as_float(w[i])));
+    return m;
+  }
+  __device__ __forceinline__ float lo(int k) const { return __uint_as_float(w[2 * k]); }
+  __device__ __forceinline__ float hi(int k) const { return __uint_as_float(w[2 * k + 1]); }
+  __device__ __forceinline__ uint32_t signs() const {
+    uint32_t r = 0;
+#pragma unroll
+    for (int i = 0; i < 16; i++) r |= (w[i] >> 31) << i;
+    return r;
+  }
+};
+
+// --------------------------------------------- programmatic dependent launch
+
+// Every kernel starts with this: wait until the grids it depends on (earlier
+// work in the stream) have completed and their writes are visible, before any
+// global memory access, then allow the next grid in the stream to be
+// scheduled. When the kernel was launched without programmatic serialization
+// both instructions are no-ops.
+__device__ __forceinline__ void pdl_enter() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Launches `kernel` with programmatic stream serialization, so its launch and
+// CTA scheduling overlap the tail of the previous grid in the stream.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), uint32_t grid, cudaStream_t stream,
+                              Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 // ----------------------------------------------------------- block reduce
 

@@ -12,9 +12,20 @@
 //                                          (|u| > 6 -> 6, NaN -> +6), or a
 //                                          sign-kept zero when eff == 0
 //   packed byte k of a row = q[2k] | q[2k+1] << 4.
-// Divisions use __fdiv_rn (IEEE), products __fmul_rn: the kernel performs the
-// same fp32 operations in the same order as the definition, so every code is
-// bit-identical to it.
+// g, s and eff use IEEE division / multiplication (__fdiv_rn, __fmul_rn).
+//
+// E2M1 codes without a division per element. The code is a monotone step
+// function of the correctly rounded quotient f = fl(x / eff). With
+// r = fl(1 / eff) (IEEE reciprocal, once per block), the two products
+// lo = fl(x * fl(r * (1 - 2^-20))) and hi = fl(x * fl(r * (1 + 2^-20)))
+// bracket f strictly: three roundings move a product by at most 3 * 2^-24
+// relative, far inside the 2^-20 margin, while f itself lies within 2^-24 of
+// x / eff. So whenever E2M1(lo) == E2M1(hi), that code is E2M1(f) (a tie of
+// f on a midpoint would put lo and hi on opposite sides of it). Products
+// that fall below the fp32 normal range are far below the first midpoint
+// (0.25), products that overflow are far above 6, so the bracket argument
+// only needs eff to be a finite normal number. Otherwise, and for the rare
+// lane whose bracket straddles a midpoint, the lane divides exactly.
 //
 // Passes: the tensor amax must be known before any block can be quantized,
 // so a first kernel reduces |x| into per-CTA partial maxima (workspace), and
@@ -23,18 +34,19 @@
 // so its first reads hit the tail of the tensor that the amax pass left in
 // the 126 MB L2.
 //
-// Work split of the block pass: a lane owns 8 consecutive elements, two lanes
-// one block of 16, a warp 16 consecutive blocks per step (512 contiguous bytes
-// of bf16 in, 128 bytes of packed codes out) and kSteps steps.
+// Work split of the block pass: a lane owns one block (16 elements, one
+// 256-bit load of bf16), writes 8 packed bytes and one scale byte, so a warp
+// reads 1 KiB and writes 256 + 32 contiguous bytes per step.
 #include "common.cuh"
 
 namespace mxq {
 namespace {
 
 constexpr int kMaxPartials = 2048;  // CTAs of the amax pass (workspace floats)
-constexpr int kAmaxSteps = 4;       // 8-element chunks per thread per iteration
-constexpr int kSteps = 4;
-constexpr int kBlocksPerWarp = 16 * kSteps;
+constexpr int kAmaxSteps = 2;       // 16-element bf16 chunks per thread per iteration (fp32: 1)
+constexpr int kAmaxCtasPerSm = 8;   // one resident wave: grid = SMs x 8
+constexpr int kSteps = 2;
+constexpr int kBlocksPerWarp = 32 * kSteps;
 constexpr int kBlocksPerTile = kBlocksPerWarp * (kThreads / 32);
 
 enum GMode { kFromPartials = 0, kGiven = 1, kFromAmax = 2 };
@@ -43,36 +55,45 @@ __device__ __forceinline__ float decode_e4m3(uint32_t code) {
   return f16x2_to_f32x2(cvt_f16x2_from_e4m3x2(code)).x;
 }
 
+__device__ __forceinline__ bool is_finite_normal(float v) {
+  const uint32_t e = __float_as_uint(v) & 0x7f800000u;
+  return e != 0 && e != 0x7f800000u;
+}
+
+inline bool aligned32(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 31u) == 0; }
+
 // ------------------------------------------------------------- amax pass
 
-template <typename InT, bool STRIDED>
-__global__ void __launch_bounds__(kThreads)
+template <typename InT, bool V8, bool STRIDED>
+__global__ void __launch_bounds__(kThreads, kAmaxCtasPerSm)
 nvfp4_amax_kernel(const InT* __restrict__ x, uint64_t nchunks, uint32_t cpr, FastDiv rowdiv,
                   int64_t ld, float* __restrict__ partials) {
+  pdl_enter();
+  constexpr int steps = sizeof(InT) == 2 ? kAmaxSteps : 1;  // 64 bytes in flight per thread
   __shared__ float red[kThreads / 32];
   float m = 0.0f;
-  const uint64_t per_iter = uint64_t(gridDim.x) * kThreads * kAmaxSteps;
-  for (uint64_t base = uint64_t(blockIdx.x) * kThreads * kAmaxSteps; base < nchunks;
+  const uint64_t per_iter = uint64_t(gridDim.x) * kThreads * steps;
+  for (uint64_t base = uint64_t(blockIdx.x) * kThreads * steps; base < nchunks;
        base += per_iter) {
-    In8<InT> v[kAmaxSteps];
+    In16<InT> v[steps];
 #pragma unroll
-    for (int u = 0; u < kAmaxSteps; u++) {
+    for (int u = 0; u < steps; u++) {
       const uint64_t c = base + uint64_t(u) * kThreads + threadIdx.x;
       if (c < nchunks) {
         uint64_t off;
         if constexpr (STRIDED) {
           const uint64_t r = rowdiv.div(c);
-          off = r * uint64_t(ld) + (c - r * cpr) * 8;
+          off = r * uint64_t(ld) + (c - r * cpr) * 16;
         } else {
-          off = c * 8;
+          off = c * 16;
         }
-        v[u].load(x + off);
+        v[u].template load<V8>(x + off);
       } else {
         v[u].zero();
       }
     }
 #pragma unroll
-    for (int u = 0; u < kAmaxSteps; u++) m = fmaxf(m, v[u].absmax());
+    for (int u = 0; u < steps; u++) m = fmaxf(m, v[u].absmax());
   }
   m = block_max(m, red);
   if (threadIdx.x == 0) partials[blockIdx.x] = m;
@@ -81,6 +102,7 @@ nvfp4_amax_kernel(const InT* __restrict__ x, uint64_t nchunks, uint32_t cpr, Fas
 // One CTA: max over the partials into *amax.
 __global__ void __launch_bounds__(kThreads)
 nvfp4_amax_finalize_kernel(const float* __restrict__ partials, uint32_t n, float* amax) {
+  pdl_enter();
   __shared__ float red[kThreads / 32];
   float m = 0.0f;
   for (uint32_t i = threadIdx.x; i < n; i += kThreads) m = fmaxf(m, partials[i]);
@@ -105,31 +127,73 @@ struct QuantArgs {
   uint32_t ntiles;
 };
 
-template <typename InT, bool STRIDED, int GMODE>
+// Four bytes (low byte of each argument) into one word, first argument lowest.
+__device__ __forceinline__ uint32_t pack4(uint32_t b0, uint32_t b1, uint32_t b2, uint32_t b3) {
+  return __byte_perm(__byte_perm(b0, b1, 0x0040), __byte_perm(b2, b3, 0x0040), 0x5410);
+}
+
+// Packed E2M1 codes (8 bytes, element 2k in the low nibble of byte k) of the
+// lane's block for a given eff.
+template <typename InT>
+__device__ __forceinline__ uint2 e2m1_codes(const In16<InT>& v, float eff) {
+  if (eff == 0.0f) {  // zero-block guard: zeros carrying the sign of x
+    const uint32_t sg = v.signs();
+    uint32_t w0 = 0, w1 = 0;
+#pragma unroll
+    for (int i = 0; i < 8; i++) {
+      w0 |= ((sg >> i) & 1u) << (4 * i + 3);
+      w1 |= ((sg >> (i + 8)) & 1u) << (4 * i + 3);
+    }
+    return make_uint2(w0, w1);
+  }
+  if (is_finite_normal(eff)) {
+    const float r = __frcp_rn(eff);
+    const float rl = __fmul_rn(r, 0.99999904632568359375f);  // 1 - 2^-20
+    const float rh = __fmul_rn(r, 1.00000095367431640625f);  // 1 + 2^-20
+    uint32_t b[8];
+    bool agree = true;
+#pragma unroll
+    for (int k = 0; k < 8; k++) {
+      const float2 l = mul2(v.lo(k), v.hi(k), rl);
+      const float2 h = mul2(v.lo(k), v.hi(k), rh);
+      b[k] = cvt_e2m1x2(l.x, l.y);
+      agree &= (b[k] == cvt_e2m1x2(h.x, h.y));
+    }
+    if (agree) return make_uint2(pack4(b[0], b[1], b[2], b[3]), pack4(b[4], b[5], b[6], b[7]));
+  }
+  uint32_t b[8];
+#pragma unroll
+  for (int k = 0; k < 8; k++) b[k] = cvt_e2m1x2(__fdiv_rn(v.lo(k), eff), __fdiv_rn(v.hi(k), eff));
+  return make_uint2(pack4(b[0], b[1], b[2], b[3]), pack4(b[4], b[5], b[6], b[7]));
+}
+
+template <typename InT, bool V8, bool STRIDED, int GMODE>
 __global__ void __launch_bounds__(kThreads)
 nvfp4_quant_kernel(const __grid_constant__ QuantArgs a) {
+  pdl_enter();
   __shared__ float red[kThreads / 32];
   const uint32_t tile = a.ntiles - 1 - blockIdx.x;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, sub = lane & 1;
-  const uint64_t b0 = uint64_t(tile) * kBlocksPerTile + warp * kBlocksPerWarp + (lane >> 1);
+  const uint64_t tb0 = uint64_t(tile) * kBlocksPerTile;
+  const uint64_t left = a.nblocks - tb0;
+  const uint32_t nt = left < kBlocksPerTile ? uint32_t(left) : uint32_t(kBlocksPerTile);
+  const bool full = nt == kBlocksPerTile;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const uint32_t lb0 = warp * kBlocksPerWarp + lane;
   const InT* x = static_cast<const InT*>(a.x);
 
-  In8<InT> v[kSteps];
+  In16<InT> v[kSteps];
 #pragma unroll
   for (int u = 0; u < kSteps; u++) {
-    const uint64_t blk = b0 + 16 * u;
-    if (blk < a.nblocks) {
-      uint64_t off;
-      if constexpr (STRIDED) {
-        const uint64_t r = a.rowdiv.div(blk);
-        off = r * uint64_t(a.ld) + (blk - r * a.bpr) * 16;
-      } else {
-        off = blk * 16;
-      }
-      v[u].load(x + off + sub * 8);
+    const uint32_t lb = lb0 + 32 * u;
+    const InT* p;
+    if constexpr (STRIDED) {
+      const uint64_t blk = tb0 + lb;
+      const uint64_t r = a.rowdiv.div(blk);
+      p = x + r * uint64_t(a.ld) + (blk - r * a.bpr) * 16;
     } else {
-      v[u].zero();
+      p = x + (tb0 + lb) * 16;
     }
+    if (full || lb < nt) v[u].template load<V8>(p); else v[u].zero();
   }
 
   float g;
@@ -150,100 +214,102 @@ nvfp4_quant_kernel(const __grid_constant__ QuantArgs a) {
   const bool gzero = (g == 0.0f);
   const float t = __fmul_rn(6.0f, g);
 
+  uint8_t* pk = a.packed + tb0 * 8;
+  uint8_t* sc = a.bscale + tb0;
 #pragma unroll
   for (int u = 0; u < kSteps; u++) {
-    const uint64_t blk = b0 + 16 * u;
-    float amax = v[u].absmax();
-    amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, 1));
-    amax = fmaxf(amax, 0.0f);  // a block holding only NaNs has amax 0
+    const uint32_t lb = lb0 + 32 * u;
+    if (!(full || lb < nt)) continue;
+    const float amax = fmaxf(v[u].absmax(), 0.0f);  // a block holding only NaNs has amax 0
     uint32_t sb = 0;
     float eff = 0.0f;
     if (!gzero) {
-      const float s = __fdiv_rn(amax, t);
-      sb = isnan(s) ? 0x7fu : (cvt_e4m3x2(s, 0.0f) & 0xffu);
+      sb = cvt_e4m3x2(__fdiv_rn(amax, t), 0.0f) & 0xffu;  // NaN -> 0x7F
       eff = __fmul_rn(decode_e4m3(sb), g);
     }
-    uint32_t word = 0;
-    if (eff == 0.0f) {
-      // zero-block guard: codes are zeros carrying the sign of x
-#pragma unroll
-      for (int i = 0; i < 8; i++) word |= (__float_as_uint(v[u][i]) >> 31) << (4 * i + 3);
-    } else {
-#pragma unroll
-      for (int k = 0; k < 4; k++) {
-        // fminf maps NaN to 6 (and leaves the saturation to the cvt otherwise)
-        const float q0 = fminf(__fdiv_rn(v[u][2 * k], eff), 6.0f);
-        const float q1 = fminf(__fdiv_rn(v[u][2 * k + 1], eff), 6.0f);
-        word |= cvt_e2m1x2(q0, q1) << (8 * k);
-      }
-    }
-    if (blk < a.nblocks) {
-      st_u32(a.packed + blk * 8 + sub * 4, word);
-      if (sub == 0) st_u8(a.bscale + blk, sb);
-    }
+    st_v2(pk + lb * 8, e2m1_codes(v[u], eff));
+    st_u8(sc + lb, sb);
   }
 }
 
 // --------------------------------------------------------------- dequant
 
-template <typename OutT>
+template <typename OutT, bool V8>
 __global__ void __launch_bounds__(kThreads)
 nvfp4_dequant_kernel(const uint8_t* __restrict__ packed, const uint8_t* __restrict__ bscale,
                      const float* __restrict__ gs, OutT* __restrict__ y, uint64_t nblocks) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, sub = lane & 1;
-  const uint64_t b0 =
-      uint64_t(blockIdx.x) * kBlocksPerTile + warp * kBlocksPerWarp + (lane >> 1);
-  uint32_t w[kSteps], sb[kSteps];
+  pdl_enter();
+  const uint64_t tb0 = uint64_t(blockIdx.x) * kBlocksPerTile;
+  const uint64_t left = nblocks - tb0;
+  const uint32_t nt = left < kBlocksPerTile ? uint32_t(left) : uint32_t(kBlocksPerTile);
+  const bool full = nt == kBlocksPerTile;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const uint32_t lb0 = warp * kBlocksPerWarp + lane;
+  uint2 w[kSteps];
+  uint32_t sb[kSteps];
 #pragma unroll
   for (int u = 0; u < kSteps; u++) {
-    const uint64_t blk = b0 + 16 * u;
-    if (blk < nblocks) {
-      w[u] = ld_nc_u32(packed + blk * 8 + sub * 4);
-      sb[u] = ld_nc_u8(bscale + blk);
+    const uint32_t lb = lb0 + 32 * u;
+    if (full || lb < nt) {
+      w[u] = ld_nc_v2(packed + (tb0 + lb) * 8);
+      sb[u] = ld_nc_u8(bscale + tb0 + lb);
     } else {
-      w[u] = 0;
+      w[u] = make_uint2(0, 0);
       sb[u] = 0;
     }
   }
   const float g = *gs;
 #pragma unroll
   for (int u = 0; u < kSteps; u++) {
-    const uint64_t blk = b0 + 16 * u;
-    if (blk >= nblocks) continue;
+    const uint32_t lb = lb0 + 32 * u;
+    if (!(full || lb < nt)) continue;
     const float eff = __fmul_rn(decode_e4m3(sb[u]), g);
-    float f[8];
+    float f[16];
 #pragma unroll
-    for (int k = 0; k < 4; k++) {
-      const float2 p = f16x2_to_f32x2(cvt_f16x2_from_e2m1x2((w[u] >> (8 * k)) & 0xffu));
-      f[2 * k] = __fmul_rn(p.x, eff);
-      f[2 * k + 1] = __fmul_rn(p.y, eff);
+    for (int k = 0; k < 8; k++) {
+      const uint32_t byte = ((k < 4 ? w[u].x : w[u].y) >> (8 * (k & 3))) & 0xffu;
+      const float2 d = f16x2_to_f32x2(cvt_f16x2_from_e2m1x2(byte));
+      const float2 p = mul2(d.x, d.y, eff);
+      f[2 * k] = p.x;
+      f[2 * k + 1] = p.y;
     }
     if (!isfinite(eff)) {  // only then can a product be NaN (0 * inf, NaN scale)
 #pragma unroll
-      for (int i = 0; i < 8; i++)
+      for (int i = 0; i < 16; i++)
         if (isnan(f[i])) f[i] = __uint_as_float(0x7fc00000u);
     }
-    OutT* dst = y + blk * 16 + sub * 8;
+    OutT* dst = y + (tb0 + lb) * 16;
     if constexpr (sizeof(OutT) == 2) {
-      uint4 o = make_uint4(cvt_bf16x2(f[0], f[1]), cvt_bf16x2(f[2], f[3]),
-                           cvt_bf16x2(f[4], f[5]), cvt_bf16x2(f[6], f[7]));
-      if (!isfinite(eff)) {
-        uint32_t ow[4] = {o.x, o.y, o.z, o.w};
+      uint32_t o[8];
 #pragma unroll
-        for (int i = 0; i < 8; i++) {
+      for (int k = 0; k < 8; k++) o[k] = cvt_bf16x2(f[2 * k], f[2 * k + 1]);
+      if (!isfinite(eff)) {
+#pragma unroll
+        for (int i = 0; i < 16; i++) {
           if (isnan(f[i])) {
             const int sh = 16 * (i & 1);
-            ow[i >> 1] = (ow[i >> 1] & ~(0xffffu << sh)) | (0x7fc0u << sh);
+            o[i >> 1] = (o[i >> 1] & ~(0xffffu << sh)) | (0x7fc0u << sh);
           }
         }
-        o = make_uint4(ow[0], ow[1], ow[2], ow[3]);
       }
-      st_v4(dst, o);
+      if constexpr (V8) {
+        st_v8(dst, o);
+      } else {
+        st_v4(dst, make_uint4(o[0], o[1], o[2], o[3]));
+        st_v4(dst + 8, make_uint4(o[4], o[5], o[6], o[7]));
+      }
     } else {
-      st_v4(dst, make_uint4(__float_as_uint(f[0]), __float_as_uint(f[1]),
-                            __float_as_uint(f[2]), __float_as_uint(f[3])));
-      st_v4(dst + 4, make_uint4(__float_as_uint(f[4]), __float_as_uint(f[5]),
-                                __float_as_uint(f[6]), __float_as_uint(f[7])));
+      uint32_t o[16];
+#pragma unroll
+      for (int i = 0; i < 16; i++) o[i] = __float_as_uint(f[i]);
+      if constexpr (V8) {
+        st_v8(dst, *reinterpret_cast<const uint32_t(*)[8]>(&o[0]));
+        st_v8(dst + 8, *reinterpret_cast<const uint32_t(*)[8]>(&o[8]));
+      } else {
+#pragma unroll
+        for (int i = 0; i < 4; i++)
+          st_v4(dst + 4 * i, make_uint4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]));
+      }
     }
   }
 }
@@ -257,39 +323,59 @@ int sm_count() {
   return n > 0 ? n : 148;
 }
 
+template <typename InT, bool V8, bool STRIDED>
+cudaError_t launch_amax_kernel(uint32_t grid, const void* x, uint64_t nchunks, uint32_t cpr,
+                               FastDiv rd, int64_t ld, float* partials, cudaStream_t s) {
+  return launch_pdl(nvfp4_amax_kernel<InT, V8, STRIDED>, grid, s, static_cast<const InT*>(x),
+                    nchunks, cpr, rd, ld, partials);
+}
+
 // Launches the amax pass into `partials`; returns the number of partials.
 mxq_status launch_amax(const void* x, int dt, int64_t M, int64_t N, int64_t ld, float* partials,
                        uint32_t* npartials, cudaStream_t s) {
-  const uint64_t cpr = uint64_t(N) / 8;
+  const uint64_t cpr = uint64_t(N) / 16;
   const uint64_t nchunks = uint64_t(M) * cpr;
   const uint64_t per_cta = uint64_t(kThreads) * kAmaxSteps;
   uint64_t grid = (nchunks + per_cta - 1) / per_cta;
-  const uint64_t cap = std::min<uint64_t>(kMaxPartials, uint64_t(sm_count()) * 8);
+  const uint64_t cap = std::min<uint64_t>(kMaxPartials, uint64_t(sm_count()) * kAmaxCtasPerSm);
   if (grid > cap) grid = cap;
   if (grid < 1) grid = 1;
   const FastDiv rd = FastDiv::make(uint32_t(cpr));
   const bool strided = ld != N;
+  const bool v8 = aligned32(x) && (uint64_t(ld) * elem_size(dt)) % 32 == 0;
+  const uint32_t G = uint32_t(grid);
+#define MXQ_AMAX(T, V, S) e = launch_amax_kernel<T, V, S>(G, x, nchunks, uint32_t(cpr), rd, ld, partials, s)
+  cudaError_t e;
   if (dt == MXQ_BF16) {
-    const uint16_t* xp = static_cast<const uint16_t*>(x);
-    if (strided) nvfp4_amax_kernel<uint16_t, true><<<uint32_t(grid), kThreads, 0, s>>>(xp, nchunks, uint32_t(cpr), rd, ld, partials);
-    else nvfp4_amax_kernel<uint16_t, false><<<uint32_t(grid), kThreads, 0, s>>>(xp, nchunks, uint32_t(cpr), rd, ld, partials);
+    if (v8) { if (strided) MXQ_AMAX(uint16_t, true, true); else MXQ_AMAX(uint16_t, true, false); }
+    else { if (strided) MXQ_AMAX(uint16_t, false, true); else MXQ_AMAX(uint16_t, false, false); }
   } else {
-    const float* xp = static_cast<const float*>(x);
-    if (strided) nvfp4_amax_kernel<float, true><<<uint32_t(grid), kThreads, 0, s>>>(xp, nchunks, uint32_t(cpr), rd, ld, partials);
-    else nvfp4_amax_kernel<float, false><<<uint32_t(grid), kThreads, 0, s>>>(xp, nchunks, uint32_t(cpr), rd, ld, partials);
+    if (v8) { if (strided) MXQ_AMAX(float, true, true); else MXQ_AMAX(float, true, false); }
+    else { if (strided) MXQ_AMAX(float, false, true); else MXQ_AMAX(float, false, false); }
   }
-  *npartials = uint32_t(grid);
-  return check_launch();
+#undef MXQ_AMAX
+  *npartials = G;
+  return launched(e);
 }
 
-template <typename InT, bool STRIDED>
+template <typename InT, bool V8, bool STRIDED>
 mxq_status launch_quant_mode(const QuantArgs& a, int mode, cudaStream_t s) {
   switch (mode) {
-    case kGiven: nvfp4_quant_kernel<InT, STRIDED, kGiven><<<a.ntiles, kThreads, 0, s>>>(a); break;
-    case kFromAmax: nvfp4_quant_kernel<InT, STRIDED, kFromAmax><<<a.ntiles, kThreads, 0, s>>>(a); break;
-    default: nvfp4_quant_kernel<InT, STRIDED, kFromPartials><<<a.ntiles, kThreads, 0, s>>>(a); break;
+    case kGiven:
+      return launched(launch_pdl(nvfp4_quant_kernel<InT, V8, STRIDED, kGiven>, a.ntiles, s, a));
+    case kFromAmax:
+      return launched(launch_pdl(nvfp4_quant_kernel<InT, V8, STRIDED, kFromAmax>, a.ntiles, s, a));
+    default:
+      return launched(launch_pdl(nvfp4_quant_kernel<InT, V8, STRIDED, kFromPartials>, a.ntiles, s, a));
   }
-  return check_launch();
+}
+
+template <typename InT>
+mxq_status launch_quant_typed(const QuantArgs& a, int mode, bool v8, bool strided, cudaStream_t s) {
+  if (v8) return strided ? launch_quant_mode<InT, true, true>(a, mode, s)
+                         : launch_quant_mode<InT, true, false>(a, mode, s);
+  return strided ? launch_quant_mode<InT, false, true>(a, mode, s)
+                 : launch_quant_mode<InT, false, false>(a, mode, s);
 }
 
 mxq_status check_input(const void* x, int dt, int64_t M, int64_t N, int64_t ld_x) {
@@ -298,7 +384,7 @@ mxq_status check_input(const void* x, int dt, int64_t M, int64_t N, int64_t ld_x
   if (M == 0 || N == 0) return MXQ_OK;
   if (!x) return MXQ_ERR_NULL;
   const uint64_t nblocks = uint64_t(M) * (uint64_t(N) / 16);
-  if (uint64_t(N) / 8 > 0xffffffffull || (nblocks + kBlocksPerTile - 1) / kBlocksPerTile > 0x7fffffffull)
+  if (uint64_t(N) / 16 > 0xffffffffull || (nblocks + kBlocksPerTile - 1) / kBlocksPerTile > 0x7fffffffull)
     return MXQ_ERR_SHAPE;
   if (!aligned16(x) || (uint64_t(ld_x) * elem_size(dt)) % 16 != 0) return MXQ_ERR_ALIGN;
   return MXQ_OK;
@@ -329,8 +415,8 @@ mxq_status nvfp4_amax(const void* x, int dt, int64_t M, int64_t N, int64_t ld_x,
   uint32_t np = 0;
   st = launch_amax(x, dt, M, N, ld_x, static_cast<float*>(workspace), &np, s);
   if (st != MXQ_OK) return st;
-  nvfp4_amax_finalize_kernel<<<1, kThreads, 0, s>>>(static_cast<float*>(workspace), np, amax);
-  return check_launch();
+  return launched(launch_pdl(nvfp4_amax_finalize_kernel, 1, s,
+                             static_cast<const float*>(workspace), np, amax));
 }
 
 mxq_status nvfp4_quantize(const void* x, int dt, int64_t M, int64_t N, int64_t ld_x,
@@ -363,18 +449,16 @@ mxq_status nvfp4_quantize(const void* x, int dt, int64_t M, int64_t N, int64_t l
   a.amax_in = amax_in;
   a.nblocks = uint64_t(M) * a.bpr;
   a.ntiles = uint32_t((a.nblocks + kBlocksPerTile - 1) / kBlocksPerTile);
-  int mode = given ? kGiven : (amax_in ? kFromAmax : kFromPartials);
+  const int mode = given ? kGiven : (amax_in ? kFromAmax : kFromPartials);
   if (pass1) {
     a.partials = static_cast<const float*>(workspace);
     st = launch_amax(x, dt, M, N, ld_x, static_cast<float*>(workspace), &a.npartials, s);
     if (st != MXQ_OK) return st;
   }
   const bool strided = ld_x != N;
-  if (dt == MXQ_BF16)
-    return strided ? launch_quant_mode<uint16_t, true>(a, mode, s)
-                   : launch_quant_mode<uint16_t, false>(a, mode, s);
-  return strided ? launch_quant_mode<float, true>(a, mode, s)
-                 : launch_quant_mode<float, false>(a, mode, s);
+  const bool v8 = aligned32(x) && (uint64_t(ld_x) * elem_size(dt)) % 32 == 0;
+  if (dt == MXQ_BF16) return launch_quant_typed<uint16_t>(a, mode, v8, strided, s);
+  return launch_quant_typed<float>(a, mode, v8, strided, s);
 }
 
 mxq_status nvfp4_dequantize(const uint8_t* packed, const uint8_t* block_scale,
@@ -390,14 +474,16 @@ mxq_status nvfp4_dequantize(const uint8_t* packed, const uint8_t* block_scale,
   const uint64_t tiles = (nblocks + kBlocksPerTile - 1) / kBlocksPerTile;
   if (tiles > 0x7fffffffull) return MXQ_ERR_SHAPE;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const uint32_t grid = uint32_t(tiles);
+  const bool v8 = aligned32(y);
   if (out_dt == MXQ_BF16) {
-    nvfp4_dequant_kernel<uint16_t><<<uint32_t(tiles), kThreads, 0, s>>>(
-        packed, block_scale, global_scale, static_cast<uint16_t*>(y), nblocks);
-  } else {
-    nvfp4_dequant_kernel<float><<<uint32_t(tiles), kThreads, 0, s>>>(
-        packed, block_scale, global_scale, static_cast<float*>(y), nblocks);
+    uint16_t* yp = static_cast<uint16_t*>(y);
+    return launched(v8 ? launch_pdl(nvfp4_dequant_kernel<uint16_t, true>, grid, s, packed, block_scale, global_scale, yp, nblocks)
+                       : launch_pdl(nvfp4_dequant_kernel<uint16_t, false>, grid, s, packed, block_scale, global_scale, yp, nblocks));
   }
-  return check_launch();
+  float* yp = static_cast<float*>(y);
+  return launched(v8 ? launch_pdl(nvfp4_dequant_kernel<float, true>, grid, s, packed, block_scale, global_scale, yp, nblocks)
+                     : launch_pdl(nvfp4_dequant_kernel<float, false>, grid, s, packed, block_scale, global_scale, yp, nblocks));
 }
 
 }  // extern "C"
