@@ -14,18 +14,27 @@
 //   packed byte k of a row = q[2k] | q[2k+1] << 4.
 // g, s and eff use IEEE division / multiplication (__fdiv_rn, __fmul_rn).
 //
-// E2M1 codes without a division per element. The code is a monotone step
-// function of the correctly rounded quotient f = fl(x / eff). With
-// r = fl(1 / eff) (IEEE reciprocal, once per block), the two products
-// lo = fl(x * fl(r * (1 - 2^-20))) and hi = fl(x * fl(r * (1 + 2^-20)))
-// bracket f strictly: three roundings move a product by at most 3 * 2^-24
-// relative, far inside the 2^-20 margin, while f itself lies within 2^-24 of
-// x / eff. So whenever E2M1(lo) == E2M1(hi), that code is E2M1(f) (a tie of
-// f on a midpoint would put lo and hi on opposite sides of it). Products
-// that fall below the fp32 normal range are far below the first midpoint
-// (0.25), products that overflow are far above 6, so the bracket argument
-// only needs eff to be a finite normal number. Otherwise, and for the rare
-// lane whose bracket straddles a midpoint, the lane divides exactly.
+// Codes without a division per element. An E4M3 or E2M1 code is a monotone
+// step function of the correctly rounded quotient f; its steps sit at the
+// midpoints between neighbouring code values.
+//  - E2M1 (per element): with r = rcp.approx.f32(eff) (documented error
+//    <= 1 ulp), the products lo = fl(x * fl(r (1 - 2^-20))) and
+//    hi = fl(x * fl(r (1 + 2^-20))) bracket f strictly (a few 2^-24 relative
+//    roundings against the 2^-20 margin; f lies within 2^-24 of x / eff). When
+//    E2M1(lo) == E2M1(hi) that is E2M1(f); a tie of f on a midpoint puts lo
+//    and hi on opposite sides of it. Elements whose brackets disagree (bf16
+//    inputs make exact quotients such as 3.5 common) are decided exactly from
+//    the fused-multiply-add residual |x| - eff * M against the midpoint M
+//    (see e2m1_resolve), or by IEEE division for divisors below 2^-98.
+//  - E4M3 (per block): the product amax * rcp.approx(t) lies within a few
+//    ulps of f; every E4M3 midpoint has at most four significant bits, so the
+//    product rounds like f unless it is within 32 ulps of a value whose
+//    mantissa is zero below bit 19, in which case the block divides exactly.
+// Divisors outside [2^-125, 2^125) (whose approximate reciprocal would not be
+// normal) take the exact path. Products below the normal range are far below
+// the first midpoint and overflowing products far above the last, so neither
+// can change a code. The exact paths are out-of-line functions so that the
+// compiler cannot evaluate them speculatively.
 //
 // Passes: the tensor amax must be known before any block can be quantized,
 // so a first kernel reduces |x| into per-CTA partial maxima (workspace), and
@@ -55,9 +64,24 @@ __device__ __forceinline__ float decode_e4m3(uint32_t code) {
   return f16x2_to_f32x2(cvt_f16x2_from_e4m3x2(code)).x;
 }
 
-__device__ __forceinline__ bool is_finite_normal(float v) {
+// Reciprocal by the hardware approximation (<= 1 ulp for normal inputs).
+__device__ __forceinline__ float rcp_approx(float v) {
+  float r;
+  asm("rcp.approx.f32 %0, %1;" : "=f"(r) : "f"(v));
+  return r;
+}
+
+// True when |v| in [2^-125, 2^125): its approximate reciprocal is normal.
+__device__ __forceinline__ bool rcp_safe(float v) {
   const uint32_t e = __float_as_uint(v) & 0x7f800000u;
-  return e != 0 && e != 0x7f800000u;
+  return e >= (2u << 23) && e < (252u << 23);
+}
+
+// Distance-like key of v to the nearest value whose mantissa is zero below
+// bit `bits`: small (<= 64) when v is within 32 ulps of such a value.
+template <int BITS>
+__device__ __forceinline__ uint32_t grid_key(float v) {
+  return (__float_as_uint(v) + 32u) & ((1u << BITS) - 1u);
 }
 
 inline bool aligned32(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 31u) == 0; }
@@ -132,6 +156,61 @@ __device__ __forceinline__ uint32_t pack4(uint32_t b0, uint32_t b1, uint32_t b2,
   return __byte_perm(__byte_perm(b0, b1, 0x0040), __byte_perm(b2, b3, 0x0040), 0x5410);
 }
 
+// IEEE quotient, kept out of line so that the compiler cannot evaluate it
+// speculatively on the common path.
+__device__ __noinline__ float div_exact(float a, float b) { return __fdiv_rn(a, b); }
+
+// E2M1 codes of the 16 elements from correctly rounded quotients (the rare
+// path; out of line for the same reason).
+__device__ __noinline__ uint2 e2m1_exact(const float (&x)[16], float eff) {
+  uint32_t b[8];
+#pragma unroll
+  for (int k = 0; k < 8; k++) b[k] = cvt_e2m1x2(__fdiv_rn(x[2 * k], eff), __fdiv_rn(x[2 * k + 1], eff));
+  return make_uint2(pack4(b[0], b[1], b[2], b[3]), pack4(b[4], b[5], b[6], b[7]));
+}
+
+// Exact E2M1 code of fl(x / eff) when |x| / eff is known to lie within
+// 2^-19 (relative) of M, the midpoint between magnitude codes c and c + 1
+// (c in 0..6), for eff >= 2^-98. Then D = |x| - eff * M is a multiple of
+// 2^(e(eff) + e(M) - 25) of magnitude below 2^(e(eff) + e(M) - 17), i.e. a
+// number of at most 8 significant bits, so the fused multiply-add returns it
+// exactly. f = fl(|x| / eff) equals M exactly when -h_below <= D <= h_above
+// (h = eff times half an ulp of M on either side; the quotient of numbers of
+// at most 24 significant bits never falls exactly on an fp32 rounding
+// boundary, so the ends need no tie rule), is above M when D > h_above and
+// below when D < -h_below; on a tie the even code wins.
+__device__ __forceinline__ uint32_t e2m1_resolve(float x, float eff, uint32_t c) {
+  // midpoints 0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5 and their binade exponents
+  const float M = c == 0 ? 0.25f : c == 1 ? 0.75f : c == 2 ? 1.25f : c == 3 ? 1.75f
+                : c == 4 ? 2.5f : c == 5 ? 3.5f : 5.0f;
+  const int eM = c == 0 ? -2 : c == 1 ? -1 : c <= 3 ? 0 : c <= 5 ? 1 : 2;
+  const float h_above = __fmul_rn(eff, __uint_as_float(uint32_t(127 + eM - 24) << 23));
+  const float h_below = c == 0 ? __fmul_rn(h_above, 0.5f) : h_above;  // 0.25 is a power of two
+  const float D = __fmaf_rn(-eff, M, fabsf(x));
+  const uint32_t mag = D > h_above ? c + 1 : (D < -h_below ? c : ((c & 1u) ? c + 1 : c));
+  return mag | ((__float_as_uint(x) >> 31) << 3);
+}
+
+// Byte of two E2M1 codes for (x0, x1) when the bracket codes cl (from the
+// lower products) and ch (upper) disagree in at least one nibble: each
+// disagreeing nibble is decided exactly. Out of line so that the common path
+// only pays a predicted-not-taken branch per pair.
+__device__ __noinline__ uint32_t fix_pair(float x0, float x1, float eff, uint32_t cl, uint32_t ch) {
+  const bool fma_ok = (__float_as_uint(eff) & 0x7f800000u) >= (29u << 23);  // eff >= 2^-98
+  uint32_t code = cl & 0xffu;
+#pragma unroll
+  for (int e = 0; e < 2; e++) {
+    const uint32_t nl = (cl >> (4 * e)) & 0xfu, nh = (ch >> (4 * e)) & 0xfu;
+    if (nl != nh) {
+      const float xe = e ? x1 : x0;
+      const uint32_t c = min(nl & 7u, nh & 7u);
+      const uint32_t q = fma_ok ? e2m1_resolve(xe, eff, c) : (cvt_e2m1x2(__fdiv_rn(xe, eff), 0.0f) & 0xfu);
+      code = (code & ~(0xfu << (4 * e))) | (q << (4 * e));
+    }
+  }
+  return code;
+}
+
 // Packed E2M1 codes (8 bytes, element 2k in the low nibble of byte k) of the
 // lane's block for a given eff.
 template <typename InT>
@@ -146,25 +225,30 @@ __device__ __forceinline__ uint2 e2m1_codes(const In16<InT>& v, float eff) {
     }
     return make_uint2(w0, w1);
   }
-  if (is_finite_normal(eff)) {
-    const float r = __frcp_rn(eff);
+  if (rcp_safe(eff)) {
+    const float r = rcp_approx(eff);
     const float rl = __fmul_rn(r, 0.99999904632568359375f);  // 1 - 2^-20
     const float rh = __fmul_rn(r, 1.00000095367431640625f);  // 1 + 2^-20
     uint32_t b[8];
-    bool agree = true;
 #pragma unroll
     for (int k = 0; k < 8; k++) {
       const float2 l = mul2(v.lo(k), v.hi(k), rl);
       const float2 h = mul2(v.lo(k), v.hi(k), rh);
-      b[k] = cvt_e2m1x2(l.x, l.y);
-      agree &= (b[k] == cvt_e2m1x2(h.x, h.y));
+      const uint32_t cl = cvt_e2m1x2(l.x, l.y), ch = cvt_e2m1x2(h.x, h.y);
+      // a code boundary inside the bracket (exact quotients such as 3.5 are
+      // common with bf16 inputs): decide those elements exactly
+      b[k] = __builtin_expect(cl != ch, 0) ? fix_pair(v.lo(k), v.hi(k), eff, cl, ch) : cl;
     }
-    if (agree) return make_uint2(pack4(b[0], b[1], b[2], b[3]), pack4(b[4], b[5], b[6], b[7]));
+    const uint2 out = make_uint2(pack4(b[0], b[1], b[2], b[3]), pack4(b[4], b[5], b[6], b[7]));
+    return out;
   }
-  uint32_t b[8];
+  float x[16];
 #pragma unroll
-  for (int k = 0; k < 8; k++) b[k] = cvt_e2m1x2(__fdiv_rn(v.lo(k), eff), __fdiv_rn(v.hi(k), eff));
-  return make_uint2(pack4(b[0], b[1], b[2], b[3]), pack4(b[4], b[5], b[6], b[7]));
+  for (int k = 0; k < 8; k++) {
+    x[2 * k] = v.lo(k);
+    x[2 * k + 1] = v.hi(k);
+  }
+  return e2m1_exact(x, eff);
 }
 
 template <typename InT, bool V8, bool STRIDED, int GMODE>
@@ -213,6 +297,8 @@ nvfp4_quant_kernel(const __grid_constant__ QuantArgs a) {
   }
   const bool gzero = (g == 0.0f);
   const float t = __fmul_rn(6.0f, g);
+  const bool t_ok = rcp_safe(t);
+  const float rt = rcp_approx(t);
 
   uint8_t* pk = a.packed + tb0 * 8;
   uint8_t* sc = a.bscale + tb0;
@@ -224,7 +310,11 @@ nvfp4_quant_kernel(const __grid_constant__ QuantArgs a) {
     uint32_t sb = 0;
     float eff = 0.0f;
     if (!gzero) {
-      sb = cvt_e4m3x2(__fdiv_rn(amax, t), 0.0f) & 0xffu;  // NaN -> 0x7F
+      // E4M3 code of fl(amax / t); the approximate quotient decides unless it
+      // is within 32 ulps of a value with four significant bits
+      float s = __fmul_rn(amax, rt);
+      if (__builtin_expect(!t_ok || grid_key<19>(s) <= 64u, 0)) s = div_exact(amax, t);
+      sb = cvt_e4m3x2(s, 0.0f) & 0xffu;  // NaN -> 0x7F
       eff = __fmul_rn(decode_e4m3(sb), g);
     }
     st_v2(pk + lb * 8, e2m1_codes(v[u], eff));
