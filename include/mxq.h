@@ -28,7 +28,7 @@
  *  - Tensor pointers are DEVICE pointers owned by the caller (for example
  *    PyTorch tensors); host pointers appear only where stated. The library
  *    never allocates, frees or synchronizes, and keeps no state between
- *    calls.
+ *    calls (except the fixed scratch array of nvfp4_quantize_noalloc).
  *  - Work is enqueued on `stream` (NULL = the legacy default stream) and runs
  *    asynchronously; outputs are ready when the stream reaches that point.
  *  - Arguments are checked on the host before anything is enqueued. A call
@@ -173,6 +173,29 @@ mxq_status nvfp4_quantize(const void* x, int dt, int64_t M, int64_t N, int64_t l
                           uint8_t* packed, uint8_t* block_scale, float* global_scale,
                           const float* amax_in, uint32_t flags, void* workspace,
                           size_t ws_bytes, mxq_stream_t stream);
+
+/* nvfp4_quantize without a workspace argument, for callers that cannot
+ * allocate device memory at the point where they quantize: code running
+ * inside a serving engine or plugin whose device memory is planned up front,
+ * or a C program with no device allocator of its own. (The pages have no
+ * counterpart to this entry point; it is an interface convenience.)
+ * Arguments, results and errors are those of nvfp4_quantize. The scratch of
+ * the tensor-amax pass (2048 fp32 partial maxima, 8 KiB) lives in a fixed
+ * array inside the library, which every GPU that loads the library holds
+ * until the process exits; the call allocates nothing.
+ *  - The first call on a device looks up that array's device address with the
+ *    caller's current device (one cudaGetSymbolAddress); make that first call
+ *    before any stream capture. stream must belong to the current device.
+ *  - Every call on a device shares the one array, so calls whose work
+ *    overlaps on the GPU (for example on two streams) race and give wrong
+ *    results; serialize them. Nothing in the array needs to start at zero:
+ *    each call writes every slot it reads.
+ *  - A call whose scratch need (mxq_nvfp4_workspace_bytes(M, N)) exceeds the
+ *    array is rejected with MXQ_ERR_WORKSPACE; today the need is 8 KiB for
+ *    every M and N. */
+mxq_status nvfp4_quantize_noalloc(const void* x, int dt, int64_t M, int64_t N, int64_t ld_x,
+                                  uint8_t* packed, uint8_t* block_scale, float* global_scale,
+                                  const float* amax_in, uint32_t flags, mxq_stream_t stream);
 
 /* NVFP4 dequantize: eff = decode_e4m3(s_b) * g and y = decode_e2m1(q) * eff,
  * both fp32 products, written as fp32 or bf16 (RNE). global_scale is a device

@@ -12,6 +12,7 @@
 #include <cuda_runtime.h>
 #include <algorithm>
 #include <cstring>
+#include <mutex>
 #include <utility>
 
 #include "mxq.h"

@@ -577,3 +577,76 @@ mxq_status nvfp4_dequantize(const uint8_t* packed, const uint8_t* block_scale,
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// nvfp4_quantize_noalloc: the same quantization for callers that cannot
+// allocate device memory when they quantize, e.g. code that runs inside a
+// serving engine or plugin with a fixed, pre-planned memory budget, or a C
+// program with no device allocator at hand. Its only scratch (the per-CTA
+// partial maxima of the tensor-amax pass) lives in the fixed array below,
+// which every GPU that loads this library holds until the process exits.
+
+namespace mxq {
+namespace {
+
+constexpr int kNoallocPartials = kMaxPartials;  // 2048 floats = 8 KiB per device
+static __device__ __align__(256) float g_noalloc_partials[kNoallocPartials];
+
+constexpr int kMaxDevices = 256;
+std::mutex g_noalloc_mu;
+float* g_noalloc_ptr[kMaxDevices] = {};  // device address of the array, per device
+
+// Device address of g_noalloc_partials on the current device. The first call
+// on a device looks it up (cudaGetSymbolAddress, with that device current);
+// later calls reuse it.
+mxq_status noalloc_scratch(float** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) {
+    record_cuda_error(e);
+    return MXQ_ERR_CUDA;
+  }
+  if (dev < 0 || dev >= kMaxDevices) return MXQ_ERR_ARG;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_partials);
+    if (e != cudaSuccess) {
+      record_cuda_error(e);
+      return MXQ_ERR_CUDA;
+    }
+    g_noalloc_ptr[dev] = static_cast<float*>(p);
+  }
+  *out = g_noalloc_ptr[dev];
+  return MXQ_OK;
+}
+
+}  // namespace
+}  // namespace mxq
+
+extern "C" mxq_status nvfp4_quantize_noalloc(const void* x, int dt, int64_t M, int64_t N,
+                                             int64_t ld_x, uint8_t* packed,
+                                             uint8_t* block_scale, float* global_scale,
+                                             const float* amax_in, uint32_t flags,
+                                             mxq_stream_t stream) {
+  using namespace mxq;
+  // the same argument checks as nvfp4_quantize, before the one-time set-up
+  if (flags & ~MXQ_NVFP4_GLOBAL_GIVEN) return MXQ_ERR_ARG;
+  if ((flags & MXQ_NVFP4_GLOBAL_GIVEN) && amax_in) return MXQ_ERR_ARG;
+  mxq_status st = check_input(x, dt, M, N, ld_x);
+  if (st != MXQ_OK) return st;
+  if (M == 0 || N == 0) return MXQ_OK;
+  if (!packed || !block_scale || !global_scale) return MXQ_ERR_NULL;
+  if (!aligned16(packed)) return MXQ_ERR_ALIGN;
+  // scratch needed by this call versus what the fixed array holds
+  const size_t need = mxq_nvfp4_workspace_bytes(M, N);
+  if (need > sizeof(float) * kNoallocPartials) return MXQ_ERR_WORKSPACE;
+  const bool pass1 = !(flags & MXQ_NVFP4_GLOBAL_GIVEN) && amax_in == nullptr;
+  float* scratch = nullptr;
+  if (pass1) {
+    st = noalloc_scratch(&scratch);
+    if (st != MXQ_OK) return st;
+  }
+  return nvfp4_quantize(x, dt, M, N, ld_x, packed, block_scale, global_scale, amax_in, flags,
+                        scratch, scratch ? sizeof(float) * kNoallocPartials : 0, stream);
+}

@@ -139,6 +139,20 @@ def test_nvfp4_validation():
     assert L.nvfp4_dequantize(A, A, A, 4, 64, A, 9, None) == DTYPE
 
 
+def test_nvfp4_noalloc_validation():
+    f = ctypes.CDLL(mxq.library_path).nvfp4_quantize_noalloc
+    vp, i64, i32, u32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_uint32
+    f.argtypes = [vp, i32, i64, i64, i64, vp, vp, vp, vp, u32, vp]
+    f.restype = i32
+    assert f(A, 0, 4, 64, 64, A, A, A, None, 2, None) == ARG
+    assert f(A, 0, 4, 64, 64, A, A, A, A, 1, None) == ARG
+    assert f(A, 0, 4, 40, 40, A, A, A, None, 0, None) == SHAPE
+    assert f(None, 0, 4, 64, 64, A, A, A, None, 0, None) == NULL
+    assert f(A, 0, 4, 64, 64, A, A, None, None, 0, None) == NULL
+    assert f(A, 0, 4, 64, 64, A + 4, A, A, None, 0, None) == ALIGN
+    assert f(None, 0, 0, 64, 64, None, None, None, None, 0, None) == OK
+
+
 def test_python_binding_rejects_cpu_tensors():
     import torch
     with pytest.raises(ValueError):
