@@ -41,6 +41,7 @@ import workloads as W  # noqa: E402
 METRIC = "MXFP8 quantize GB/s (read+write) and % of B200 HBM peak, bit-exact"
 SPEC_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
+SAMPLE_EVERY = 16
 M_ROWS, N_COLS = 16384, 7168
 
 
@@ -75,9 +76,17 @@ def hbm_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def kernel_source_sha():
+KERNEL_SOURCES = {"mxfp8_quant_kernel": ("common.cuh", "mxfp8.cu"),
+                  "mxfp8_dequant_kernel": ("common.cuh", "mxfp8.cu"),
+                  "nvfp4_amax_kernel": ("common.cuh", "nvfp4.cu"),
+                  "nvfp4_quant_kernel": ("common.cuh", "nvfp4.cu"),
+                  "nvfp4_dequant_kernel": ("common.cuh", "nvfp4.cu")}
+
+
+def kernel_source_sha(kernel):
+    """Hash of the source files a kernel is built from."""
     h = hashlib.sha256()
-    for f in ("common.cuh", "mxfp8.cu", "nvfp4.cu"):
+    for f in KERNEL_SOURCES[kernel]:
         with open(os.path.join(ROOT, "nvfp4_block_scaled_sm_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
@@ -89,7 +98,7 @@ def recorded_traffic(kernel):
     try:
         with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
             rec = json.load(f)[kernel]
-        if rec.get("source_sha") == kernel_source_sha():
+        if rec.get("source_sha") == kernel_source_sha(kernel):
             return int(rec["dram_bytes_per_launch"])
     except Exception:
         pass
@@ -180,27 +189,29 @@ def reduce_max(value: float, world: int, device) -> float:
 
 def time_oracle_round_trip(x: np.ndarray, min_seconds: float):
     """Oracle MXFP8 quantize + swizzle + dequantize of the rows `x`, repeated
-    until min_seconds have elapsed; returns (seconds per pass, passes)."""
+    until min_seconds have elapsed; returns (seconds per pass, passes,
+    (qweight, scale, dequantized bf16 bits))."""
     import oracle
     oracle.build()
     passes, t0 = 0, time.perf_counter()
     while True:
         q, s = oracle.mxfp8_quantize(x)
         oracle.swizzle_scales(s)
-        oracle.mxfp8_dequantize(q, s, out="bf16")
+        y = oracle.mxfp8_dequantize(q, s, out="bf16")
         passes += 1
         el = time.perf_counter() - t0
         if el >= min_seconds:
-            return el / passes, passes
+            return el / passes, passes, (q, s, y)
 
 
 def cpu_baseline(x_full: np.ndarray, rows: int = 2048, min_seconds: float = 12.0):
+    """The oracle timed on the first `rows` rows; also returns its outputs."""
     x = np.ascontiguousarray(x_full[:rows])
-    sec, passes = time_oracle_round_trip(x, min_seconds)
+    sec, passes, outs = time_oracle_round_trip(x, min_seconds)
     nbytes = mxfp8_quant_bytes(rows, N_COLS) + mxfp8_dequant_bytes(rows, N_COLS)
     return {"value": nbytes / sec / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
             "sample": f"first {rows} of {M_ROWS} rows of the activation workload, quantize "
-                      f"(+swizzle) + dequantize, {passes} passes, single-threaded scalar C"}
+                      f"(+swizzle) + dequantize, {passes} passes, single-threaded scalar C"}, outs
 
 
 def run_reference(args):
@@ -208,7 +219,7 @@ def run_reference(args):
     if rank != 0:
         return
     x_all = W.activation(M=M_ROWS, N=N_COLS)
-    t_row, _ = time_oracle_round_trip(np.ascontiguousarray(x_all[:64]), 0.5)
+    t_row, _, _ = time_oracle_round_trip(np.ascontiguousarray(x_all[:64]), 0.5)
     t_row /= 64
     budget = 150.0
     rows = int(max(1, min(M_ROWS, budget / max(1, args.steps + args.warmup) / t_row)))
@@ -288,7 +299,11 @@ def run(args):
     torch.cuda.synchronize(device)
 
     K = args.steps
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    # Per-kernel durations come from events around the two kernels of every
+    # SAMPLE_EVERY-th step only: an event recorded between two kernels ends
+    # their programmatic overlap, so events on every step would slow the step.
+    sampled = [k for k in range(K) if k % SAMPLE_EVERY == SAMPLE_EVERY - 1] or [K - 1]
+    ev = {k: [torch.cuda.Event(enable_timing=True) for _ in range(3)] for k in sampled}
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if world > 1:
         torch.distributed.barrier()
@@ -296,30 +311,29 @@ def run(args):
     with ClockSampler(device) as clk:
         t_start.record(stream)
         for k in range(K):
-            ev[k][0].record(stream)
+            e = ev.get(k)
+            if e:
+                e[0].record(stream)
             L.mxfp8_quantize(P[0], 0, M, N, N, P[1], P[2], P[3], sp)
-            ev[k][1].record(stream)
+            if e:
+                e[1].record(stream)
             L.mxfp8_dequantize(P[1], P[2], M, N, P[4], 0, sp)
-            ev[k][2].record(stream)
+            if e:
+                e[2].record(stream)
         t_end.record(stream)
         torch.cuda.synchronize(device)
     if world > 1:
         torch.distributed.barrier()
     elapsed_ms = t_start.elapsed_time(t_end)
-    q_ms = [ev[k][0].elapsed_time(ev[k][1]) for k in range(K)]
-    d_ms = [ev[k][1].elapsed_time(ev[k][2]) for k in range(K)]
+    q_ms = [ev[k][0].elapsed_time(ev[k][1]) for k in sampled]
+    d_ms = [ev[k][1].elapsed_time(ev[k][2]) for k in sampled]
     max_ms = reduce_max(elapsed_ms, world, device)
 
-    # correctness of what was timed: the last step's outputs against the oracle on sampled rows
-    verified = None
-    if rank == 0 and not args.no_verify:
-        import oracle
-        rows = np.random.default_rng(7).choice(M, 64, replace=False)
-        qo, so = oracle.mxfp8_quantize(np.ascontiguousarray(xb[rows]))
-        yo = oracle.mxfp8_dequantize(qo, so, out="bf16")
-        qh, sh = q.cpu().numpy()[rows], s.cpu().numpy()[rows]
-        yh = y.view(torch.int16).cpu().numpy().view(np.uint16)[rows]
-        verified = bool(np.array_equal(qh, qo) and np.array_equal(sh, so) and np.array_equal(yh, yo))
+    # outputs of the timed region's last step, kept for the CPU-baseline leg's check
+    n_check = 2048
+    q_last = q[:n_check].cpu().numpy()
+    s_last = s[:n_check].cpu().numpy()
+    y_last = y[:n_check].view(torch.int16).cpu().numpy().view(np.uint16)
 
     # end-to-end through the public API: pinned host input -> device, quantize,
     # dequantize, all outputs -> pinned host, every step
@@ -390,11 +404,16 @@ def run(args):
                 "ms_per_step": e2e_ms, "steps": e2e_steps,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": 2 * K,
+        "kernel_time_sampling": f"events around both kernels on every {SAMPLE_EVERY}th step "
+                                f"({len(sampled)} of {K} steps)",
         "clocks": clk.summary(),
-        "verified_bit_exact_sampled_rows": verified,
     }
     if not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(xb)
+        line["cpu_baseline"], (qo, so, yo) = cpu_baseline(xb, n_check)
+        line["verified_bit_exact_first_rows"] = {
+            "rows": n_check,
+            "equal_to_oracle": bool(np.array_equal(q_last, qo) and np.array_equal(s_last, so)
+                                    and np.array_equal(y_last, yo))}
     print(json.dumps(line), flush=True)
     if args.suite:
         run_suite(device)
@@ -499,7 +518,6 @@ def main():
     ap.add_argument("--suite-only", default=None,
                     help="time only the workload kernels whose workload name contains this")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--no-verify", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
