@@ -479,6 +479,12 @@ def run_suite(device, only=None):
         emit("mxfp8_dequantize->fp32 activation 16384x7168",
              mxfp8_dequant_bytes(M_ROWS, N_COLS, 4),
              time_kernel(lambda: mxq.mxfp8_dequantize(q, s, torch.float32), 30))
+        emit("mxfp8_quantize_columnwise activation 16384x7168",
+             mxfp8_quant_bytes(M_ROWS, N_COLS, swizzled=False),
+             time_kernel(lambda: mxq.mxfp8_quantize_columnwise(x), 30))
+        emit("mxfp8_quantize rowwise+columnwise (one read) activation 16384x7168",
+             2 * mxfp8_quant_bytes(M_ROWS, N_COLS, swizzled=False) - 2 * M_ROWS * N_COLS,
+             time_kernel(lambda: mxq.mxfp8_quantize_columnwise(x, rowwise=True), 30))
         xf = x.float()
         emit("mxfp8_quantize fp32-input activation 16384x7168",
              mxfp8_quant_bytes(M_ROWS, N_COLS, in_bytes=4, swizzled=False),

@@ -139,6 +139,25 @@ mxq_status mxfp8_quantize_grouped(int32_t E, const void* const* xs, const int64_
                                   int64_t N, int dt, uint8_t* qweight, uint8_t* scale,
                                   mxq_stream_t stream);
 
+/* MXFP8 columnwise quantize: groups of 32 consecutive ROWS of one column (the
+ * layout a backward GEMM reads), i.e. the rowwise quantize of the transposed
+ * tensor. Rows are zero-padded to a multiple of 32 and the result cropped
+ * back ("PR #1935 完整报告 ...", 实现拆解 item 1); for columnwise groups the
+ * zero padding takes part in the last group of every column.
+ *  x          [M, N] bf16 or fp32, row stride ld_x elements; N % 16 == 0.
+ *  qweight_t  [N, M] uint8 E4M3 codes (transposed, row-major): qweight_t[c, r]
+ *             is the code of x[r, c].
+ *  scale_t    [N, ceil(M/32)] uint8 E8M0 bytes.
+ *  qweight, scale  both NULL, or the rowwise outputs of mxfp8_quantize
+ *             ([M, N] and [M, N/32], compact; then N % 32 == 0): the fused
+ *             mode produces both layouts from one read of x.
+ * Per group the rule of mxfp8_quantize applies (amax over non-NaN elements,
+ * E8M0 byte, E4M3 RNE with saturation). One launch; tiles of 128 rows x 256
+ * bytes staged in shared memory. */
+mxq_status mxfp8_quantize_columnwise(const void* x, int dt, int64_t M, int64_t N, int64_t ld_x,
+                                     uint8_t* qweight_t, uint8_t* scale_t, uint8_t* qweight,
+                                     uint8_t* scale, mxq_stream_t stream);
+
 /* ------------------------------------------------------------------ NVFP4 */
 
 /* Workspace bytes nvfp4_quantize / nvfp4_amax need (per-CTA partial maxima of

@@ -22,7 +22,7 @@ import torch
 
 __all__ = [
     "MxqError", "lib", "library_path",
-    "mxfp8_quantize", "mxfp8_dequantize", "mxfp8_quantize_grouped",
+    "mxfp8_quantize", "mxfp8_dequantize", "mxfp8_quantize_grouped", "mxfp8_quantize_columnwise",
     "nvfp4_amax", "nvfp4_quantize", "nvfp4_dequantize",
     "swizzled_scale_bytes", "nvfp4_workspace_bytes",
     "as_float8_e4m3", "as_float8_e8m0", "as_float4_e2m1x2",
@@ -59,10 +59,12 @@ def _load() -> ctypes.CDLL:
     L.mxfp8_quantize.argtypes = [vp, i32, i64, i64, i64, vp, vp, vp, vp]
     L.mxfp8_dequantize.argtypes = [vp, vp, i64, i64, vp, i32, vp]
     L.mxfp8_quantize_grouped.argtypes = [i32, vp, vp, i64, i32, vp, vp, vp]
+    L.mxfp8_quantize_columnwise.argtypes = [vp, i32, i64, i64, i64, vp, vp, vp, vp, vp]
     L.nvfp4_amax.argtypes = [vp, i32, i64, i64, i64, vp, vp, sz, vp]
     L.nvfp4_quantize.argtypes = [vp, i32, i64, i64, i64, vp, vp, vp, vp, u32, vp, sz, vp]
     L.nvfp4_dequantize.argtypes = [vp, vp, vp, i64, i64, vp, i32, vp]
-    for f in ("mxfp8_quantize", "mxfp8_dequantize", "mxfp8_quantize_grouped", "nvfp4_amax",
+    for f in ("mxfp8_quantize", "mxfp8_dequantize", "mxfp8_quantize_grouped",
+              "mxfp8_quantize_columnwise", "nvfp4_amax",
               "nvfp4_quantize", "nvfp4_dequantize"):
         getattr(L, f).restype = i32
     return L
@@ -208,6 +210,32 @@ def mxfp8_quantize_grouped(xs: torch.Tensor | Sequence[torch.Tensor]):
     if stacked:
         return q.view(xs.shape), s.view(*xs.shape[:-1], N // 32)
     return q, s
+
+
+def mxfp8_quantize_columnwise(x: torch.Tensor, *, rowwise: bool = False):
+    """MXFP8 columnwise quantize (groups of 32 rows per column, rows past M
+    counting as zeros) of a bf16/fp32 tensor seen as [M, N].
+
+    Returns ``(qweight_t, scale_t)``: uint8 [N, M] E4M3 codes (the transposed
+    layout) and uint8 [N, ceil(M/32)] E8M0 bytes. With ``rowwise=True`` the
+    same launch also returns the rowwise ``(qweight, scale)`` of
+    ``mxfp8_quantize`` first: ``(qweight, scale, qweight_t, scale_t)``."""
+    _require_cuda(x)
+    dt = _dtype_code(x.dtype)
+    M, N, ld = _rows_view(x)
+    dev = x.device
+    q_t = torch.empty((N, M), dtype=torch.uint8, device=dev)
+    s_t = torch.empty((N, (M + 31) // 32), dtype=torch.uint8, device=dev)
+    q = s = None
+    if rowwise:
+        q = torch.empty((M, N), dtype=torch.uint8, device=dev)
+        s = torch.empty((M, N // 32), dtype=torch.uint8, device=dev)
+    _check("mxfp8_quantize_columnwise",
+           lib.mxfp8_quantize_columnwise(_ptr(x), dt, M, N, ld, _ptr(q_t), _ptr(s_t), _ptr(q),
+                                         _ptr(s), _stream(x)))
+    if rowwise:
+        return (q.view(*x.shape[:-1], N), s.view(*x.shape[:-1], N // 32), q_t, s_t)
+    return q_t, s_t
 
 
 # ------------------------------------------------------------------ NVFP4

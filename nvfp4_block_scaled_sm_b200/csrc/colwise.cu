@@ -1,0 +1,342 @@
+// colwise.cu -- MXFP8 columnwise quantize (groups of 32 consecutive rows of
+// one column, the operand layout of a backward GEMM), optionally fused with
+// the rowwise quantize so that the input is read once, for sm_100a.
+//
+// Method: each column group is quantized by the rowwise rule of mxfp8.cu
+// (NaN-ignoring amax, E8M0 byte = 127 / 254 / clamp(E(amax) - 8, 0, 254),
+// E4M3 RNE with saturation). Following the adapter contract of "PR #1935
+// 完整报告 -- Use TransformerEngine for MXFP8 quantization" (实现拆解 item 1:
+// zero-pad rows to a multiple of 32, quantize, crop back), rows past M count
+// as zeros in the last group of each column; for columnwise groups that
+// padding is part of the result. Outputs are transposed and cropped:
+// q_t [N, M] (q_t[c, r] is the code of x[r, c]) and scale_t [N, ceil(M/32)].
+//
+// Work split (HBM-bound: 2 bytes read, 1 + 1/32 written per bf16 element;
+// the fused mode writes 2 + 2/32): a CTA stages a tile of 128 rows x 256
+// bytes (128 bf16 or 64 fp32 columns) in shared memory with coalesced
+// 16-byte loads, rows past M and columns past N zero-filled; row pitch 272
+// bytes so that both phases below read shared memory without bank
+// conflicts.
+//  - Column phase: a thread owns one 4-byte word column (two bf16 columns or
+//    one fp32 column) and one 32-row group, reads its 32 words down the
+//    rows (consecutive lanes read consecutive words), reduces both bf16
+//    column maxima with one max.xorsign.abs.bf16x2 tree, and writes a 32-byte
+//    column group of q_t per column (a full 32-byte sector).
+//  - Row phase (fused mode): a thread owns one (row, 32-column) group of the
+//    tile, reads it as 16-byte shared loads and writes 32 bytes of q.
+// The transposed codes are staged in shared memory as well, so that every
+// q_t row segment of the tile (128 bytes) is written as a full line by 8
+// consecutive lanes, and the tile's 4 scale bytes of a column as one word.
+#include "common.cuh"
+
+#ifndef MXQ_COLWISE_ROWS_FAST
+#define MXQ_COLWISE_ROWS_FAST false  // CTA order: column tiles vary fastest
+#endif
+
+namespace mxq {
+namespace {
+
+constexpr int kTileRows = 128;
+constexpr int kRowBytes = 256;               // one tile row
+constexpr int kPitch = kRowBytes + 16;       // padded shared-memory row pitch
+constexpr int kWordCols = kRowBytes / 4;     // 64 word columns per tile
+constexpr int kOutPitch = kTileRows + 16;    // shared pitch of a transposed code row
+
+__device__ __forceinline__ uint32_t e8m0_byte(float amax) {
+  const uint32_t bits = __float_as_uint(amax);
+  const uint32_t E = bits >> 23;
+  uint32_t b = max(E, 8u) - 8u;
+  b = (E == 255) ? 254u : b;
+  b = (bits == 0) ? 127u : b;
+  return b;
+}
+
+__device__ __forceinline__ float pow2_quant(uint32_t b) {
+  return __uint_as_float(b == 254 ? 0x00400000u : (254u - b) << 23);
+}
+
+__device__ __forceinline__ uint32_t lds32(const uint8_t* p) {
+  uint32_t v;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(static_cast<uint32_t>(__cvta_generic_to_shared(p))));
+  return v;
+}
+
+__device__ __forceinline__ uint4 lds128(const uint8_t* p) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(static_cast<uint32_t>(__cvta_generic_to_shared(p))));
+  return v;
+}
+
+__device__ __forceinline__ void sts128(uint8_t* p, uint4 v) {
+  asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(
+                   static_cast<uint32_t>(__cvta_generic_to_shared(p))),
+               "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+               : "memory");
+}
+
+// Store the first `valid` (<= 32) bytes of a 32-byte group; 16-byte stores
+// when the destination is 16-byte aligned, byte stores otherwise.
+__device__ __forceinline__ void store_group(uint8_t* dst, const uint4& lo, const uint4& hi,
+                                            int valid, bool aligned) {
+  if (aligned && valid == 32) {
+    st_v4(dst, lo);
+    st_v4(dst + 16, hi);
+    return;
+  }
+  if (aligned && valid >= 16) {
+    st_v4(dst, lo);
+    const uint32_t w[4] = {hi.x, hi.y, hi.z, hi.w};
+    for (int i = 16; i < valid; i++) st_u8(dst + i, (w[(i - 16) >> 2] >> (8 * (i & 3))) & 0xffu);
+    return;
+  }
+  const uint32_t w[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+  for (int i = 0; i < valid; i++) st_u8(dst + i, (w[i >> 2] >> (8 * (i & 3))) & 0xffu);
+}
+
+struct ColArgs {
+  const uint8_t* x;      // input base (bytes)
+  int64_t ld_bytes;      // input row stride in bytes
+  int64_t M, N;
+  uint32_t n_ct;         // column tiles
+  uint32_t n_rt;         // row tiles
+  uint32_t gt;           // groups per column: ceil(M / 32)
+  uint8_t* q_t;          // [N, M]
+  uint8_t* scale_t;      // [N, gt]
+  uint8_t* q;            // [M, N] (fused mode)
+  uint8_t* scale;        // [M, N / 32] (fused mode)
+  bool q_t_aligned;      // every q_t row start is 16-byte aligned (M % 16 == 0)
+  bool scale_words;      // scale_t 4-byte aligned and ceil(M/32) % 4 == 0
+};
+
+// 32 E4M3 codes (as two 16-byte halves) of one column of 32 values given as
+// fp32, times the power-of-two multiplier `mul`.
+__device__ __forceinline__ void column_codes(const float (&f)[32], float mul, uint4& lo, uint4& hi) {
+  uint32_t c[16];
+#pragma unroll
+  for (int k = 0; k < 16; k++) {
+    const float2 p = mul2(f[2 * k], f[2 * k + 1], mul);
+    c[k] = cvt_e4m3x2(p.x, p.y);
+  }
+  lo = make_uint4(__byte_perm(c[0], c[1], 0x5410), __byte_perm(c[2], c[3], 0x5410),
+                  __byte_perm(c[4], c[5], 0x5410), __byte_perm(c[6], c[7], 0x5410));
+  hi = make_uint4(__byte_perm(c[8], c[9], 0x5410), __byte_perm(c[10], c[11], 0x5410),
+                  __byte_perm(c[12], c[13], 0x5410), __byte_perm(c[14], c[15], 0x5410));
+}
+
+template <typename InT, bool ROW, bool ROWS_FAST>
+__global__ void __launch_bounds__(kThreads)
+mxfp8_colwise_kernel(const __grid_constant__ ColArgs a) {
+  pdl_enter();
+  __shared__ __align__(16) uint8_t tile[kTileRows * kPitch];
+  constexpr int kEsize = sizeof(InT);
+  constexpr int kTileCols = kRowBytes / kEsize;
+  uint8_t* qs = tile;  // transposed codes, written once the input tile is consumed
+  static_assert(kTileCols * kOutPitch <= kTileRows * kPitch, "qs must fit in the tile");
+  __shared__ __align__(16) uint8_t ss[kTileCols * 4];          // scales [column][group]
+  const int t = threadIdx.x;
+  const uint32_t ct = ROWS_FAST ? blockIdx.x / a.n_rt : blockIdx.x % a.n_ct;
+  const uint32_t rt = ROWS_FAST ? blockIdx.x % a.n_rt : blockIdx.x / a.n_ct;
+  const int64_t r0 = int64_t(rt) * kTileRows, c0 = int64_t(ct) * kTileCols;
+  const int rows = a.M - r0 < kTileRows ? int(a.M - r0) : kTileRows;
+  const int row_bytes = (a.N - c0 < kTileCols ? int(a.N - c0) : kTileCols) * kEsize;  // multiple of 32
+
+  // stage the tile: 128 rows x 16 chunks of 16 bytes, 8 chunks per thread
+  uint4 buf[8];
+#pragma unroll
+  for (int i = 0; i < 8; i++) {
+    const int idx = i * kThreads + t, r = idx >> 4, ch = idx & 15;
+    if (r < rows && ch * 16 < row_bytes)
+      buf[i] = ld_nc_v4(a.x + (r0 + r) * a.ld_bytes + c0 * kEsize + ch * 16);
+    else
+      buf[i] = make_uint4(0, 0, 0, 0);
+  }
+#pragma unroll
+  for (int i = 0; i < 8; i++) {
+    const int idx = i * kThreads + t;
+    sts128(tile + (idx >> 4) * kPitch + (idx & 15) * 16, buf[i]);
+  }
+  __syncthreads();
+
+  // row phase (fused mode): (row, 32-column group) pairs of the tile
+  if constexpr (ROW) {
+    constexpr int kGroups = kTileCols / 32;             // 4 (bf16) or 2 (fp32)
+    constexpr int kPerThread = kTileRows * kGroups / kThreads;
+    const int64_t S = a.N / 32;
+#pragma unroll
+    for (int j = 0; j < kPerThread; j++) {
+      const int r = t & (kTileRows - 1);
+      const int k = (t >> 7) * kPerThread + j;
+      if (r < rows && k * 32 * kEsize < row_bytes) {
+        const uint8_t* src = tile + r * kPitch + k * 32 * kEsize;
+        float f[32];
+        float amax;
+        if constexpr (kEsize == 2) {
+          uint32_t w[16];
+#pragma unroll
+          for (int i = 0; i < 4; i++) {
+            const uint4 q4 = lds128(src + 16 * i);
+            w[4 * i] = q4.x; w[4 * i + 1] = q4.y; w[4 * i + 2] = q4.z; w[4 * i + 3] = q4.w;
+          }
+          uint32_t m = absmax_bf16x2(w[0], w[1]);
+#pragma unroll
+          for (int i = 2; i < 16; i++) m = absmax_bf16x2(m, w[i]);
+          m &= 0x7fff7fffu;
+          amax = fmaxf(fmaxf(bf16_lo(m), bf16_hi(m)), 0.0f);
+#pragma unroll
+          for (int i = 0; i < 16; i++) {
+            f[2 * i] = bf16_lo(w[i]);
+            f[2 * i + 1] = bf16_hi(w[i]);
+          }
+        } else {
+          amax = 0.0f;
+#pragma unroll
+          for (int i = 0; i < 8; i++) {
+            const uint4 q4 = lds128(src + 16 * i);
+            f[4 * i] = __uint_as_float(q4.x); f[4 * i + 1] = __uint_as_float(q4.y);
+            f[4 * i + 2] = __uint_as_float(q4.z); f[4 * i + 3] = __uint_as_float(q4.w);
+          }
+#pragma unroll
+          for (int i = 0; i < 32; i++) amax = fmaxf(amax, fabsf(f[i]));
+        }
+        const uint32_t b = e8m0_byte(amax);
+        uint4 lo, hi;
+        column_codes(f, pow2_quant(b), lo, hi);
+        uint8_t* dst = a.q + (r0 + r) * a.N + c0 + 32 * k;
+        st_v4(dst, lo);
+        st_v4(dst + 16, hi);
+        st_u8(a.scale + (r0 + r) * S + c0 / 32 + k, b);
+      }
+    }
+  }
+  // column phase: word column w, group g (rows 32g .. 32g + 31 of the tile).
+  // The codes stay in registers until every thread has read the input tile;
+  // then they go to the transposed tile qs[column][row], which reuses the
+  // input tile's shared memory.
+  {
+    const int w = t & (kWordCols - 1), g = t >> 6;
+    const bool active = 32 * g < rows && w * 4 < row_bytes;
+    uint4 code[kEsize == 2 ? 4 : 2];
+    uint32_t sb[2] = {0, 0};
+    if (active) {
+      uint32_t v[32];
+#pragma unroll
+      for (int i = 0; i < 32; i++) v[i] = lds32(tile + (32 * g + i) * kPitch + 4 * w);
+      float f[32];
+      if constexpr (kEsize == 2) {
+        uint32_t m = absmax_bf16x2(v[0], v[1]);
+#pragma unroll
+        for (int i = 2; i < 32; i++) m = absmax_bf16x2(m, v[i]);
+        m &= 0x7fff7fffu;
+        sb[0] = e8m0_byte(fmaxf(bf16_lo(m), 0.0f));
+        sb[1] = e8m0_byte(fmaxf(bf16_hi(m), 0.0f));
+#pragma unroll
+        for (int i = 0; i < 32; i++) f[i] = bf16_lo(v[i]);
+        column_codes(f, pow2_quant(sb[0]), code[0], code[1]);
+#pragma unroll
+        for (int i = 0; i < 32; i++) f[i] = bf16_hi(v[i]);
+        column_codes(f, pow2_quant(sb[1]), code[2], code[3]);
+      } else {
+        float amax = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 32; i++) {
+          f[i] = __uint_as_float(v[i]);
+          amax = fmaxf(amax, fabsf(f[i]));
+        }
+        sb[0] = e8m0_byte(amax);
+        column_codes(f, pow2_quant(sb[0]), code[0], code[1]);
+      }
+    }
+    __syncthreads();  // the input tile is dead from here on
+    if (active) {
+      constexpr int kCols = 4 / kEsize;  // columns per word
+#pragma unroll
+      for (int e = 0; e < kCols; e++) {
+        const int col = kCols * w + e;
+        sts128(qs + col * kOutPitch + 32 * g, code[2 * e]);
+        sts128(qs + col * kOutPitch + 32 * g + 16, code[2 * e + 1]);
+        ss[col * 4 + g] = uint8_t(sb[e]);
+      }
+    }
+  }
+  __syncthreads();
+
+  // write the transposed tile: 8 consecutive lanes write one q_t row's
+  // 128-byte segment (rows of the tile past M are not written)
+  {
+    const int cols = row_bytes / kEsize;
+#pragma unroll
+    for (int i = 0; i < kTileCols * 8 / kThreads; i++) {
+      const int idx = i * kThreads + t, col = idx >> 3, ch = idx & 7;
+      const int nbytes = rows - 16 * ch;  // valid bytes of this 16-byte chunk
+      if (col < cols && nbytes > 0) {
+        uint8_t* dst = a.q_t + (c0 + col) * a.M + r0 + 16 * ch;
+        const uint4 val = lds128(qs + col * kOutPitch + 16 * ch);
+        if (a.q_t_aligned && nbytes >= 16) {
+          st_v4(dst, val);
+        } else {
+          const uint32_t wv[4] = {val.x, val.y, val.z, val.w};
+          for (int j = 0; j < (nbytes < 16 ? nbytes : 16); j++)
+            st_u8(dst + j, (wv[j >> 2] >> (8 * (j & 3))) & 0xffu);
+        }
+      }
+    }
+    // scales: the tile's 4 groups of a column are 4 consecutive bytes of scale_t
+    if (t < cols) {
+      const int ng = (rows + 31) / 32;
+      uint8_t* dst = a.scale_t + (c0 + t) * a.gt + r0 / 32;
+      if (ng == 4 && a.scale_words) {
+        st_u32(dst, *reinterpret_cast<const uint32_t*>(ss + 4 * t));
+      } else {
+        for (int j = 0; j < ng; j++) st_u8(dst + j, ss[4 * t + j]);
+      }
+    }
+  }
+}
+
+}  // namespace
+}  // namespace mxq
+
+extern "C" mxq_status mxfp8_quantize_columnwise(const void* x, int dt, int64_t M, int64_t N,
+                                                int64_t ld_x, uint8_t* qweight_t,
+                                                uint8_t* scale_t, uint8_t* qweight,
+                                                uint8_t* scale, mxq_stream_t stream) {
+  using namespace mxq;
+  if (!valid_dtype(dt)) return MXQ_ERR_DTYPE;
+  const bool fused = qweight != nullptr || scale != nullptr;
+  if (M < 0 || N < 0 || N % 16 != 0 || ld_x < N || (fused && N % 32 != 0)) return MXQ_ERR_SHAPE;
+  if (M == 0 || N == 0) return MXQ_OK;
+  if (!x || !qweight_t || !scale_t || (fused && (!qweight || !scale))) return MXQ_ERR_NULL;
+  const int es = elem_size(dt);
+  if (!aligned16(x) || (uint64_t(ld_x) * es) % 16 != 0 || !aligned16(qweight_t) ||
+      (fused && !aligned16(qweight)))
+    return MXQ_ERR_ALIGN;
+  const uint64_t tile_cols = uint64_t(kRowBytes / es);
+  const uint64_t tile_rows = kTileRows;
+  const uint64_t n_rt = (uint64_t(M) + tile_rows - 1) / tile_rows;
+  const uint64_t n_ct = (uint64_t(N) + tile_cols - 1) / tile_cols;
+  if (n_rt * n_ct > 0x7fffffffull) return MXQ_ERR_SHAPE;
+  ColArgs a{};
+  a.x = static_cast<const uint8_t*>(x);
+  a.ld_bytes = ld_x * es;
+  a.M = M;
+  a.N = N;
+  a.n_ct = uint32_t(n_ct);
+  a.n_rt = uint32_t(n_rt);
+  a.gt = uint32_t((uint64_t(M) + 31) / 32);
+  a.q_t = qweight_t;
+  a.scale_t = scale_t;
+  a.q = qweight;
+  a.scale = scale;
+  a.q_t_aligned = (M % 16) == 0;
+  a.scale_words = (reinterpret_cast<uintptr_t>(scale_t) & 3u) == 0 && (a.gt & 3u) == 0;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const uint32_t grid = uint32_t(n_rt * n_ct);
+  if (dt == MXQ_BF16) {
+    return launched(fused ? launch_pdl(mxfp8_colwise_kernel<uint16_t, true, MXQ_COLWISE_ROWS_FAST>, grid, s, a)
+                          : launch_pdl(mxfp8_colwise_kernel<uint16_t, false, MXQ_COLWISE_ROWS_FAST>, grid, s, a));
+  }
+  return launched(fused ? launch_pdl(mxfp8_colwise_kernel<float, true, MXQ_COLWISE_ROWS_FAST>, grid, s, a)
+                        : launch_pdl(mxfp8_colwise_kernel<float, false, MXQ_COLWISE_ROWS_FAST>, grid, s, a));
+}

@@ -66,6 +66,7 @@ def lib() -> ctypes.CDLL:
             L.orc_mxfp8_quantize.argtypes = [vp, i32, i64, i64, i64, vp, vp]
             L.orc_mxfp8_dequantize.argtypes = [vp, vp, i64, i64, vp, i32]
             L.orc_swizzle_scales.argtypes = [vp, i64, i64, vp]
+            L.orc_mxfp8_quantize_colwise.argtypes = [vp, i32, i64, i64, i64, vp, vp]
             L.orc_nvfp4_global_amax.argtypes = [vp, i32, i64, i64, i64]
             L.orc_nvfp4_global_amax.restype = f32
             L.orc_nvfp4_quantize.argtypes = [vp, i32, i64, i64, i64, vp, vp, vp, i32]
@@ -75,6 +76,7 @@ def lib() -> ctypes.CDLL:
                 getattr(L, f).argtypes = [vp, i64, vp]
                 getattr(L, f).restype = None
             for f in ("orc_mxfp8_quantize", "orc_mxfp8_dequantize", "orc_swizzle_scales",
+                      "orc_mxfp8_quantize_colwise",
                       "orc_nvfp4_quantize", "orc_nvfp4_dequantize"):
                 getattr(L, f).restype = i32
             _lib = L
@@ -193,6 +195,19 @@ def mxfp8_quantize_padded(x: np.ndarray, row_align: int = 32):
     padded[:M] = flat
     q, s = mxfp8_quantize(padded)
     return q[:M].reshape(*lead, N), s[:M].reshape(*lead, N // 32)
+
+
+def mxfp8_quantize_colwise(x: np.ndarray):
+    """Columnwise MXFP8 of a 2-D input [M, N]: groups of 32 rows per column,
+    rows past M counting as zeros. Returns transposed, cropped outputs
+    (q_t uint8 [N, M], scale_t uint8 [N, ceil(M/32)])."""
+    a, dt = _as_input(x)
+    M, N = a.shape
+    q_t = np.empty((N, M), np.uint8)
+    s_t = np.empty((N, (M + 31) // 32), np.uint8)
+    _check(lib().orc_mxfp8_quantize_colwise(_ptr(a), dt, M, N, N, _ptr(q_t), _ptr(s_t)),
+           "mxfp8_quantize_colwise")
+    return q_t, s_t
 
 
 def mxfp8_dequantize(q: np.ndarray, s: np.ndarray, out: str = "bf16") -> np.ndarray:

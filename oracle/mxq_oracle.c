@@ -408,3 +408,41 @@ void orc_e8m0_from_amax_array(const double* a, int64_t n, uint8_t* out) {
 void orc_bf16_round_array(const double* d, int64_t n, uint16_t* out) {
   for (int64_t i = 0; i < n; i++) out[i] = orc_bf16_round(d[i]);
 }
+
+/* ------------------------------------------------------- MXFP8 columnwise */
+
+/* MXFP8 columnwise quantize of x [M, N] (row stride ld_x): groups of 32
+ * consecutive ROWS of one column, i.e. the rowwise quantize of the transposed
+ * tensor. Following the adapter contract ("PR #1935 完整报告 -- Use
+ * TransformerEngine for MXFP8 quantization", 实现拆解 item 1: pad rows to a
+ * multiple of 32 with zeros, quantize, crop back), rows past M count as zeros
+ * in the last group of each column. Outputs, transposed and cropped:
+ *   q_t     [N, M]            q_t[c, r] = E4M3 code of x[r, c]
+ *   scale_t [N, ceil(M/32)]   scale_t[c, j] = E8M0 byte of rows 32j..32j+31
+ * Each group is quantized by exactly the rowwise rule (orc_e8m0_from_amax,
+ * orc_e4m3_encode). */
+int orc_mxfp8_quantize_colwise(const void* x, int dt, int64_t M, int64_t N, int64_t ld_x,
+                               uint8_t* q_t, uint8_t* scale_t) {
+  if (dt != ORC_BF16 && dt != ORC_FP32) return ORC_ERR_DTYPE;
+  if (M < 0 || N < 0 || ld_x < N) return ORC_ERR_SHAPE;
+  int64_t G = (M + 31) / 32;
+  for (int64_t c = 0; c < N; c++) {
+    for (int64_t j = 0; j < G; j++) {
+      double amax = 0.0;
+      for (int i = 0; i < 32; i++) {
+        int64_t r = 32 * j + i;
+        double v = (r < M) ? load_elem(x, dt, r * ld_x + c) : 0.0;
+        if (!isnan(v) && fabs(v) > amax) amax = fabs(v);
+      }
+      uint8_t b = orc_e8m0_from_amax(amax);
+      scale_t[c * G + j] = b;
+      for (int i = 0; i < 32; i++) {
+        int64_t r = 32 * j + i;
+        if (r >= M) break;
+        double v = load_elem(x, dt, r * ld_x + c);
+        q_t[c * M + r] = orc_e4m3_encode(ldexp(v, 127 - (int)b));
+      }
+    }
+  }
+  return ORC_OK;
+}

@@ -212,3 +212,33 @@ def test_swizzle_inverse_recovers_compact(orc):
     mask = np.ones(out.size, bool)
     mask[off.reshape(-1)] = False
     assert np.all(out[mask] == 0)
+
+
+# -------------------------------------------------------------- columnwise
+
+@pytest.mark.parametrize("M,N", [(64, 96), (37, 32), (1, 16), (100, 48)])
+def test_colwise_is_rowwise_of_padded_transpose(orc, M, N):
+    """Columnwise groups of the row-padded tensor are the rowwise groups of
+    its transpose: compare with the pinned rowwise oracle and with the torch
+    formulation on the transposed, zero-padded input, then crop."""
+    x = W.planted(seed=M * 3 + N, M=max(M, 8), N=max(N, 32))[:M, :N]
+    Mp = (M + 31) // 32 * 32
+    padded = np.zeros((Mp, N), np.uint16)
+    padded[:M] = x
+    xt = np.ascontiguousarray(padded.T)
+    q_t, s_t = orc.mxfp8_quantize_colwise(np.ascontiguousarray(x))
+    q_r, s_r = orc.mxfp8_quantize(xt)
+    q_torch, s_torch = refs.mxfp8_quantize_torch(xt)
+    assert np.array_equal(q_t, q_r[:, :M]) and np.array_equal(s_t, s_r)
+    assert np.array_equal(q_t, q_torch[:, :M]) and np.array_equal(s_t, s_torch)
+
+
+def test_colwise_padding_only_touches_last_group(orc):
+    """Zero padding never raises an amax: for M a multiple of 32 the result
+    does not depend on padding at all, and cropping a taller tensor with the
+    same first rows changes only the last group of each column."""
+    x = W.activation(seed=91, M=96, N=64)
+    q_full, s_full = orc.mxfp8_quantize_colwise(x)
+    q_cut, s_cut = orc.mxfp8_quantize_colwise(np.ascontiguousarray(x[:70]))
+    assert np.array_equal(q_cut[:, :64], q_full[:, :64])
+    assert np.array_equal(s_cut[:, :2], s_full[:, :2])
