@@ -67,6 +67,10 @@ def lib() -> ctypes.CDLL:
             L.orc_mxfp8_dequantize.argtypes = [vp, vp, i64, i64, vp, i32]
             L.orc_swizzle_scales.argtypes = [vp, i64, i64, vp]
             L.orc_mxfp8_quantize_colwise.argtypes = [vp, i32, i64, i64, i64, vp, vp]
+            L.orc_mxfp4_quantize.argtypes = [vp, i32, i64, i64, i64, vp, vp]
+            L.orc_mxfp4_dequantize.argtypes = [vp, vp, i64, i64, vp, i32]
+            L.orc_e8m0_from_amax_emax.argtypes = [f64, i32]
+            L.orc_e8m0_from_amax_emax.restype = u8
             L.orc_nvfp4_global_amax.argtypes = [vp, i32, i64, i64, i64]
             L.orc_nvfp4_global_amax.restype = f32
             L.orc_nvfp4_quantize.argtypes = [vp, i32, i64, i64, i64, vp, vp, vp, i32]
@@ -76,7 +80,7 @@ def lib() -> ctypes.CDLL:
                 getattr(L, f).argtypes = [vp, i64, vp]
                 getattr(L, f).restype = None
             for f in ("orc_mxfp8_quantize", "orc_mxfp8_dequantize", "orc_swizzle_scales",
-                      "orc_mxfp8_quantize_colwise",
+                      "orc_mxfp8_quantize_colwise", "orc_mxfp4_quantize", "orc_mxfp4_dequantize",
                       "orc_nvfp4_quantize", "orc_nvfp4_dequantize"):
                 getattr(L, f).restype = i32
             _lib = L
@@ -244,6 +248,45 @@ def mxfp8_quantize_grouped(xs):
         qs.append(q)
         ss.append(s)
     return np.concatenate(qs, 0), np.concatenate(ss, 0)
+
+
+# -------------------------------------------------------------------- MXFP4
+
+def e8m0_from_amax_emax(amax: float, emax: int) -> int:
+    return int(lib().orc_e8m0_from_amax_emax(float(amax), emax))
+
+
+def mxfp4_quantize(x: np.ndarray):
+    """Returns (packed uint8 [M, N/2], scale uint8 [M, N/32])."""
+    a, dt = _as_input(x)
+    M, N = a.shape
+    packed = np.empty((M, N // 2), np.uint8)
+    s = np.empty((M, N // 32), np.uint8)
+    _check(lib().orc_mxfp4_quantize(_ptr(a), dt, M, N, N, _ptr(packed), _ptr(s)), "mxfp4_quantize")
+    return packed, s
+
+
+def mxfp4_dequantize(packed: np.ndarray, s: np.ndarray, out: str = "bf16") -> np.ndarray:
+    packed = np.ascontiguousarray(packed, np.uint8)
+    s = np.ascontiguousarray(s, np.uint8)
+    M, half = packed.shape
+    N = half * 2
+    y = np.empty((M, N), np.uint16 if out == "bf16" else np.float32)
+    _check(lib().orc_mxfp4_dequantize(_ptr(packed), _ptr(s), M, N, _ptr(y), BF16 if out == "bf16" else FP32),
+           "mxfp4_dequantize")
+    return y
+
+
+def fake_quantize(x: np.ndarray, fmt: str, out: str = "bf16") -> np.ndarray:
+    """QAT simulate ("V4 mxfp4 #1372": mxfp4_simulate_qat(kv, 32)): the
+    dequantization of the quantization, for fmt "mxfp8" or "mxfp4"."""
+    if fmt == "mxfp8":
+        q, s = mxfp8_quantize(x)
+        return mxfp8_dequantize(q, s, out=out)
+    if fmt == "mxfp4":
+        p, s = mxfp4_quantize(x)
+        return mxfp4_dequantize(p, s, out=out)
+    raise ValueError(fmt)
 
 
 # -------------------------------------------------------------------- NVFP4

@@ -446,3 +446,72 @@ int orc_mxfp8_quantize_colwise(const void* x, int dt, int64_t M, int64_t N, int6
   }
   return ORC_OK;
 }
+
+/* ------------------------------------------------------------------ MXFP4 */
+
+/* E8M0 byte of a group under the OCP MX rule for an element format whose
+ * largest normal has exponent emax: scale = 2^(floor(log2 amax) - emax),
+ * byte = 127 + that exponent clamped to [0, 254]; 127 for amax == 0, 254 for
+ * amax == inf. emax = 8 gives orc_e8m0_from_amax (E4M3), emax = 2 the E2M1
+ * rule (largest normal 6 = 1.5 * 2^2). */
+uint8_t orc_e8m0_from_amax_emax(double amax, int emax) {
+  if (amax == 0.0) return 127;
+  if (isinf(amax)) return 254;
+  int e;
+  frexp(amax, &e);
+  long b = 127 + ((long)e - 1) - emax;
+  if (b < 0) b = 0;
+  if (b > 254) b = 254;
+  return (uint8_t)b;
+}
+
+/* MXFP4 rowwise quantize ("V4 mxfp4 #1372": mxfp4_simulate_qat(kv, 32), E2M1
+ * stored two per byte as float4_e2m1fn_x2): groups of 32 consecutive
+ * elements along the last dim; amax over non-NaN elements; byte by the OCP
+ * MX rule with emax 2; code = E2M1(x * 2^(127 - byte)) (RNE, |.| > 6 -> 6,
+ * NaN -> +6, signed zeros kept); packed[r, k] = q[r, 2k] | q[r, 2k+1] << 4.
+ * Readings: the MX scale rule of the MXFP8 path carried over with E2M1's emax;
+ * NaN as in the NVFP4 path. N must be a multiple of 32. */
+int orc_mxfp4_quantize(const void* x, int dt, int64_t M, int64_t N, int64_t ld_x,
+                       uint8_t* packed, uint8_t* scale) {
+  if (dt != ORC_BF16 && dt != ORC_FP32) return ORC_ERR_DTYPE;
+  if (M < 0 || N < 0 || N % 32 != 0 || ld_x < N) return ORC_ERR_SHAPE;
+  int64_t S = N / 32;
+  for (int64_t r = 0; r < M; r++) {
+    for (int64_t j = 0; j < S; j++) {
+      double amax = 0.0;
+      for (int i = 0; i < 32; i++) {
+        double v = load_elem(x, dt, r * ld_x + 32 * j + i);
+        if (!isnan(v) && fabs(v) > amax) amax = fabs(v);
+      }
+      uint8_t b = orc_e8m0_from_amax_emax(amax, 2);
+      scale[r * S + j] = b;
+      uint8_t codes[32];
+      for (int i = 0; i < 32; i++) {
+        double v = load_elem(x, dt, r * ld_x + 32 * j + i);
+        codes[i] = orc_e2m1_encode(ldexp(v, 127 - (int)b));
+      }
+      for (int k = 0; k < 16; k++)
+        packed[r * (N / 2) + 16 * j + k] = (uint8_t)(codes[2 * k] | (codes[2 * k + 1] << 4));
+    }
+  }
+  return ORC_OK;
+}
+
+/* MXFP4 dequantize: y = decode_e2m1(q) * 2^(scale - 127), exact in double,
+ * then fp32 (exact except overflow to inf at byte 254) or bf16 (RNE). */
+int orc_mxfp4_dequantize(const uint8_t* packed, const uint8_t* scale, int64_t M, int64_t N,
+                         void* y, int out_dt) {
+  if (out_dt != ORC_BF16 && out_dt != ORC_FP32) return ORC_ERR_DTYPE;
+  if (M < 0 || N < 0 || N % 32 != 0) return ORC_ERR_SHAPE;
+  int64_t S = N / 32;
+  for (int64_t r = 0; r < M; r++) {
+    for (int64_t c = 0; c < N; c++) {
+      uint8_t byte = packed[r * (N / 2) + c / 2];
+      uint8_t code = (c % 2 == 0) ? (byte & 0x0F) : (byte >> 4);
+      double d = orc_e2m1_decode(code) * orc_e8m0_value(scale[r * S + c / 32]);
+      store_out(y, out_dt, r * N + c, d);
+    }
+  }
+  return ORC_OK;
+}
