@@ -4,6 +4,8 @@
  *
  *   MXFP8 rowwise: groups of 32 consecutive elements along the last dim share
  *   one power-of-two E8M0 scale; elements are FP8 E4M3.
+ *   MXFP4 rowwise: the same power-of-two E8M0 scale per group of 32, with
+ *   FP4 E2M1 elements packed two per byte.
  *   NVFP4 two-level: an fp32 global scale times per-16-element E4M3 block
  *   scales; elements are FP4 E2M1, packed two per byte.
  *
@@ -18,8 +20,8 @@
  *    E2M1 stored two per byte (float4_e2m1fn_x2, last dim N//2), with
  *    N % block_size == 0.
  *  - "Add FP8, NVFP4, and QARL training and export", review "What looked
- *    solid": NVFP4 two-level global + FP8-block scaling, "effective =
- *    block_scale * global_scale", zero blocks guarded.
+ *    solid": NVFP4 two-level global + FP8-block scaling, the effective
+ *    scale being the block scale times the global scale, zero blocks guarded.
  *  - "feat(training): MXFP8 混合精度训练落地", and the same xorl review,
  *    item 2: failures are visible, never a silent downgrade -- this library
  *    has no fallback path; every error is a status code.
@@ -73,11 +75,15 @@ typedef enum {
 
 typedef enum { MXQ_BF16 = 0, MXQ_FP32 = 1 } mxq_dtype;
 
+/* MX element formats (mx_fake_quantize). */
+typedef enum { MXQ_FMT_MXFP8 = 0, MXQ_FMT_MXFP4 = 1 } mxq_mx_format;
+
 #define MXQ_ABI_VERSION 1
 #define MXQ_MXFP8_GROUP 32
 #define MXQ_NVFP4_BLOCK 16
 #define MXQ_GROUPED_MAX_EXPERTS 1024
 #define MXQ_NVFP4_GLOBAL_GIVEN 1u
+#define MXQ_NVFP4_MAX_SLICES 1024
 
 /* Version of this ABI (MXQ_ABI_VERSION of the built library). */
 int mxq_abi_version(void);
@@ -158,6 +164,54 @@ mxq_status mxfp8_quantize_columnwise(const void* x, int dt, int64_t M, int64_t N
                                      uint8_t* qweight_t, uint8_t* scale_t, uint8_t* qweight,
                                      uint8_t* scale, mxq_stream_t stream);
 
+/* ------------------------------------------------------------------ MXFP4 */
+
+/* MXFP4 rowwise quantize ("V4 mxfp4 #1372": E8M0 power-of-two scales per
+ * group of 32, E2M1 elements stored as float4_e2m1fn_x2 with last dim N/2;
+ * the QAT simulation mxfp4_simulate_qat(kv, 32) uses the same groups).
+ * The rule of mxfp8_quantize with E2M1 in place of E4M3: byte = 127 if
+ * amax == 0, 254 if amax is infinite, else clamp(floor(log2 amax) - 2 + 127,
+ * 0, 254) (2 = exponent of E2M1's largest value, 6 = 1.5 * 2^2); the code is
+ * E2M1(x * 2^(127 - byte)) rounded to nearest even, |.| > 6 saturating to 6,
+ * NaN -> +6 (0x7), zero results keeping the sign.
+ *  x        [M, N] bf16 or fp32 (dt), row stride ld_x elements; N % 32 == 0.
+ *  packed   [M, N/2] uint8: element 2k in the low nibble, 2k+1 in the high.
+ *  scale    [M, N/32] uint8 E8M0 bytes, compact.
+ *  scale_swz  NULL, or mxq_swizzled_scale_bytes(M, N/32) bytes receiving the
+ *           scales in the 128x4-tile layout described at mxfp8_quantize.
+ * Errors as for mxfp8_quantize. */
+mxq_status mxfp4_quantize(const void* x, int dt, int64_t M, int64_t N, int64_t ld_x,
+                          uint8_t* packed, uint8_t* scale, uint8_t* scale_swz,
+                          mxq_stream_t stream);
+
+/* MXFP4 dequantize: y[r, c] = decode_e2m1(code) * 2^(scale[r, c/32] - 127),
+ * exact in fp32 (overflow to inf only for scale bytes above 252), written as
+ * fp32 or bf16 (round to nearest even). Scale byte 255 gives NaN (0x7FC0 /
+ * 0x7FC00000). packed [M, N/2], scale [M, N/32], y [M, N] of out_dt. */
+mxq_status mxfp4_dequantize(const uint8_t* packed, const uint8_t* scale, int64_t M, int64_t N,
+                            void* y, int out_dt, mxq_stream_t stream);
+
+/* Grouped MXFP4 quantize of E expert tensors in one launch: arguments and
+ * layout as for mxfp8_quantize_grouped, outputs packed [sum rows, N/2] and
+ * scale [sum rows, N/32], identical to mxfp4_quantize of the stacked rows. */
+mxq_status mxfp4_quantize_grouped(int32_t E, const void* const* xs, const int64_t* rows,
+                                  int64_t N, int dt, uint8_t* packed, uint8_t* scale,
+                                  mxq_stream_t stream);
+
+/* ------------------------------------------------------- fake quantize */
+
+/* Fused fake-quantize (QAT simulation: "V4 mxfp4 #1372", mxfp4_simulate_qat;
+ * "PR #1935 完整报告 ...", the round trip through (qweight, scale)):
+ * y = dequantize(quantize(x)) for fmt MXQ_FMT_MXFP8 or MXQ_FMT_MXFP4, in one
+ * pass that reads x once and writes y once; the codes and scales are never
+ * stored. Bytes of y are identical to mxfp8_/mxfp4_quantize followed by the
+ * matching dequantize with out_dt.
+ *  x  [M, N] bf16 or fp32 (dt), row stride ld_x; N % 32 == 0.
+ *  y  [M, N] of out_dt, contiguous, 16-byte aligned; may not overlap x.
+ * Errors: unknown fmt -> MXQ_ERR_ARG; otherwise as for mxfp8_quantize. */
+mxq_status mx_fake_quantize(int fmt, const void* x, int dt, int64_t M, int64_t N, int64_t ld_x,
+                            void* y, int out_dt, mxq_stream_t stream);
+
 /* ------------------------------------------------------------------ NVFP4 */
 
 /* Workspace bytes nvfp4_quantize / nvfp4_amax need (per-CTA partial maxima of
@@ -215,6 +269,48 @@ mxq_status nvfp4_quantize(const void* x, int dt, int64_t M, int64_t N, int64_t l
 mxq_status nvfp4_quantize_noalloc(const void* x, int dt, int64_t M, int64_t N, int64_t ld_x,
                                   uint8_t* packed, uint8_t* block_scale, float* global_scale,
                                   const float* amax_in, uint32_t flags, mxq_stream_t stream);
+
+/* ------------------------------------------- NVFP4, one global scale per slice */
+
+/* Workspace bytes of nvfp4_quantize_sliced / nvfp4_amax_sliced:
+ * 4 * (2048 + n_slices); 0 for n_slices outside [1, MXQ_NVFP4_MAX_SLICES]. */
+size_t mxq_nvfp4_sliced_workspace_bytes(int32_t n_slices);
+
+/* NVFP4 quantize of x [M, N] cut into n_slices consecutive row ranges, each
+ * with its own global scale ("Add FP8, NVFP4, and QARL training and export",
+ * review: _nvfp4_block_quantize_per_slice, weight_scale_2 per expert;
+ * non-blocking item 3: a fused gate/up weight takes one global scale per
+ * half during QAT and one shared scale per expert at export). Each slice is
+ * quantized exactly as nvfp4_quantize would quantize a tensor holding only
+ * its rows: g_s = A_s / 2688 with A_s the slice's amax, then the block rule
+ * of nvfp4_quantize with g_s. Typical slicings of a stacked expert weight
+ * [E, R, N]: R rows per slice (one scale per expert), or R/2 (one scale per
+ * gate / up half of a fused gate/up weight whose first R/2 rows are the
+ * gate).
+ *  slice_rows    HOST array of n_slices row counts (>= 0, summing to M), read
+ *                during the call only; 1 <= n_slices <= MXQ_NVFP4_MAX_SLICES.
+ *  packed, block_scale  as for nvfp4_quantize ([M, N/2], [M, N/16]).
+ *  global_scales device fp32 [n_slices]: written (g_s; 0 for an empty slice),
+ *                or read with flags & MXQ_NVFP4_GLOBAL_GIVEN.
+ *  amax_in       NULL, or device fp32 [n_slices] slice amaxes (for example
+ *                all-reduced across ranks): g_s = amax_in[s] / 2688.
+ *  workspace     >= mxq_nvfp4_sliced_workspace_bytes(n_slices), when the
+ *                slice amaxes are computed here.
+ * M == 0 or N == 0 writes nothing. Errors as for nvfp4_quantize, and
+ * MXQ_ERR_SHAPE for a bad slicing. Two launches (amax pass, block pass), or
+ * one with GLOBAL_GIVEN or amax_in. */
+mxq_status nvfp4_quantize_sliced(const void* x, int dt, int64_t M, int64_t N, int64_t ld_x,
+                                 int32_t n_slices, const int64_t* slice_rows, uint8_t* packed,
+                                 uint8_t* block_scale, float* global_scales,
+                                 const float* amax_in, uint32_t flags, void* workspace,
+                                 size_t ws_bytes, mxq_stream_t stream);
+
+/* Slice amaxes (max |x| over each slice's non-NaN elements, 0 for an empty
+ * slice) into device fp32 amax[n_slices]: the amax pass of
+ * nvfp4_quantize_sliced on its own. */
+mxq_status nvfp4_amax_sliced(const void* x, int dt, int64_t M, int64_t N, int64_t ld_x,
+                             int32_t n_slices, const int64_t* slice_rows, float* amax,
+                             void* workspace, size_t ws_bytes, mxq_stream_t stream);
 
 /* NVFP4 dequantize: eff = decode_e4m3(s_b) * g and y = decode_e2m1(q) * eff,
  * both fp32 products, written as fp32 or bf16 (RNE). global_scale is a device

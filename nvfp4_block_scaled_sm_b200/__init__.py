@@ -1,4 +1,4 @@
-"""Block-scaled low-precision quantization (MXFP8 / NVFP4) for NVIDIA B200.
+"""Block-scaled low-precision quantization (MXFP8 / MXFP4 / NVFP4) for NVIDIA B200.
 
 Python binding of ``libmxq.so`` (C ABI declared in ``include/mxq.h``). This
 module only marshals arguments: it allocates outputs with torch on the input's
@@ -23,7 +23,9 @@ import torch
 __all__ = [
     "MxqError", "lib", "library_path",
     "mxfp8_quantize", "mxfp8_dequantize", "mxfp8_quantize_grouped", "mxfp8_quantize_columnwise",
+    "mxfp4_quantize", "mxfp4_dequantize", "mxfp4_quantize_grouped", "mx_fake_quantize",
     "nvfp4_amax", "nvfp4_quantize", "nvfp4_dequantize",
+    "nvfp4_amax_sliced", "nvfp4_quantize_sliced", "nvfp4_quantize_experts",
     "swizzled_scale_bytes", "nvfp4_workspace_bytes",
     "as_float8_e4m3", "as_float8_e8m0", "as_float4_e2m1x2",
 ]
@@ -32,6 +34,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 library_path = os.path.join(_HERE, "libmxq.so")
 
 BF16, FP32 = 0, 1
+FMT_MXFP8, FMT_MXFP4 = 0, 1
 NVFP4_GLOBAL_GIVEN = 1
 
 
@@ -60,11 +63,22 @@ def _load() -> ctypes.CDLL:
     L.mxfp8_dequantize.argtypes = [vp, vp, i64, i64, vp, i32, vp]
     L.mxfp8_quantize_grouped.argtypes = [i32, vp, vp, i64, i32, vp, vp, vp]
     L.mxfp8_quantize_columnwise.argtypes = [vp, i32, i64, i64, i64, vp, vp, vp, vp, vp]
+    L.mxfp4_quantize.argtypes = [vp, i32, i64, i64, i64, vp, vp, vp, vp]
+    L.mxfp4_dequantize.argtypes = [vp, vp, i64, i64, vp, i32, vp]
+    L.mxfp4_quantize_grouped.argtypes = [i32, vp, vp, i64, i32, vp, vp, vp]
+    L.mx_fake_quantize.argtypes = [i32, vp, i32, i64, i64, i64, vp, i32, vp]
     L.nvfp4_amax.argtypes = [vp, i32, i64, i64, i64, vp, vp, sz, vp]
     L.nvfp4_quantize.argtypes = [vp, i32, i64, i64, i64, vp, vp, vp, vp, u32, vp, sz, vp]
     L.nvfp4_dequantize.argtypes = [vp, vp, vp, i64, i64, vp, i32, vp]
+    L.mxq_nvfp4_sliced_workspace_bytes.argtypes = [i32]
+    L.mxq_nvfp4_sliced_workspace_bytes.restype = sz
+    L.nvfp4_quantize_sliced.argtypes = [vp, i32, i64, i64, i64, i32, vp, vp, vp, vp, vp, u32, vp,
+                                        sz, vp]
+    L.nvfp4_amax_sliced.argtypes = [vp, i32, i64, i64, i64, i32, vp, vp, vp, sz, vp]
     for f in ("mxfp8_quantize", "mxfp8_dequantize", "mxfp8_quantize_grouped",
-              "mxfp8_quantize_columnwise", "nvfp4_amax",
+              "mxfp8_quantize_columnwise", "mxfp4_quantize", "mxfp4_dequantize",
+              "mxfp4_quantize_grouped", "mx_fake_quantize", "nvfp4_amax",
+              "nvfp4_quantize_sliced", "nvfp4_amax_sliced",
               "nvfp4_quantize", "nvfp4_dequantize"):
         getattr(L, f).restype = i32
     return L
@@ -136,52 +150,38 @@ def nvfp4_workspace_bytes(M: int = 0, N: int = 0) -> int:
 
 # ------------------------------------------------------------------ MXFP8
 
-def mxfp8_quantize(x: torch.Tensor, *, swizzled: bool = False):
-    """MXFP8 rowwise quantize of a bf16/fp32 CUDA tensor.
-
-    Returns ``(qweight, scale)``: uint8 E4M3 codes shaped like ``x`` and uint8
-    E8M0 bytes shaped ``x.shape[:-1] + (N // 32,)``; with ``swizzled=True`` a
-    third flat uint8 tensor holds the scales in the 128x4-tile layout read by
-    block-scaled tensor-core MMA.
-    """
+def _mx_quantize(fn: str, x: torch.Tensor, swizzled: bool, per_byte: int):
     _require_cuda(x)
     dt = _dtype_code(x.dtype)
     M, N, ld = _rows_view(x)
-    q = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
+    q = torch.empty((*x.shape[:-1], N // per_byte), dtype=torch.uint8, device=x.device)
     s = torch.empty((*x.shape[:-1], N // 32), dtype=torch.uint8, device=x.device)
     swz = None
     if swizzled:
         swz = torch.empty(max(swizzled_scale_bytes(M, N // 32), 0), dtype=torch.uint8,
                           device=x.device)
-    _check("mxfp8_quantize", lib.mxfp8_quantize(_ptr(x), dt, M, N, ld, _ptr(q), _ptr(s),
-                                                _ptr(swz), _stream(x)))
+    _check(fn, getattr(lib, fn)(_ptr(x), dt, M, N, ld, _ptr(q), _ptr(s), _ptr(swz), _stream(x)))
     return (q, s, swz) if swizzled else (q, s)
 
 
-def mxfp8_dequantize(qweight: torch.Tensor, scale: torch.Tensor,
-                     dtype: torch.dtype = torch.bfloat16) -> torch.Tensor:
-    """decode(q) * 2^(scale - 127), as bf16 (RNE) or fp32 (exact)."""
-    _require_cuda(qweight, scale)
-    if qweight.dtype != torch.uint8 or scale.dtype != torch.uint8:
-        raise TypeError("qweight and scale must be uint8")
-    if not (qweight.is_contiguous() and scale.is_contiguous()):
-        raise ValueError("qweight and scale must be contiguous")
-    N = qweight.shape[-1]
-    M = qweight.numel() // N if N else 0
+def _mx_dequantize(fn: str, q: torch.Tensor, scale: torch.Tensor, dtype: torch.dtype,
+                   per_byte: int) -> torch.Tensor:
+    _require_cuda(q, scale)
+    if q.dtype != torch.uint8 or scale.dtype != torch.uint8:
+        raise TypeError("codes and scale must be uint8")
+    if not (q.is_contiguous() and scale.is_contiguous()):
+        raise ValueError("codes and scale must be contiguous")
+    N = q.shape[-1] * per_byte
+    M = q.numel() * per_byte // N if N else 0
     if scale.numel() != M * (N // 32):
-        raise ValueError("scale does not match qweight")
-    y = torch.empty(qweight.shape, dtype=dtype, device=qweight.device)
-    _check("mxfp8_dequantize", lib.mxfp8_dequantize(_ptr(qweight), _ptr(scale), M, N, _ptr(y),
-                                                    _dtype_code(dtype), _stream(qweight)))
+        raise ValueError("scale does not match the codes")
+    y = torch.empty((*q.shape[:-1], N), dtype=dtype, device=q.device)
+    _check(fn, getattr(lib, fn)(_ptr(q), _ptr(scale), M, N, _ptr(y), _dtype_code(dtype),
+                                _stream(q)))
     return y
 
 
-def mxfp8_quantize_grouped(xs: torch.Tensor | Sequence[torch.Tensor]):
-    """Grouped MXFP8 of expert tensors sharing N, in one launch.
-
-    ``xs`` is a stacked [E, M, N] tensor (results [E, M, N] and [E, M, N/32])
-    or a sequence of contiguous [M_e, N] tensors (results concatenated along
-    rows: [sum M_e, N] and [sum M_e, N/32])."""
+def _mx_quantize_grouped(fn: str, xs, per_byte: int):
     stacked = isinstance(xs, torch.Tensor)
     parts = list(xs.unbind(0)) if stacked else list(xs)
     if not parts:
@@ -199,17 +199,42 @@ def mxfp8_quantize_grouped(xs: torch.Tensor | Sequence[torch.Tensor]):
     E = len(parts)
     total = sum(rows)
     dev = parts[0].device
-    q = torch.empty((total, N), dtype=torch.uint8, device=dev)
+    q = torch.empty((total, N // per_byte), dtype=torch.uint8, device=dev)
     s = torch.empty((total, N // 32), dtype=torch.uint8, device=dev)
     ptrs = (ctypes.c_void_p * E)(*[p.data_ptr() for p in parts])
     rws = (ctypes.c_int64 * E)(*rows)
-    _check("mxfp8_quantize_grouped",
-           lib.mxfp8_quantize_grouped(E, ctypes.cast(ptrs, ctypes.c_void_p),
-                                      ctypes.cast(rws, ctypes.c_void_p), N, dt, _ptr(q), _ptr(s),
-                                      _stream(parts[0])))
+    _check(fn, getattr(lib, fn)(E, ctypes.cast(ptrs, ctypes.c_void_p),
+                                ctypes.cast(rws, ctypes.c_void_p), N, dt, _ptr(q), _ptr(s),
+                                _stream(parts[0])))
     if stacked:
-        return q.view(xs.shape), s.view(*xs.shape[:-1], N // 32)
+        return q.view(*xs.shape[:-1], N // per_byte), s.view(*xs.shape[:-1], N // 32)
     return q, s
+
+
+def mxfp8_quantize(x: torch.Tensor, *, swizzled: bool = False):
+    """MXFP8 rowwise quantize of a bf16/fp32 CUDA tensor.
+
+    Returns ``(qweight, scale)``: uint8 E4M3 codes shaped like ``x`` and uint8
+    E8M0 bytes shaped ``x.shape[:-1] + (N // 32,)``; with ``swizzled=True`` a
+    third flat uint8 tensor holds the scales in the 128x4-tile layout read by
+    block-scaled tensor-core MMA.
+    """
+    return _mx_quantize("mxfp8_quantize", x, swizzled, 1)
+
+
+def mxfp8_dequantize(qweight: torch.Tensor, scale: torch.Tensor,
+                     dtype: torch.dtype = torch.bfloat16) -> torch.Tensor:
+    """decode(q) * 2^(scale - 127), as bf16 (RNE) or fp32 (exact)."""
+    return _mx_dequantize("mxfp8_dequantize", qweight, scale, dtype, 1)
+
+
+def mxfp8_quantize_grouped(xs: torch.Tensor | Sequence[torch.Tensor]):
+    """Grouped MXFP8 of expert tensors sharing N, in one launch.
+
+    ``xs`` is a stacked [E, M, N] tensor (results [E, M, N] and [E, M, N/32])
+    or a sequence of contiguous [M_e, N] tensors (results concatenated along
+    rows: [sum M_e, N] and [sum M_e, N/32])."""
+    return _mx_quantize_grouped("mxfp8_quantize_grouped", xs, 1)
 
 
 def mxfp8_quantize_columnwise(x: torch.Tensor, *, rowwise: bool = False):
@@ -236,6 +261,48 @@ def mxfp8_quantize_columnwise(x: torch.Tensor, *, rowwise: bool = False):
     if rowwise:
         return (q.view(*x.shape[:-1], N), s.view(*x.shape[:-1], N // 32), q_t, s_t)
     return q_t, s_t
+
+
+# ------------------------------------------------------------------ MXFP4
+
+def mxfp4_quantize(x: torch.Tensor, *, swizzled: bool = False):
+    """MXFP4 rowwise quantize ("V4 mxfp4 #1372"): E8M0 scale per 32 elements
+    (emax 2), E2M1 codes packed two per byte, even element in the low nibble.
+
+    Returns ``(packed, scale)``: uint8 ``x.shape[:-1] + (N // 2,)`` and uint8
+    ``x.shape[:-1] + (N // 32,)``; ``swizzled=True`` adds the 128x4-tile
+    scale layout as a third, flat tensor."""
+    return _mx_quantize("mxfp4_quantize", x, swizzled, 2)
+
+
+def mxfp4_dequantize(packed: torch.Tensor, scale: torch.Tensor,
+                     dtype: torch.dtype = torch.bfloat16) -> torch.Tensor:
+    """decode_e2m1(code) * 2^(scale - 127), as bf16 (RNE) or fp32 (exact)."""
+    return _mx_dequantize("mxfp4_dequantize", packed, scale, dtype, 2)
+
+
+def mxfp4_quantize_grouped(xs: torch.Tensor | Sequence[torch.Tensor]):
+    """Grouped MXFP4 of expert tensors sharing N, in one launch (layout as
+    :func:`mxfp8_quantize_grouped`, codes packed [.., N // 2])."""
+    return _mx_quantize_grouped("mxfp4_quantize_grouped", xs, 2)
+
+
+def mx_fake_quantize(x: torch.Tensor, fmt: str = "mxfp4",
+                     dtype: torch.dtype | None = None) -> torch.Tensor:
+    """QAT simulation: dequantize(quantize(x)) for ``fmt`` "mxfp8" or
+    "mxfp4" in one pass (codes never stored), as ``dtype`` (default: the
+    dtype of ``x``)."""
+    formats = {"mxfp8": FMT_MXFP8, "mxfp4": FMT_MXFP4}
+    if fmt not in formats:
+        raise ValueError(f"fmt must be one of {sorted(formats)}")
+    _require_cuda(x)
+    dt = _dtype_code(x.dtype)
+    dtype = x.dtype if dtype is None else dtype
+    M, N, ld = _rows_view(x)
+    y = torch.empty(x.shape, dtype=dtype, device=x.device)
+    _check("mx_fake_quantize", lib.mx_fake_quantize(formats[fmt], _ptr(x), dt, M, N, ld, _ptr(y),
+                                                    _dtype_code(dtype), _stream(x)))
+    return y
 
 
 # ------------------------------------------------------------------ NVFP4
@@ -287,6 +354,96 @@ def nvfp4_quantize(x: torch.Tensor, global_scale: torch.Tensor | None = None,
                               flags, _ptr(ws), 0 if ws is None else ws.numel() * ws.element_size(),
                               _stream(x)))
     return packed, bs, g
+
+
+def _slice_array(slice_rows, M):
+    rows = [int(r) for r in slice_rows]
+    if not rows or any(r < 0 for r in rows) or sum(rows) != M:
+        raise ValueError(f"slice_rows must be non-negative and sum to the {M} rows")
+    return (ctypes.c_int64 * len(rows))(*rows), len(rows)
+
+
+def _sliced_workspace(n, dev, workspace):
+    if workspace is not None:
+        return workspace
+    return torch.empty(int(lib.mxq_nvfp4_sliced_workspace_bytes(n)), dtype=torch.uint8, device=dev)
+
+
+def nvfp4_amax_sliced(x: torch.Tensor, slice_rows: Sequence[int],
+                      workspace: torch.Tensor | None = None) -> torch.Tensor:
+    """Per-slice amax (non-NaN max |x|) of consecutive row ranges of x seen as
+    [M, N], as an fp32 CUDA tensor [len(slice_rows)]."""
+    _require_cuda(x)
+    dt = _dtype_code(x.dtype)
+    M, N, ld = _rows_view(x)
+    rows, S = _slice_array(slice_rows, M)
+    out = torch.zeros(S, dtype=torch.float32, device=x.device)
+    ws = _sliced_workspace(S, x.device, workspace)
+    _check("nvfp4_amax_sliced",
+           lib.nvfp4_amax_sliced(_ptr(x), dt, M, N, ld, S, ctypes.cast(rows, ctypes.c_void_p),
+                                 _ptr(out), _ptr(ws), ws.numel() * ws.element_size(), _stream(x)))
+    return out
+
+
+def nvfp4_quantize_sliced(x: torch.Tensor, slice_rows: Sequence[int],
+                          global_scales: torch.Tensor | None = None,
+                          amax: torch.Tensor | None = None,
+                          workspace: torch.Tensor | None = None):
+    """NVFP4 quantize with one global scale per slice of consecutive rows of
+    x seen as [M, N] (slice s holds slice_rows[s] rows): each slice is
+    quantized as :func:`nvfp4_quantize` would quantize it alone.
+
+    Returns ``(packed, block_scale, global_scales)`` with packed / block_scale
+    shaped as for :func:`nvfp4_quantize` and fp32 ``global_scales``
+    [len(slice_rows)]. ``global_scales`` (given g per slice) or ``amax``
+    (given slice amaxes) skip the amax pass."""
+    _require_cuda(x)
+    dt = _dtype_code(x.dtype)
+    M, N, ld = _rows_view(x)
+    rows, S = _slice_array(slice_rows, M)
+    dev = x.device
+    packed = torch.empty((*x.shape[:-1], N // 2), dtype=torch.uint8, device=dev)
+    bs = torch.empty((*x.shape[:-1], N // 16), dtype=torch.uint8, device=dev)
+    flags = 0
+    if global_scales is not None:
+        if global_scales.dtype != torch.float32 or global_scales.numel() != S:
+            raise TypeError("global_scales must be fp32 with one value per slice")
+        g = global_scales.to(dev).contiguous()
+        flags = NVFP4_GLOBAL_GIVEN
+    else:
+        g = torch.zeros(S, dtype=torch.float32, device=dev)
+    if amax is not None:
+        if amax.dtype != torch.float32 or amax.numel() != S:
+            raise TypeError("amax must be fp32 with one value per slice")
+        amax = amax.contiguous()
+    ws = None
+    if global_scales is None and amax is None:
+        ws = _sliced_workspace(S, dev, workspace)
+    _check("nvfp4_quantize_sliced",
+           lib.nvfp4_quantize_sliced(_ptr(x), dt, M, N, ld, S, ctypes.cast(rows, ctypes.c_void_p),
+                                     _ptr(packed), _ptr(bs), _ptr(g), _ptr(amax), flags, _ptr(ws),
+                                     0 if ws is None else ws.numel() * ws.element_size(),
+                                     _stream(x)))
+    return packed, bs, g
+
+
+def nvfp4_quantize_experts(w: torch.Tensor, *, per_half: bool = False,
+                           global_scales: torch.Tensor | None = None):
+    """NVFP4 of a stacked expert weight [E, R, N] with one global scale per
+    expert, or with ``per_half=True`` one per half of each expert's rows
+    (fused gate/up weights: rows [0, R/2) gate, [R/2, R) up).
+
+    Returns ``(packed [E, R, N/2], block_scale [E, R, N/16], global_scales)``
+    with global_scales fp32 [E] or [E, 2]."""
+    if w.dim() != 3:
+        raise ValueError("expected a stacked [E, R, N] weight")
+    E, R, _ = w.shape
+    if per_half and R % 2:
+        raise ValueError("per_half needs an even number of rows per expert")
+    rows = [R // 2] * (2 * E) if per_half else [R] * E
+    gs = None if global_scales is None else global_scales.reshape(-1)
+    p, b, g = nvfp4_quantize_sliced(w, rows, global_scales=gs)
+    return p, b, g.view(E, 2) if per_half else g
 
 
 def nvfp4_dequantize(packed: torch.Tensor, block_scale: torch.Tensor, global_scale: torch.Tensor,

@@ -42,19 +42,6 @@ constexpr int kPitch = kRowBytes + 16;       // padded shared-memory row pitch
 constexpr int kWordCols = kRowBytes / 4;     // 64 word columns per tile
 constexpr int kOutPitch = kTileRows + 16;    // shared pitch of a transposed code row
 
-__device__ __forceinline__ uint32_t e8m0_byte(float amax) {
-  const uint32_t bits = __float_as_uint(amax);
-  const uint32_t E = bits >> 23;
-  uint32_t b = max(E, 8u) - 8u;
-  b = (E == 255) ? 254u : b;
-  b = (bits == 0) ? 127u : b;
-  return b;
-}
-
-__device__ __forceinline__ float pow2_quant(uint32_t b) {
-  return __uint_as_float(b == 254 ? 0x00400000u : (254u - b) << 23);
-}
-
 __device__ __forceinline__ uint32_t lds32(const uint8_t* p) {
   uint32_t v;
   asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(static_cast<uint32_t>(__cvta_generic_to_shared(p))));
@@ -74,25 +61,6 @@ __device__ __forceinline__ void sts128(uint8_t* p, uint4 v) {
                    static_cast<uint32_t>(__cvta_generic_to_shared(p))),
                "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
                : "memory");
-}
-
-// Store the first `valid` (<= 32) bytes of a 32-byte group; 16-byte stores
-// when the destination is 16-byte aligned, byte stores otherwise.
-__device__ __forceinline__ void store_group(uint8_t* dst, const uint4& lo, const uint4& hi,
-                                            int valid, bool aligned) {
-  if (aligned && valid == 32) {
-    st_v4(dst, lo);
-    st_v4(dst + 16, hi);
-    return;
-  }
-  if (aligned && valid >= 16) {
-    st_v4(dst, lo);
-    const uint32_t w[4] = {hi.x, hi.y, hi.z, hi.w};
-    for (int i = 16; i < valid; i++) st_u8(dst + i, (w[(i - 16) >> 2] >> (8 * (i & 3))) & 0xffu);
-    return;
-  }
-  const uint32_t w[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
-  for (int i = 0; i < valid; i++) st_u8(dst + i, (w[i >> 2] >> (8 * (i & 3))) & 0xffu);
 }
 
 struct ColArgs {
@@ -200,7 +168,7 @@ mxfp8_colwise_kernel(const __grid_constant__ ColArgs a) {
 #pragma unroll
           for (int i = 0; i < 32; i++) amax = fmaxf(amax, fabsf(f[i]));
         }
-        const uint32_t b = e8m0_byte(amax);
+        const uint32_t b = mx_scale_byte<8>(amax);
         uint4 lo, hi;
         column_codes(f, pow2_quant(b), lo, hi);
         uint8_t* dst = a.q + (r0 + r) * a.N + c0 + 32 * k;
@@ -229,8 +197,8 @@ mxfp8_colwise_kernel(const __grid_constant__ ColArgs a) {
 #pragma unroll
         for (int i = 2; i < 32; i++) m = absmax_bf16x2(m, v[i]);
         m &= 0x7fff7fffu;
-        sb[0] = e8m0_byte(fmaxf(bf16_lo(m), 0.0f));
-        sb[1] = e8m0_byte(fmaxf(bf16_hi(m), 0.0f));
+        sb[0] = mx_scale_byte<8>(fmaxf(bf16_lo(m), 0.0f));
+        sb[1] = mx_scale_byte<8>(fmaxf(bf16_hi(m), 0.0f));
 #pragma unroll
         for (int i = 0; i < 32; i++) f[i] = bf16_lo(v[i]);
         column_codes(f, pow2_quant(sb[0]), code[0], code[1]);
@@ -244,7 +212,7 @@ mxfp8_colwise_kernel(const __grid_constant__ ColArgs a) {
           f[i] = __uint_as_float(v[i]);
           amax = fmaxf(amax, fabsf(f[i]));
         }
-        sb[0] = e8m0_byte(amax);
+        sb[0] = mx_scale_byte<8>(amax);
         column_codes(f, pow2_quant(sb[0]), code[0], code[1]);
       }
     }

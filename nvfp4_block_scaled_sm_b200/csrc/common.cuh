@@ -213,6 +213,34 @@ __device__ __forceinline__ uint32_t e4m3_nan_bytes(uint32_t w) {
   return ((w & 0x7f7f7f7fu) + 0x01010101u) & 0x80808080u;
 }
 
+// ------------------------------------------------------------ MX scales
+
+// Biased E8M0 exponent of a group's amax (amax >= 0, not NaN) by the OCP MX
+// rule for an element format whose largest normal has exponent EMAX (8 for
+// E4M3, 2 for E2M1): 127 for amax == 0, 254 for amax == inf, else
+// clamp(E(amax) - EMAX, 0, 254) with E the biased fp32 exponent field (the
+// same number as floor(log2 amax) + 127 - EMAX, clamped).
+template <int EMAX>
+__device__ __forceinline__ uint32_t mx_scale_byte(float amax) {
+  const uint32_t bits = __float_as_uint(amax);
+  const uint32_t E = bits >> 23;
+  uint32_t b = max(E, uint32_t(EMAX)) - uint32_t(EMAX);
+  b = (E == 255) ? 254u : b;
+  b = (bits == 0) ? 127u : b;
+  return b;
+}
+
+// 2^(127 - b) for b in [0, 254]; b == 254 is the fp32 subnormal 2^-127.
+__device__ __forceinline__ float pow2_quant(uint32_t b) {
+  return __uint_as_float(b == 254 ? 0x00400000u : (254u - b) << 23);
+}
+
+// 2^(b - 127) for a scale byte b; 0 is the fp32 subnormal 2^-127 and 255
+// (the E8M0 NaN) is NaN.
+__device__ __forceinline__ float pow2_dequant(uint32_t b) {
+  return __uint_as_float(b == 0 ? 0x00400000u : (b == 255 ? 0x7fc00000u : b << 23));
+}
+
 // ------------------------------------------------------ 8-element lanes
 
 // Eight consecutive input elements held by one lane: one 16-byte load of

@@ -1,0 +1,675 @@
+// mx_rowwise.cu -- MX rowwise quantize (compact + optional swizzled scales,
+// single tensor or a group of expert tensors in one launch), dequantize and
+// fused fake-quantize, for the two MX element formats: MXFP8 (E4M3 codes, one
+// byte each) and MXFP4 (E2M1 codes, two per byte), for sm_100a.
+//
+// Method ("PR #1935 完整报告 -- Use TransformerEngine for MXFP8 quantization",
+// 实现拆解 items 1 and 4; "V4 mxfp4 #1372", description and
+// mxfp4_simulate_qat): groups of 32 consecutive elements along the last dim;
+// per group amax = max |x| over its non-NaN elements, E8M0 byte = 127 for
+// amax == 0, 254 for amax == inf, else clamp(E(amax) - emax, 0, 254) where E
+// is the biased fp32 exponent field (the same number as floor(log2 amax) +
+// 127 - emax, clamped; emax = 8 for E4M3, 2 for E2M1), and
+// q = CODE(x * 2^(127 - byte)) rounded to nearest even with saturation to the
+// format's largest value (448 for E4M3, 6 for E2M1). Fake-quantize writes
+// decode(q) * 2^(byte - 127), the dequantization of the quantization, without
+// storing q.
+//
+// Exactness of the fp32 path: for finite amax the byte is at most 254 - emax,
+// so the multiplier 2^(127 - byte) is a normal fp32 power of two and
+// x * multiplier is exact whenever the product is an fp32 normal. Products
+// below 2^-126 (where fp32 would round) are far below half the smallest
+// non-zero code (2^-10 for E4M3, 0.25 for E2M1), so they encode to a zero of
+// the right sign either way. An infinite amax gives byte 254 and the
+// subnormal multiplier 2^-127 (built from its bit pattern), again exact for
+// every product that can encode to non-zero. cvt.rn.satfinite.e4m3x2.f32
+// rounds to nearest even, saturates finite and infinite values to +-448,
+// keeps the sign of zero and writes every NaN as 0x7F;
+// cvt.rn.satfinite.e2m1x2.f32 does the same with +-6 and writes NaN as +6
+// (0x7). Both are checked exhaustively against the oracle by the GPU tests.
+//
+// Work split (HBM-bound: 2 bytes read and 1 + 1/32 (MXFP8) or 1/2 + 1/32
+// (MXFP4) written per bf16 element): a lane owns 16 consecutive elements
+// (one 256-bit load of bf16, two of fp32, when 32-byte aligned), two lanes a
+// group, a warp 16 consecutive groups per step (1 KiB of contiguous bf16) and
+// kSteps steps, a CTA kGroupsPerTile consecutive groups. All loads of a lane
+// are issued before any is used. The tile's base pointers are formed once in
+// 64-bit arithmetic; lane offsets inside a tile are 32-bit, and full tiles
+// skip the bounds checks. Rows are never padded: groups do not cross rows,
+// so the result for M rows equals the pad-to-32-rows-then-crop contract.
+#include "common.cuh"
+
+namespace mxq {
+namespace {
+
+constexpr int kGroupsPerStep = 16;  // per warp and step
+constexpr int kSteps = 2;
+constexpr int kGroupsPerWarp = kGroupsPerStep * kSteps;
+constexpr int kGroupsPerTile = kGroupsPerWarp * (kThreads / 32);
+
+// Element formats. kE4M3: MXFP8, one code byte per element. kE2M1: MXFP4, two
+// codes per byte, element 2k in the low nibble.
+constexpr int kE4M3 = 0;
+constexpr int kE2M1 = 1;
+template <int FMT>
+constexpr int kEmax = FMT == kE4M3 ? 8 : 2;
+template <int FMT>
+constexpr uint32_t kCodeBytes = FMT == kE4M3 ? 32 : 16;  // code bytes per group
+
+// Byte offset of scale (r, c) in the 128x4-tile layout of block-scaled MMA.
+__device__ __forceinline__ uint64_t swz_offset(uint64_t r, uint32_t c, uint32_t Sp4) {
+  return (((r >> 7) * Sp4 + (c >> 2)) << 9) + ((r & 31) << 4) + (((r >> 5) & 3) << 2) + (c & 3);
+}
+
+// E4M3 codes of the lane's 16 elements times `mul` (low byte = first element).
+template <typename InT>
+__device__ __forceinline__ uint4 to_e4m3(const In16<InT>& v, float mul) {
+  uint32_t c[8];
+#pragma unroll
+  for (int k = 0; k < 8; k++) {
+    const float2 p = mul2(v.lo(k), v.hi(k), mul);
+    c[k] = cvt_e4m3x2(p.x, p.y);
+  }
+  return make_uint4(__byte_perm(c[0], c[1], 0x5410), __byte_perm(c[2], c[3], 0x5410),
+                    __byte_perm(c[4], c[5], 0x5410), __byte_perm(c[6], c[7], 0x5410));
+}
+
+// E2M1 codes of the lane's 16 elements times `mul`, two per byte with the
+// even element in the low nibble (8 bytes, first element in the low byte).
+template <typename InT>
+__device__ __forceinline__ uint2 to_e2m1(const In16<InT>& v, float mul) {
+  uint32_t c[8];
+#pragma unroll
+  for (int k = 0; k < 8; k++) {
+    const float2 p = mul2(v.lo(k), v.hi(k), mul);
+    c[k] = cvt_e2m1x2(p.x, p.y);
+  }
+  return make_uint2(c[0] | (c[1] << 8) | (c[2] << 16) | (c[3] << 24),
+                    c[4] | (c[5] << 8) | (c[6] << 16) | (c[7] << 24));
+}
+
+template <int MAXE>
+struct QuantArgs {
+  uint8_t* q;
+  uint8_t* scale;
+  uint8_t* swz;          // swizzled scales (SWZ only)
+  int64_t ld;            // input row stride in elements (STRIDED only)
+  FastDiv rows;          // group index -> row, i.e. division by S
+  uint32_t S;            // groups per row
+  uint32_t Sp4;          // ceil(S / 4)
+  uint64_t M;            // rows (SWZ padding)
+  uint64_t pad_a;        // swizzle padding entries right of the real scale columns
+  uint64_t pad_b;        // swizzle padding entries below the real rows
+  int32_t E;             // experts
+  const void* x[MAXE];
+  uint64_t gbase[MAXE + 1];  // first output group of expert e; gbase[E] = all groups
+  uint32_t tbase[MAXE + 1];  // first CTA of expert e; tbase[E] = grid size
+};
+
+// Zero bytes of the swizzled layout outside the real [M, S] scales.
+template <int MAXE>
+__device__ __forceinline__ void fill_swizzle_padding(const QuantArgs<MAXE>& a) {
+  const uint64_t total = a.pad_a + a.pad_b;
+  const uint32_t Sp = a.Sp4 * 4;
+  const uint64_t stride = uint64_t(gridDim.x) * kThreads;
+  for (uint64_t p = uint64_t(blockIdx.x) * kThreads + threadIdx.x; p < total; p += stride) {
+    uint64_t r;
+    uint32_t c;
+    if (p < a.pad_a) {
+      const uint32_t w = Sp - a.S;
+      r = p / w;
+      c = a.S + uint32_t(p % w);
+    } else {
+      const uint64_t t = p - a.pad_a;
+      r = a.M + t / Sp;
+      c = uint32_t(t % Sp);
+    }
+    st_u8(a.swz + swz_offset(r, c, a.Sp4), 0);
+  }
+}
+
+template <typename InT, bool V8, bool STRIDED, bool SWZ, int MAXE, int FMT>
+__global__ void __launch_bounds__(kThreads)
+mx_quant_kernel(const __grid_constant__ QuantArgs<MAXE> a) {
+  pdl_enter();
+  const uint32_t tile = blockIdx.x;
+  int e = 0;
+  if constexpr (MAXE > 1) {
+    int lo = 0, hi = a.E;  // invariant: tbase[lo] <= tile < tbase[hi]
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (a.tbase[mid] <= tile) lo = mid; else hi = mid;
+    }
+    e = lo;
+  }
+  const uint64_t tg0 = uint64_t(tile - a.tbase[e]) * kGroupsPerTile;  // tile's first group
+  const uint64_t left = a.gbase[e + 1] - a.gbase[e] - tg0;
+  const uint32_t nt = left < kGroupsPerTile ? uint32_t(left) : uint32_t(kGroupsPerTile);
+  const bool full = nt == kGroupsPerTile;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const uint32_t half = lane & 1;
+  const uint32_t lg0 = warp * kGroupsPerWarp + (lane >> 1);  // tile-local group of step 0
+
+  const InT* x = static_cast<const InT*>(a.x[e]);
+  constexpr uint32_t CB = kCodeBytes<FMT>;
+  uint8_t* qt = a.q + (a.gbase[e] + tg0) * CB + half * (CB / 2);
+  uint8_t* st = a.scale + a.gbase[e] + tg0;
+
+  // row / column of the lane's group (strided input, swizzled scales)
+  uint64_t r = 0;
+  uint32_t c = 0;
+  if constexpr (STRIDED || SWZ) {
+    const uint64_t g = tg0 + lg0;
+    r = a.rows.div(g);
+    c = uint32_t(g - r * a.S);
+  }
+  uint64_t rr[kSteps];
+  uint32_t cc[kSteps];
+#pragma unroll
+  for (int u = 0; u < kSteps; u++) {
+    rr[u] = r;
+    cc[u] = c;
+    if constexpr (STRIDED || SWZ) {
+      c += kGroupsPerStep;
+      while (c >= a.S) {
+        c -= a.S;
+        ++r;
+      }
+    }
+  }
+
+  In16<InT> v[kSteps];
+#pragma unroll
+  for (int u = 0; u < kSteps; u++) {
+    const uint32_t lg = lg0 + u * kGroupsPerStep;
+    const InT* p;
+    if constexpr (STRIDED) {
+      p = x + rr[u] * uint64_t(a.ld) + cc[u] * 32 + half * 16;
+    } else {
+      p = x + (tg0 + lg) * 32 + half * 16;
+    }
+    if (full || lg < nt) v[u].template load<V8>(p); else v[u].zero();
+  }
+
+#pragma unroll
+  for (int u = 0; u < kSteps; u++) {
+    const uint32_t lg = lg0 + u * kGroupsPerStep;
+    float amax = v[u].absmax();
+    amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, 1));
+    amax = fmaxf(amax, 0.0f);  // a group holding only NaNs has amax 0
+    const uint32_t b = mx_scale_byte<kEmax<FMT>>(amax);
+    uint4 o4;
+    uint2 o2;
+    if constexpr (FMT == kE4M3) o4 = to_e4m3(v[u], pow2_quant(b));
+    else o2 = to_e2m1(v[u], pow2_quant(b));
+    if (full || lg < nt) {
+      if constexpr (FMT == kE4M3) st_v4(qt + lg * CB, o4);
+      else st_v2(qt + lg * CB, o2);
+      if (half == 0) {
+        st_u8(st + lg, b);
+        if constexpr (SWZ) st_u8(a.swz + swz_offset(rr[u], cc[u], a.Sp4), b);
+      }
+    }
+  }
+  if constexpr (SWZ) fill_swizzle_padding(a);
+}
+
+// ------------------------------------------------------- decode and store
+
+// decode(code) * mul of a lane's 16 E4M3 codes (four words, first code in the
+// low byte of cw[0]); exact in fp32 except for overflow to inf.
+__device__ __forceinline__ void decode_e4m3_16(const uint32_t (&cw)[4], float mul,
+                                               float (&f)[16]) {
+#pragma unroll
+  for (int k = 0; k < 8; k++) {
+    const float2 d = f16x2_to_f32x2(cvt_f16x2_from_e4m3x2(cw[k >> 1] >> (16 * (k & 1))));
+    const float2 p = mul2(d.x, d.y, mul);
+    f[2 * k] = p.x;
+    f[2 * k + 1] = p.y;
+  }
+}
+
+// The same for 16 E2M1 codes, two per byte, even element in the low nibble.
+__device__ __forceinline__ void decode_e2m1_16(uint2 cw, float mul, float (&f)[16]) {
+#pragma unroll
+  for (int k = 0; k < 8; k++) {
+    const uint32_t byte = ((k < 4 ? cw.x : cw.y) >> (8 * (k & 3))) & 0xffu;
+    const float2 d = f16x2_to_f32x2(cvt_f16x2_from_e2m1x2(byte));
+    const float2 p = mul2(d.x, d.y, mul);
+    f[2 * k] = p.x;
+    f[2 * k + 1] = p.y;
+  }
+}
+
+// True if any of the four words holds the E4M3 NaN code 0x7F or 0xFF.
+__device__ __forceinline__ bool any_e4m3_nan(const uint32_t (&cw)[4]) {
+  const uint32_t m = 0x7f7f7f7fu, o = 0x01010101u;
+  return ((((cw[0] & m) + o) | ((cw[1] & m) + o) | ((cw[2] & m) + o) | ((cw[3] & m) + o)) &
+          0x80808080u) != 0;
+}
+
+// Writes a lane's 16 fp32 values as OutT (bf16: round to nearest even). When
+// `any_nan`, every element i with is_nan(i) is written as the canonical NaN
+// (0x7FC0 / 0x7FC00000) instead.
+template <typename OutT, bool V8, typename IsNan>
+__device__ __forceinline__ void store16(OutT* dst, const float (&f)[16], bool any_nan,
+                                        IsNan is_nan) {
+  if constexpr (sizeof(OutT) == 2) {
+    uint32_t w[8];
+#pragma unroll
+    for (int k = 0; k < 8; k++) w[k] = cvt_bf16x2(f[2 * k], f[2 * k + 1]);
+    if (any_nan) {
+#pragma unroll
+      for (int i = 0; i < 16; i++) {
+        if (is_nan(i)) {
+          const int sh = 16 * (i & 1);
+          w[i >> 1] = (w[i >> 1] & ~(0xffffu << sh)) | (0x7fc0u << sh);
+        }
+      }
+    }
+    if constexpr (V8) {
+      st_v8(dst, w);
+    } else {
+      st_v4(dst, make_uint4(w[0], w[1], w[2], w[3]));
+      st_v4(dst + 8, make_uint4(w[4], w[5], w[6], w[7]));
+    }
+  } else {
+    uint32_t w[16];
+#pragma unroll
+    for (int i = 0; i < 16; i++) w[i] = __float_as_uint(f[i]);
+    if (any_nan) {
+#pragma unroll
+      for (int i = 0; i < 16; i++)
+        if (is_nan(i)) w[i] = 0x7fc00000u;
+    }
+    if constexpr (V8) {
+      st_v8(dst, *reinterpret_cast<const uint32_t(*)[8]>(&w[0]));
+      st_v8(dst + 8, *reinterpret_cast<const uint32_t(*)[8]>(&w[8]));
+    } else {
+#pragma unroll
+      for (int i = 0; i < 4; i++)
+        st_v4(dst + 4 * i, make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]));
+    }
+  }
+}
+
+// ---------------------------------------------------------------- dequant
+
+// A lane owns 16 codes (one 16-byte load of E4M3 codes, one 8-byte load of
+// packed E2M1) and writes 16 outputs (32 bytes of bf16, 64 of fp32, with
+// 256-bit stores when 32-byte aligned); two lanes a group; 16 groups per warp
+// step.
+constexpr int kDqSteps = 2;
+constexpr int kDqGroupsPerWarp = 16 * kDqSteps;
+constexpr int kDqGroupsPerTile = kDqGroupsPerWarp * (kThreads / 32);
+
+template <typename OutT, bool V8, int FMT>
+__global__ void __launch_bounds__(kThreads)
+mx_dequant_kernel(const uint8_t* __restrict__ q, const uint8_t* __restrict__ scale,
+                  OutT* __restrict__ y, uint64_t ng) {
+  pdl_enter();
+  constexpr uint32_t CB = kCodeBytes<FMT>;
+  const uint64_t g0 = uint64_t(blockIdx.x) * kDqGroupsPerTile;
+  const uint64_t left = ng - g0;
+  const uint32_t nt = left < kDqGroupsPerTile ? uint32_t(left) : uint32_t(kDqGroupsPerTile);
+  const bool full = nt == kDqGroupsPerTile;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const uint32_t half = lane & 1;
+  const uint32_t lg0 = warp * kDqGroupsPerWarp + (lane >> 1);
+  const uint8_t* qt = q + g0 * CB + half * (CB / 2);
+  const uint8_t* st = scale + g0;
+  OutT* yt = y + g0 * 32 + half * 16;
+
+  uint32_t c[kDqSteps][4];
+  uint32_t b[kDqSteps];
+#pragma unroll
+  for (int u = 0; u < kDqSteps; u++) {
+    const uint32_t lg = lg0 + u * 16;
+    c[u][0] = c[u][1] = c[u][2] = c[u][3] = 0;
+    b[u] = 127;
+    if (full || lg < nt) {
+      if constexpr (FMT == kE4M3) {
+        const uint4 t = ld_nc_v4(qt + lg * CB);
+        c[u][0] = t.x; c[u][1] = t.y; c[u][2] = t.z; c[u][3] = t.w;
+      } else {
+        const uint2 t = ld_nc_v2(qt + lg * CB);
+        c[u][0] = t.x; c[u][1] = t.y;
+      }
+      b[u] = ld_nc_u8(st + lg);
+    }
+  }
+#pragma unroll
+  for (int u = 0; u < kDqSteps; u++) {
+    const uint32_t lg = lg0 + u * 16;
+    if (!(full || lg < nt)) continue;
+    const float mul = pow2_dequant(b[u]);
+    const uint32_t (&cw)[4] = c[u];
+    const uint32_t bu = b[u];
+    float f[16];
+    if constexpr (FMT == kE4M3) {
+      decode_e4m3_16(cw, mul, f);
+      store16<OutT, V8>(yt + lg * 32, f, any_e4m3_nan(cw) || bu == 255, [&](int i) {
+        return ((cw[i >> 2] >> (8 * (i & 3))) & 0x7f) == 0x7f || bu == 255;
+      });
+    } else {
+      // E2M1 has no NaN code: only the E8M0 NaN scale gives NaN outputs.
+      decode_e2m1_16(make_uint2(cw[0], cw[1]), mul, f);
+      store16<OutT, V8>(yt + lg * 32, f, bu == 255, [](int) { return true; });
+    }
+  }
+}
+
+// ----------------------------------------------------------- fake quantize
+
+struct FakeArgs {
+  const void* x;
+  void* y;
+  int64_t ld;       // input row stride in elements (STRIDED only)
+  FastDiv rows;     // group index -> row
+  uint32_t S;       // groups per row
+  uint64_t groups;  // M * S
+};
+
+// y = decode(quantize(x)) * 2^(byte - 127) per group, quantize exactly as in
+// mx_quant_kernel, decode exactly as in mx_dequant_kernel; the codes stay in
+// registers. Work split as in mx_quant_kernel; y is contiguous [M, N].
+template <typename InT, typename OutT, bool V8, bool STRIDED, int FMT>
+__global__ void __launch_bounds__(kThreads)
+mx_fake_quant_kernel(const __grid_constant__ FakeArgs a) {
+  pdl_enter();
+  const uint64_t tg0 = uint64_t(blockIdx.x) * kGroupsPerTile;
+  const uint64_t left = a.groups - tg0;
+  const uint32_t nt = left < kGroupsPerTile ? uint32_t(left) : uint32_t(kGroupsPerTile);
+  const bool full = nt == kGroupsPerTile;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const uint32_t half = lane & 1;
+  const uint32_t lg0 = warp * kGroupsPerWarp + (lane >> 1);
+  const InT* x = static_cast<const InT*>(a.x);
+  OutT* yt = static_cast<OutT*>(a.y) + tg0 * 32 + half * 16;
+
+  uint64_t r = 0;
+  uint32_t c = 0;
+  if constexpr (STRIDED) {
+    const uint64_t g = tg0 + lg0;
+    r = a.rows.div(g);
+    c = uint32_t(g - r * a.S);
+  }
+  In16<InT> v[kSteps];
+#pragma unroll
+  for (int u = 0; u < kSteps; u++) {
+    const uint32_t lg = lg0 + u * kGroupsPerStep;
+    const InT* p;
+    if constexpr (STRIDED) {
+      p = x + r * uint64_t(a.ld) + c * 32 + half * 16;
+      c += kGroupsPerStep;
+      while (c >= a.S) {
+        c -= a.S;
+        ++r;
+      }
+    } else {
+      p = x + (tg0 + lg) * 32 + half * 16;
+    }
+    if (full || lg < nt) v[u].template load<V8>(p); else v[u].zero();
+  }
+
+#pragma unroll
+  for (int u = 0; u < kSteps; u++) {
+    const uint32_t lg = lg0 + u * kGroupsPerStep;
+    float amax = v[u].absmax();
+    amax = fmaxf(amax, __shfl_xor_sync(kFull, amax, 1));
+    amax = fmaxf(amax, 0.0f);
+    const uint32_t b = mx_scale_byte<kEmax<FMT>>(amax);
+    const float dmul = pow2_dequant(b);
+    float f[16];
+    if constexpr (FMT == kE4M3) {
+      const uint4 o = to_e4m3(v[u], pow2_quant(b));
+      const uint32_t cw[4] = {o.x, o.y, o.z, o.w};
+      decode_e4m3_16(cw, dmul, f);
+      if (full || lg < nt) {
+        store16<OutT, V8>(yt + lg * 32, f, any_e4m3_nan(cw), [&](int i) {
+          return ((cw[i >> 2] >> (8 * (i & 3))) & 0x7f) == 0x7f;
+        });
+      }
+    } else {
+      decode_e2m1_16(to_e2m1(v[u], pow2_quant(b)), dmul, f);
+      if (full || lg < nt) store16<OutT, V8>(yt + lg * 32, f, false, [](int) { return false; });
+    }
+  }
+}
+
+// ------------------------------------------------------------------ host
+
+inline bool aligned32(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 31u) == 0; }
+
+template <typename InT, bool V8, bool STRIDED, bool SWZ, int MAXE, int FMT>
+mxq_status launch_quant(const QuantArgs<MAXE>& a, uint32_t grid, cudaStream_t stream) {
+  return launched(launch_pdl(mx_quant_kernel<InT, V8, STRIDED, SWZ, MAXE, FMT>, grid, stream, a));
+}
+
+template <typename InT, bool V8, int FMT>
+mxq_status dispatch_single(const QuantArgs<1>& a, bool strided, bool swz, uint32_t grid,
+                           cudaStream_t s) {
+  if (strided) {
+    return swz ? launch_quant<InT, V8, true, true, 1, FMT>(a, grid, s)
+               : launch_quant<InT, V8, true, false, 1, FMT>(a, grid, s);
+  }
+  return swz ? launch_quant<InT, V8, false, true, 1, FMT>(a, grid, s)
+             : launch_quant<InT, V8, false, false, 1, FMT>(a, grid, s);
+}
+
+template <int FMT>
+mxq_status quantize_impl(const void* x, int dt, int64_t M, int64_t N, int64_t ld_x,
+                         uint8_t* q, uint8_t* scale, uint8_t* scale_swz, mxq_stream_t stream) {
+  if (!valid_dtype(dt)) return MXQ_ERR_DTYPE;
+  if (M < 0 || N < 0 || N % 32 != 0 || ld_x < N) return MXQ_ERR_SHAPE;
+  if (M == 0 || N == 0) return MXQ_OK;
+  if (!x || !q || !scale) return MXQ_ERR_NULL;
+  const uint64_t S = uint64_t(N) / 32;
+  const uint64_t groups = uint64_t(M) * S;
+  const uint64_t tiles = (groups + kGroupsPerTile - 1) / kGroupsPerTile;
+  if (S > 0xffffffffull || tiles > 0x7fffffffull) return MXQ_ERR_SHAPE;
+  const uint64_t row_bytes = uint64_t(ld_x) * elem_size(dt);
+  if (!aligned16(x) || row_bytes % 16 != 0 || !aligned16(q)) return MXQ_ERR_ALIGN;
+
+  QuantArgs<1> a{};
+  a.q = q;
+  a.scale = scale;
+  a.swz = scale_swz;
+  a.ld = ld_x;
+  a.rows = FastDiv::make(uint32_t(S));
+  a.S = uint32_t(S);
+  a.Sp4 = uint32_t((S + 3) / 4);
+  a.M = uint64_t(M);
+  const uint64_t Mp = (uint64_t(M) + 127) / 128 * 128, Sp = uint64_t(a.Sp4) * 4;
+  a.pad_a = uint64_t(M) * (Sp - S);
+  a.pad_b = (Mp - uint64_t(M)) * Sp;
+  a.E = 1;
+  a.x[0] = x;
+  a.gbase[0] = 0;
+  a.gbase[1] = groups;
+  a.tbase[0] = 0;
+  a.tbase[1] = uint32_t(tiles);
+  const bool strided = ld_x != N;
+  const bool swz = scale_swz != nullptr;
+  const bool v8 = aligned32(x) && row_bytes % 32 == 0;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const uint32_t grid = uint32_t(tiles);
+  if (dt == MXQ_BF16) {
+    return v8 ? dispatch_single<uint16_t, true, FMT>(a, strided, swz, grid, s)
+              : dispatch_single<uint16_t, false, FMT>(a, strided, swz, grid, s);
+  }
+  return v8 ? dispatch_single<float, true, FMT>(a, strided, swz, grid, s)
+            : dispatch_single<float, false, FMT>(a, strided, swz, grid, s);
+}
+
+template <int FMT>
+mxq_status dequantize_impl(const uint8_t* q, const uint8_t* scale, int64_t M, int64_t N, void* y,
+                           int out_dt, mxq_stream_t stream) {
+  if (!valid_dtype(out_dt)) return MXQ_ERR_DTYPE;
+  if (M < 0 || N < 0 || N % 32 != 0) return MXQ_ERR_SHAPE;
+  if (M == 0 || N == 0) return MXQ_OK;
+  if (!q || !scale || !y) return MXQ_ERR_NULL;
+  if (!aligned16(q) || !aligned16(y)) return MXQ_ERR_ALIGN;
+  const uint64_t groups = uint64_t(M) * (uint64_t(N) / 32);
+  const uint64_t tiles = (groups + kDqGroupsPerTile - 1) / kDqGroupsPerTile;
+  if (tiles > 0x7fffffffull) return MXQ_ERR_SHAPE;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const uint32_t grid = uint32_t(tiles);
+  const bool v8 = aligned32(y);
+  if (out_dt == MXQ_BF16) {
+    uint16_t* yp = static_cast<uint16_t*>(y);
+    return launched(v8 ? launch_pdl(mx_dequant_kernel<uint16_t, true, FMT>, grid, s, q, scale, yp, groups)
+                       : launch_pdl(mx_dequant_kernel<uint16_t, false, FMT>, grid, s, q, scale, yp, groups));
+  }
+  float* yp = static_cast<float*>(y);
+  return launched(v8 ? launch_pdl(mx_dequant_kernel<float, true, FMT>, grid, s, q, scale, yp, groups)
+                     : launch_pdl(mx_dequant_kernel<float, false, FMT>, grid, s, q, scale, yp, groups));
+}
+
+template <int MAXE, int FMT>
+mxq_status grouped_impl(int32_t E, const void* const* xs, const int64_t* rows, int64_t N,
+                        int dt, uint8_t* q, uint8_t* scale, cudaStream_t stream) {
+  QuantArgs<MAXE> a{};
+  const uint64_t S = uint64_t(N) / 32;
+  uint64_t groups = 0, tiles = 0;
+  bool v8 = true;
+  a.E = E;
+  for (int32_t e = 0; e < E; e++) {
+    a.x[e] = xs[e];
+    a.gbase[e] = groups;
+    a.tbase[e] = uint32_t(tiles);
+    const uint64_t ng = uint64_t(rows[e]) * S;
+    if (ng && !aligned32(xs[e])) v8 = false;
+    groups += ng;
+    tiles += (ng + kGroupsPerTile - 1) / kGroupsPerTile;
+    if (tiles > 0x7fffffffull) return MXQ_ERR_SHAPE;
+  }
+  a.gbase[E] = groups;
+  a.tbase[E] = uint32_t(tiles);
+  if (tiles == 0) return MXQ_OK;
+  a.q = q;
+  a.scale = scale;
+  a.S = uint32_t(S);
+  const uint32_t grid = uint32_t(tiles);
+  if (dt == MXQ_BF16) {
+    return v8 ? launch_quant<uint16_t, true, false, false, MAXE, FMT>(a, grid, stream)
+              : launch_quant<uint16_t, false, false, false, MAXE, FMT>(a, grid, stream);
+  }
+  return v8 ? launch_quant<float, true, false, false, MAXE, FMT>(a, grid, stream)
+            : launch_quant<float, false, false, false, MAXE, FMT>(a, grid, stream);
+}
+
+template <int FMT>
+mxq_status grouped_entry(int32_t E, const void* const* xs, const int64_t* rows, int64_t N,
+                         int dt, uint8_t* q, uint8_t* scale, mxq_stream_t stream) {
+  if (!valid_dtype(dt)) return MXQ_ERR_DTYPE;
+  if (E < 1 || E > MXQ_GROUPED_MAX_EXPERTS || N < 0 || N % 32 != 0) return MXQ_ERR_SHAPE;
+  if (!xs || !rows) return MXQ_ERR_NULL;
+  if (uint64_t(N) / 32 > 0xffffffffull) return MXQ_ERR_SHAPE;
+  int64_t total = 0;
+  for (int32_t e = 0; e < E; e++) {
+    if (rows[e] < 0) return MXQ_ERR_SHAPE;
+    if (rows[e] > 0 && N > 0) {
+      if (!xs[e]) return MXQ_ERR_NULL;
+      if (!aligned16(xs[e])) return MXQ_ERR_ALIGN;
+    }
+    total += rows[e];
+  }
+  if (total == 0 || N == 0) return MXQ_OK;
+  if (!q || !scale) return MXQ_ERR_NULL;
+  if (!aligned16(q)) return MXQ_ERR_ALIGN;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (E <= 64) return grouped_impl<64, FMT>(E, xs, rows, N, dt, q, scale, s);
+  return grouped_impl<MXQ_GROUPED_MAX_EXPERTS, FMT>(E, xs, rows, N, dt, q, scale, s);
+}
+
+template <typename InT, typename OutT, int FMT>
+mxq_status launch_fake(const FakeArgs& a, bool v8, bool strided, uint32_t grid, cudaStream_t s) {
+  if (v8) {
+    return launched(strided ? launch_pdl(mx_fake_quant_kernel<InT, OutT, true, true, FMT>, grid, s, a)
+                            : launch_pdl(mx_fake_quant_kernel<InT, OutT, true, false, FMT>, grid, s, a));
+  }
+  return launched(strided ? launch_pdl(mx_fake_quant_kernel<InT, OutT, false, true, FMT>, grid, s, a)
+                          : launch_pdl(mx_fake_quant_kernel<InT, OutT, false, false, FMT>, grid, s, a));
+}
+
+template <int FMT>
+mxq_status fake_dispatch(const FakeArgs& a, int dt, int out_dt, bool v8, bool strided,
+                         uint32_t grid, cudaStream_t s) {
+  if (dt == MXQ_BF16) {
+    return out_dt == MXQ_BF16 ? launch_fake<uint16_t, uint16_t, FMT>(a, v8, strided, grid, s)
+                              : launch_fake<uint16_t, float, FMT>(a, v8, strided, grid, s);
+  }
+  return out_dt == MXQ_BF16 ? launch_fake<float, uint16_t, FMT>(a, v8, strided, grid, s)
+                            : launch_fake<float, float, FMT>(a, v8, strided, grid, s);
+}
+
+}  // namespace
+}  // namespace mxq
+
+extern "C" {
+
+mxq_status mxfp8_quantize(const void* x, int dt, int64_t M, int64_t N, int64_t ld_x,
+                          uint8_t* qweight, uint8_t* scale, uint8_t* scale_swz,
+                          mxq_stream_t stream) {
+  return mxq::quantize_impl<mxq::kE4M3>(x, dt, M, N, ld_x, qweight, scale, scale_swz, stream);
+}
+
+mxq_status mxfp8_dequantize(const uint8_t* qweight, const uint8_t* scale, int64_t M,
+                            int64_t N, void* y, int out_dt, mxq_stream_t stream) {
+  return mxq::dequantize_impl<mxq::kE4M3>(qweight, scale, M, N, y, out_dt, stream);
+}
+
+mxq_status mxfp8_quantize_grouped(int32_t E, const void* const* xs, const int64_t* rows,
+                                  int64_t N, int dt, uint8_t* qweight, uint8_t* scale,
+                                  mxq_stream_t stream) {
+  return mxq::grouped_entry<mxq::kE4M3>(E, xs, rows, N, dt, qweight, scale, stream);
+}
+
+mxq_status mxfp4_quantize(const void* x, int dt, int64_t M, int64_t N, int64_t ld_x,
+                          uint8_t* packed, uint8_t* scale, uint8_t* scale_swz,
+                          mxq_stream_t stream) {
+  return mxq::quantize_impl<mxq::kE2M1>(x, dt, M, N, ld_x, packed, scale, scale_swz, stream);
+}
+
+mxq_status mxfp4_dequantize(const uint8_t* packed, const uint8_t* scale, int64_t M, int64_t N,
+                            void* y, int out_dt, mxq_stream_t stream) {
+  return mxq::dequantize_impl<mxq::kE2M1>(packed, scale, M, N, y, out_dt, stream);
+}
+
+mxq_status mxfp4_quantize_grouped(int32_t E, const void* const* xs, const int64_t* rows,
+                                  int64_t N, int dt, uint8_t* packed, uint8_t* scale,
+                                  mxq_stream_t stream) {
+  return mxq::grouped_entry<mxq::kE2M1>(E, xs, rows, N, dt, packed, scale, stream);
+}
+
+mxq_status mx_fake_quantize(int fmt, const void* x, int dt, int64_t M, int64_t N, int64_t ld_x,
+                            void* y, int out_dt, mxq_stream_t stream) {
+  using namespace mxq;
+  if (fmt != MXQ_FMT_MXFP8 && fmt != MXQ_FMT_MXFP4) return MXQ_ERR_ARG;
+  if (!valid_dtype(dt) || !valid_dtype(out_dt)) return MXQ_ERR_DTYPE;
+  if (M < 0 || N < 0 || N % 32 != 0 || ld_x < N) return MXQ_ERR_SHAPE;
+  if (M == 0 || N == 0) return MXQ_OK;
+  if (!x || !y) return MXQ_ERR_NULL;
+  const uint64_t S = uint64_t(N) / 32;
+  const uint64_t groups = uint64_t(M) * S;
+  const uint64_t tiles = (groups + kGroupsPerTile - 1) / kGroupsPerTile;
+  if (S > 0xffffffffull || tiles > 0x7fffffffull) return MXQ_ERR_SHAPE;
+  const uint64_t row_bytes = uint64_t(ld_x) * elem_size(dt);
+  if (!aligned16(x) || row_bytes % 16 != 0 || !aligned16(y)) return MXQ_ERR_ALIGN;
+  FakeArgs a{};
+  a.x = x;
+  a.y = y;
+  a.ld = ld_x;
+  a.rows = FastDiv::make(uint32_t(S));
+  a.S = uint32_t(S);
+  a.groups = groups;
+  const bool v8 = aligned32(x) && row_bytes % 32 == 0 && aligned32(y);
+  const bool strided = ld_x != N;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const uint32_t grid = uint32_t(tiles);
+  return fmt == MXQ_FMT_MXFP8 ? fake_dispatch<kE4M3>(a, dt, out_dt, v8, strided, grid, s)
+                              : fake_dispatch<kE2M1>(a, dt, out_dt, v8, strided, grid, s);
+}
+
+}  // extern "C"

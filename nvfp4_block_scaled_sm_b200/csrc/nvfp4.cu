@@ -2,8 +2,8 @@
 // dequantize, for sm_100a.
 //
 // Method ("Add FP8, NVFP4, and QARL training and export", review "What looked
-// solid": two-level global + FP8-block scaling, effective = block_scale *
-// global_scale, zero blocks guarded; "V4 mxfp4 #1372", review of
+// solid": two-level global + FP8-block scaling, the effective scale being the
+// block scale times the global scale, zero blocks guarded; "V4 mxfp4 #1372", review of
 // fp4_act_quant: E2M1 packed two per byte, N % block_size == 0), in fp32:
 //   g     = A / 2688                       A = max |x| over non-NaN elements
 //   s_b   = E4M3(amax_b / (6 g))           per block of 16, RNE, saturating
@@ -88,22 +88,22 @@ inline bool aligned32(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 
 // ------------------------------------------------------------- amax pass
 
+// max |x| over the non-NaN elements of 16-element chunks [c0, c1) (chunk c
+// = row c / cpr, columns 16 (c % cpr) ..), taken by CTA j of `ctas` CTAs that
+// share the range; 0 for a thread with no chunk.
 template <typename InT, bool V8, bool STRIDED>
-__global__ void __launch_bounds__(kThreads, kAmaxCtasPerSm)
-nvfp4_amax_kernel(const InT* __restrict__ x, uint64_t nchunks, uint32_t cpr, FastDiv rowdiv,
-                  int64_t ld, float* __restrict__ partials) {
-  pdl_enter();
+__device__ __forceinline__ float amax_chunks(const InT* __restrict__ x, uint64_t c0, uint64_t c1,
+                                             uint64_t j, uint64_t ctas, uint32_t cpr,
+                                             FastDiv rowdiv, int64_t ld) {
   constexpr int steps = sizeof(InT) == 2 ? kAmaxSteps : 1;  // 64 bytes in flight per thread
-  __shared__ float red[kThreads / 32];
   float m = 0.0f;
-  const uint64_t per_iter = uint64_t(gridDim.x) * kThreads * steps;
-  for (uint64_t base = uint64_t(blockIdx.x) * kThreads * steps; base < nchunks;
-       base += per_iter) {
+  const uint64_t per_iter = ctas * kThreads * steps;
+  for (uint64_t base = c0 + j * kThreads * steps; base < c1; base += per_iter) {
     In16<InT> v[steps];
 #pragma unroll
     for (int u = 0; u < steps; u++) {
       const uint64_t c = base + uint64_t(u) * kThreads + threadIdx.x;
-      if (c < nchunks) {
+      if (c < c1) {
         uint64_t off;
         if constexpr (STRIDED) {
           const uint64_t r = rowdiv.div(c);
@@ -119,6 +119,16 @@ nvfp4_amax_kernel(const InT* __restrict__ x, uint64_t nchunks, uint32_t cpr, Fas
 #pragma unroll
     for (int u = 0; u < steps; u++) m = fmaxf(m, v[u].absmax());
   }
+  return m;
+}
+
+template <typename InT, bool V8, bool STRIDED>
+__global__ void __launch_bounds__(kThreads, kAmaxCtasPerSm)
+nvfp4_amax_kernel(const InT* __restrict__ x, uint64_t nchunks, uint32_t cpr, FastDiv rowdiv,
+                  int64_t ld, float* __restrict__ partials) {
+  pdl_enter();
+  __shared__ float red[kThreads / 32];
+  float m = amax_chunks<InT, V8, STRIDED>(x, 0, nchunks, blockIdx.x, gridDim.x, cpr, rowdiv, ld);
   m = block_max(m, red);
   if (threadIdx.x == 0) partials[blockIdx.x] = m;
 }
@@ -251,15 +261,13 @@ __device__ __forceinline__ uint2 e2m1_codes(const In16<InT>& v, float eff) {
   return e2m1_exact(x, eff);
 }
 
-template <typename InT, bool V8, bool STRIDED, int GMODE>
-__global__ void __launch_bounds__(kThreads)
-nvfp4_quant_kernel(const __grid_constant__ QuantArgs a) {
-  pdl_enter();
-  __shared__ float red[kThreads / 32];
-  const uint32_t tile = a.ntiles - 1 - blockIdx.x;
-  const uint64_t tb0 = uint64_t(tile) * kBlocksPerTile;
-  const uint64_t left = a.nblocks - tb0;
-  const uint32_t nt = left < kBlocksPerTile ? uint32_t(left) : uint32_t(kBlocksPerTile);
+// Quantizes the tile of blocks [tb0, tb0 + nt) (block = 16 elements, row-
+// major over the [M, N] view): all loads are issued first, then get_g()
+// supplies the global scale (it may reduce partial maxima meanwhile; every
+// thread of the CTA calls it), then scales and codes are written.
+template <typename InT, bool V8, bool STRIDED, typename GetG>
+__device__ __forceinline__ void quant_tile(const QuantArgs& a, uint64_t tb0, uint32_t nt,
+                                           GetG get_g) {
   const bool full = nt == kBlocksPerTile;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const uint32_t lb0 = warp * kBlocksPerWarp + lane;
@@ -280,21 +288,7 @@ nvfp4_quant_kernel(const __grid_constant__ QuantArgs a) {
     if (full || lb < nt) v[u].template load<V8>(p); else v[u].zero();
   }
 
-  float g;
-  if constexpr (GMODE == kGiven) {
-    g = *a.gs;
-  } else {
-    float A;
-    if constexpr (GMODE == kFromAmax) {
-      A = *a.amax_in;
-    } else {
-      float m = 0.0f;
-      for (uint32_t i = threadIdx.x; i < a.npartials; i += kThreads) m = fmaxf(m, a.partials[i]);
-      A = block_max(m, red);
-    }
-    g = __fdiv_rn(A, 2688.0f);
-    if (blockIdx.x == 0 && threadIdx.x == 0) *a.gs = g;
-  }
+  const float g = get_g();
   const bool gzero = (g == 0.0f);
   const float t = __fmul_rn(6.0f, g);
   const bool t_ok = rcp_safe(t);
@@ -320,6 +314,131 @@ nvfp4_quant_kernel(const __grid_constant__ QuantArgs a) {
     st_v2(pk + lb * 8, e2m1_codes(v[u], eff));
     st_u8(sc + lb, sb);
   }
+}
+
+template <typename InT, bool V8, bool STRIDED, int GMODE>
+__global__ void __launch_bounds__(kThreads)
+nvfp4_quant_kernel(const __grid_constant__ QuantArgs a) {
+  pdl_enter();
+  __shared__ float red[kThreads / 32];
+  const uint32_t tile = a.ntiles - 1 - blockIdx.x;
+  const uint64_t tb0 = uint64_t(tile) * kBlocksPerTile;
+  const uint64_t left = a.nblocks - tb0;
+  const uint32_t nt = left < kBlocksPerTile ? uint32_t(left) : uint32_t(kBlocksPerTile);
+  quant_tile<InT, V8, STRIDED>(a, tb0, nt, [&]() {
+    float g;
+    if constexpr (GMODE == kGiven) {
+      g = *a.gs;
+    } else {
+      float A;
+      if constexpr (GMODE == kFromAmax) {
+        A = *a.amax_in;
+      } else {
+        float m = 0.0f;
+        for (uint32_t i = threadIdx.x; i < a.npartials; i += kThreads) m = fmaxf(m, a.partials[i]);
+        A = block_max(m, red);
+      }
+      g = __fdiv_rn(A, 2688.0f);
+      if (blockIdx.x == 0 && threadIdx.x == 0) *a.gs = g;
+    }
+    return g;
+  });
+}
+
+// ------------------------------------------------ per-slice global scales
+
+// A tensor cut into S consecutive row ranges ("slices"), each with its own
+// global scale. Block (= amax chunk) ranges, amax-pass CTAs and quant tiles
+// are assigned per slice, so no CTA spans two slices.
+template <int MAXS>
+struct SliceTable {
+  int32_t S;
+  uint64_t bbase[MAXS + 1];  // first block of slice s; bbase[S] = all blocks
+  uint32_t cbase[MAXS + 1];  // first amax-pass CTA (= partial) of slice s
+  uint32_t tbase[MAXS + 1];  // first quant tile of slice s
+};
+
+// The slice whose range [base[s], base[s+1]) holds v (v < base[S]).
+__device__ __forceinline__ int find_slice(const uint32_t* base, int S, uint32_t v) {
+  int lo = 0, hi = S;  // invariant: base[lo] <= v < base[hi]
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (base[mid] <= v) lo = mid; else hi = mid;
+  }
+  return lo;
+}
+
+template <typename InT, bool V8, bool STRIDED, int MAXS>
+__global__ void __launch_bounds__(kThreads, kAmaxCtasPerSm)
+nvfp4_amax_sliced_kernel(const InT* __restrict__ x, uint32_t cpr, FastDiv rowdiv, int64_t ld,
+                         float* __restrict__ partials, const __grid_constant__ SliceTable<MAXS> t) {
+  pdl_enter();
+  __shared__ float red[kThreads / 32];
+  const int s = find_slice(t.cbase, t.S, blockIdx.x);
+  float m = amax_chunks<InT, V8, STRIDED>(x, t.bbase[s], t.bbase[s + 1], blockIdx.x - t.cbase[s],
+                                          t.cbase[s + 1] - t.cbase[s], cpr, rowdiv, ld);
+  m = block_max(m, red);
+  if (threadIdx.x == 0) partials[blockIdx.x] = m;
+}
+
+// One warp per slice: max over the slice's partials into amax[s] (0 for an
+// empty slice).
+template <int MAXS>
+__global__ void __launch_bounds__(kThreads)
+nvfp4_amax_sliced_finalize_kernel(const float* __restrict__ partials, float* __restrict__ amax,
+                                  const __grid_constant__ SliceTable<MAXS> t) {
+  pdl_enter();
+  const int lane = threadIdx.x & 31;
+  const int s = blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5);
+  if (s >= t.S) return;
+  float m = 0.0f;
+  for (uint32_t i = t.cbase[s] + lane; i < t.cbase[s + 1]; i += 32) m = fmaxf(m, partials[i]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(kFull, m, o));
+  if (lane == 0) amax[s] = m;
+}
+
+template <typename InT, bool V8, bool STRIDED, int GMODE, int MAXS>
+__global__ void __launch_bounds__(kThreads)
+nvfp4_quant_sliced_kernel(const __grid_constant__ QuantArgs a,
+                          const __grid_constant__ SliceTable<MAXS> t) {
+  pdl_enter();
+  __shared__ float red[kThreads / 32];
+  if constexpr (GMODE != kGiven) {
+    // global scales of empty slices (no tile of theirs runs)
+    if (blockIdx.x == 0) {
+      for (int e = threadIdx.x; e < t.S; e += kThreads) {
+        if (t.bbase[e] == t.bbase[e + 1]) {
+          if constexpr (GMODE == kFromAmax) a.gs[e] = __fdiv_rn(a.amax_in[e], 2688.0f);
+          else a.gs[e] = 0.0f;
+        }
+      }
+    }
+  }
+  const uint32_t tile = a.ntiles - 1 - blockIdx.x;
+  const int s = find_slice(t.tbase, t.S, tile);
+  const uint64_t tb0 = t.bbase[s] + uint64_t(tile - t.tbase[s]) * kBlocksPerTile;
+  const uint64_t left = t.bbase[s + 1] - tb0;
+  const uint32_t nt = left < kBlocksPerTile ? uint32_t(left) : uint32_t(kBlocksPerTile);
+  quant_tile<InT, V8, STRIDED>(a, tb0, nt, [&]() {
+    float g;
+    if constexpr (GMODE == kGiven) {
+      g = a.gs[s];
+    } else {
+      float A;
+      if constexpr (GMODE == kFromAmax) {
+        A = a.amax_in[s];
+      } else {
+        float m = 0.0f;
+        for (uint32_t i = t.cbase[s] + threadIdx.x; i < t.cbase[s + 1]; i += kThreads)
+          m = fmaxf(m, a.partials[i]);
+        A = block_max(m, red);
+      }
+      g = __fdiv_rn(A, 2688.0f);
+      if (tile == t.tbase[s] && threadIdx.x == 0) a.gs[s] = g;
+    }
+    return g;
+  });
 }
 
 // --------------------------------------------------------------- dequant
@@ -480,6 +599,132 @@ mxq_status check_input(const void* x, int dt, int64_t M, int64_t N, int64_t ld_x
   return MXQ_OK;
 }
 
+// ------------------------------------------------------- sliced (host)
+
+mxq_status check_slices(int32_t S, const int64_t* rows, int64_t M) {
+  if (S < 1 || S > MXQ_NVFP4_MAX_SLICES) return MXQ_ERR_SHAPE;
+  if (!rows) return MXQ_ERR_NULL;
+  int64_t total = 0;
+  for (int32_t s = 0; s < S; s++) {
+    if (rows[s] < 0 || rows[s] > M - total) return MXQ_ERR_SHAPE;
+    total += rows[s];
+  }
+  return total == M ? MXQ_OK : MXQ_ERR_SHAPE;
+}
+
+// Block, amax-CTA and tile ranges per slice. The amax pass gets about
+// min(2048, SMs x 8) CTAs in all, shared out in proportion to the slices'
+// sizes, at least one per non-empty slice (so at most 2048 + S partials).
+template <int MAXS>
+mxq_status build_slices(int32_t S, const int64_t* rows, int64_t N, SliceTable<MAXS>& t) {
+  const uint64_t bpr = uint64_t(N) / 16;
+  uint64_t total = 0;
+  for (int32_t s = 0; s < S; s++) total += uint64_t(rows[s]) * bpr;
+  const uint64_t per_cta = uint64_t(kThreads) * kAmaxSteps;
+  const uint64_t K = std::min<uint64_t>(kMaxPartials, uint64_t(sm_count()) * kAmaxCtasPerSm);
+  uint64_t b = 0, c = 0, tl = 0;
+  t.S = S;
+  for (int32_t s = 0; s < S; s++) {
+    t.bbase[s] = b;
+    t.cbase[s] = uint32_t(c);
+    t.tbase[s] = uint32_t(tl);
+    const uint64_t n = uint64_t(rows[s]) * bpr;
+    if (n) {
+      uint64_t cs = uint64_t((unsigned __int128)K * n / total);
+      const uint64_t need = (n + per_cta - 1) / per_cta;
+      cs = cs > need ? need : cs;
+      c += cs < 1 ? 1 : cs;
+    }
+    tl += (n + kBlocksPerTile - 1) / kBlocksPerTile;
+    b += n;
+    if (tl > 0x7fffffffull) return MXQ_ERR_SHAPE;
+  }
+  t.bbase[S] = b;
+  t.cbase[S] = uint32_t(c);
+  t.tbase[S] = uint32_t(tl);
+  return MXQ_OK;
+}
+
+template <typename InT, bool V8, bool STRIDED, int MAXS>
+cudaError_t launch_amax_sliced_kernel(const void* x, uint32_t cpr, FastDiv rd, int64_t ld,
+                                      float* partials, const SliceTable<MAXS>& t, cudaStream_t s) {
+  return launch_pdl(nvfp4_amax_sliced_kernel<InT, V8, STRIDED, MAXS>, t.cbase[t.S], s,
+                    static_cast<const InT*>(x), cpr, rd, ld, partials, t);
+}
+
+template <int MAXS>
+mxq_status launch_amax_sliced(const void* x, int dt, int64_t N, int64_t ld, float* partials,
+                              const SliceTable<MAXS>& t, cudaStream_t s) {
+  const uint32_t cpr = uint32_t(uint64_t(N) / 16);
+  const FastDiv rd = FastDiv::make(cpr);
+  const bool strided = ld != N;
+  const bool v8 = aligned32(x) && (uint64_t(ld) * elem_size(dt)) % 32 == 0;
+#define MXQ_AMAX_S(T, V, S) e = launch_amax_sliced_kernel<T, V, S, MAXS>(x, cpr, rd, ld, partials, t, s)
+  cudaError_t e;
+  if (dt == MXQ_BF16) {
+    if (v8) { if (strided) MXQ_AMAX_S(uint16_t, true, true); else MXQ_AMAX_S(uint16_t, true, false); }
+    else { if (strided) MXQ_AMAX_S(uint16_t, false, true); else MXQ_AMAX_S(uint16_t, false, false); }
+  } else {
+    if (v8) { if (strided) MXQ_AMAX_S(float, true, true); else MXQ_AMAX_S(float, true, false); }
+    else { if (strided) MXQ_AMAX_S(float, false, true); else MXQ_AMAX_S(float, false, false); }
+  }
+#undef MXQ_AMAX_S
+  return launched(e);
+}
+
+template <typename InT, bool V8, bool STRIDED, int MAXS>
+mxq_status launch_quant_sliced_mode(const QuantArgs& a, const SliceTable<MAXS>& t, int mode,
+                                    cudaStream_t s) {
+  switch (mode) {
+    case kGiven:
+      return launched(launch_pdl(nvfp4_quant_sliced_kernel<InT, V8, STRIDED, kGiven, MAXS>, a.ntiles, s, a, t));
+    case kFromAmax:
+      return launched(launch_pdl(nvfp4_quant_sliced_kernel<InT, V8, STRIDED, kFromAmax, MAXS>, a.ntiles, s, a, t));
+    default:
+      return launched(launch_pdl(nvfp4_quant_sliced_kernel<InT, V8, STRIDED, kFromPartials, MAXS>, a.ntiles, s, a, t));
+  }
+}
+
+template <typename InT, int MAXS>
+mxq_status launch_quant_sliced_typed(const QuantArgs& a, const SliceTable<MAXS>& t, int mode,
+                                     bool v8, bool strided, cudaStream_t s) {
+  if (v8) return strided ? launch_quant_sliced_mode<InT, true, true, MAXS>(a, t, mode, s)
+                         : launch_quant_sliced_mode<InT, true, false, MAXS>(a, t, mode, s);
+  return strided ? launch_quant_sliced_mode<InT, false, true, MAXS>(a, t, mode, s)
+                 : launch_quant_sliced_mode<InT, false, false, MAXS>(a, t, mode, s);
+}
+
+template <int MAXS>
+mxq_status amax_sliced_impl(const void* x, int dt, int64_t N, int64_t ld_x, int32_t S,
+                            const int64_t* rows, float* amax, float* partials, cudaStream_t s) {
+  SliceTable<MAXS> t;
+  mxq_status st = build_slices<MAXS>(S, rows, N, t);
+  if (st != MXQ_OK) return st;
+  st = launch_amax_sliced<MAXS>(x, dt, N, ld_x, partials, t, s);
+  if (st != MXQ_OK) return st;
+  const uint32_t grid = uint32_t((S + kThreads / 32 - 1) / (kThreads / 32));
+  return launched(launch_pdl(nvfp4_amax_sliced_finalize_kernel<MAXS>, grid, s,
+                             static_cast<const float*>(partials), amax, t));
+}
+
+template <int MAXS>
+mxq_status quantize_sliced_impl(QuantArgs& a, int dt, int64_t N, int64_t ld_x, int32_t S,
+                                const int64_t* rows, int mode, float* partials, cudaStream_t s) {
+  SliceTable<MAXS> t;
+  mxq_status st = build_slices<MAXS>(S, rows, N, t);
+  if (st != MXQ_OK) return st;
+  a.ntiles = t.tbase[S];
+  if (mode == kFromPartials) {
+    a.partials = partials;
+    st = launch_amax_sliced<MAXS>(a.x, dt, N, ld_x, partials, t, s);
+    if (st != MXQ_OK) return st;
+  }
+  const bool strided = ld_x != N;
+  const bool v8 = aligned32(a.x) && (uint64_t(ld_x) * elem_size(dt)) % 32 == 0;
+  if (dt == MXQ_BF16) return launch_quant_sliced_typed<uint16_t, MAXS>(a, t, mode, v8, strided, s);
+  return launch_quant_sliced_typed<float, MAXS>(a, t, mode, v8, strided, s);
+}
+
 }  // namespace
 }  // namespace mxq
 
@@ -549,6 +794,71 @@ mxq_status nvfp4_quantize(const void* x, int dt, int64_t M, int64_t N, int64_t l
   const bool v8 = aligned32(x) && (uint64_t(ld_x) * elem_size(dt)) % 32 == 0;
   if (dt == MXQ_BF16) return launch_quant_typed<uint16_t>(a, mode, v8, strided, s);
   return launch_quant_typed<float>(a, mode, v8, strided, s);
+}
+
+size_t mxq_nvfp4_sliced_workspace_bytes(int32_t n_slices) {
+  if (n_slices < 1 || n_slices > MXQ_NVFP4_MAX_SLICES) return 0;
+  return sizeof(float) * (size_t(mxq::kMaxPartials) + size_t(n_slices));
+}
+
+mxq_status nvfp4_amax_sliced(const void* x, int dt, int64_t M, int64_t N, int64_t ld_x,
+                             int32_t n_slices, const int64_t* slice_rows, float* amax,
+                             void* workspace, size_t ws_bytes, mxq_stream_t stream) {
+  using namespace mxq;
+  mxq_status st = check_input(x, dt, M, N, ld_x);
+  if (st != MXQ_OK) return st;
+  st = check_slices(n_slices, slice_rows, M);
+  if (st != MXQ_OK) return st;
+  if (M == 0 || N == 0) return MXQ_OK;
+  if (!amax) return MXQ_ERR_NULL;
+  if (!workspace || ws_bytes < mxq_nvfp4_sliced_workspace_bytes(n_slices) ||
+      (reinterpret_cast<uintptr_t>(workspace) & 3u))
+    return MXQ_ERR_WORKSPACE;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  float* partials = static_cast<float*>(workspace);
+  if (n_slices <= 64)
+    return amax_sliced_impl<64>(x, dt, N, ld_x, n_slices, slice_rows, amax, partials, s);
+  return amax_sliced_impl<MXQ_NVFP4_MAX_SLICES>(x, dt, N, ld_x, n_slices, slice_rows, amax,
+                                                 partials, s);
+}
+
+mxq_status nvfp4_quantize_sliced(const void* x, int dt, int64_t M, int64_t N, int64_t ld_x,
+                                 int32_t n_slices, const int64_t* slice_rows, uint8_t* packed,
+                                 uint8_t* block_scale, float* global_scales,
+                                 const float* amax_in, uint32_t flags, void* workspace,
+                                 size_t ws_bytes, mxq_stream_t stream) {
+  using namespace mxq;
+  if (flags & ~MXQ_NVFP4_GLOBAL_GIVEN) return MXQ_ERR_ARG;
+  const bool given = (flags & MXQ_NVFP4_GLOBAL_GIVEN) != 0;
+  if (given && amax_in) return MXQ_ERR_ARG;
+  mxq_status st = check_input(x, dt, M, N, ld_x);
+  if (st != MXQ_OK) return st;
+  st = check_slices(n_slices, slice_rows, M);
+  if (st != MXQ_OK) return st;
+  if (M == 0 || N == 0) return MXQ_OK;
+  if (!packed || !block_scale || !global_scales) return MXQ_ERR_NULL;
+  if (!aligned16(packed)) return MXQ_ERR_ALIGN;
+  const bool pass1 = !given && !amax_in;
+  if (pass1 && (!workspace || ws_bytes < mxq_nvfp4_sliced_workspace_bytes(n_slices) ||
+                (reinterpret_cast<uintptr_t>(workspace) & 3u)))
+    return MXQ_ERR_WORKSPACE;
+  QuantArgs a{};
+  a.x = x;
+  a.ld = ld_x;
+  a.bpr = uint32_t(uint64_t(N) / 16);
+  a.rowdiv = FastDiv::make(a.bpr);
+  a.packed = packed;
+  a.bscale = block_scale;
+  a.gs = global_scales;
+  a.amax_in = amax_in;
+  a.nblocks = uint64_t(M) * a.bpr;
+  const int mode = given ? kGiven : (amax_in ? kFromAmax : kFromPartials);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  float* partials = static_cast<float*>(workspace);
+  if (n_slices <= 64)
+    return quantize_sliced_impl<64>(a, dt, N, ld_x, n_slices, slice_rows, mode, partials, s);
+  return quantize_sliced_impl<MXQ_NVFP4_MAX_SLICES>(a, dt, N, ld_x, n_slices, slice_rows, mode,
+                                                     partials, s);
 }
 
 mxq_status nvfp4_dequantize(const uint8_t* packed, const uint8_t* block_scale,

@@ -75,13 +75,14 @@ def lib() -> ctypes.CDLL:
             L.orc_nvfp4_global_amax.restype = f32
             L.orc_nvfp4_quantize.argtypes = [vp, i32, i64, i64, i64, vp, vp, vp, i32]
             L.orc_nvfp4_dequantize.argtypes = [vp, vp, f32, i64, i64, vp, i32]
+            L.orc_nvfp4_quantize_sliced.argtypes = [vp, i32, i64, i64, i64, i32, vp, vp, vp, vp, i32]
             for f in ("orc_e4m3_encode_array", "orc_e2m1_encode_array",
                       "orc_e8m0_from_amax_array", "orc_bf16_round_array"):
                 getattr(L, f).argtypes = [vp, i64, vp]
                 getattr(L, f).restype = None
             for f in ("orc_mxfp8_quantize", "orc_mxfp8_dequantize", "orc_swizzle_scales",
                       "orc_mxfp8_quantize_colwise", "orc_mxfp4_quantize", "orc_mxfp4_dequantize",
-                      "orc_nvfp4_quantize", "orc_nvfp4_dequantize"):
+                      "orc_nvfp4_quantize", "orc_nvfp4_dequantize", "orc_nvfp4_quantize_sliced"):
                 getattr(L, f).restype = i32
             _lib = L
     return _lib
@@ -311,6 +312,27 @@ def nvfp4_quantize(x: np.ndarray, global_scale: float | None = None):
     _check(lib().orc_nvfp4_quantize(_ptr(a), dt, M, N, N, _ptr(packed), _ptr(bs), _ptr(g), given),
            "nvfp4_quantize")
     return packed, bs, np.float32(g[0])
+
+
+def nvfp4_quantize_sliced(x: np.ndarray, slice_rows, global_scales=None):
+    """NVFP4 with one global scale per slice of consecutive rows ("Add FP8,
+    NVFP4, and QARL training and export", _nvfp4_block_quantize_per_slice;
+    per-half gate/up scales). Returns (packed [M, N/2], block_scale [M, N/16],
+    g float32 [n_slices])."""
+    a, dt = _as_input(x)
+    M, N = a.shape
+    rows = np.ascontiguousarray(slice_rows, np.int64)
+    S = rows.shape[0]
+    packed = np.empty((M, N // 2), np.uint8)
+    bs = np.empty((M, N // 16), np.uint8)
+    g = np.zeros(S, np.float32)
+    given = 0
+    if global_scales is not None:
+        g[:] = np.asarray(global_scales, np.float32)
+        given = 1
+    _check(lib().orc_nvfp4_quantize_sliced(_ptr(a), dt, M, N, N, S, _ptr(rows), _ptr(packed),
+                                           _ptr(bs), _ptr(g), given), "nvfp4_quantize_sliced")
+    return packed, bs, g
 
 
 def nvfp4_dequantize(packed: np.ndarray, bs: np.ndarray, g: float, out: str = "bf16") -> np.ndarray:

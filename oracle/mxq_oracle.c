@@ -10,7 +10,7 @@
  * Every function writes out the plain definition of what it computes, one
  * element at a time, in double precision (exact for every MXFP8 step), except
  * the NVFP4 scale arithmetic, which the pages fix as fp32 (global FP32 scale,
- * "effective = block_scale * global_scale") and is therefore done in IEEE
+ * the effective scale as block scale times global scale) and is therefore done in IEEE
  * binary32 with round-to-nearest-even, subnormals kept, no contraction.
  * Build: gcc -O2 -std=c11 -fno-fast-math -ffp-contract=off -fPIC -shared.
  *
@@ -24,8 +24,9 @@
  *        float8_e8m0fnu scale dtype; review: E2M1 packed two per byte
  *        (float4_e2m1fn_x2, last dim N//2), N % block_size == 0.
  *  [P2]  "Add FP8, NVFP4, and QARL training and export", review "What looked
- *        solid": NVFP4 two-level global + FP8-block scaling, "effective =
- *        block_scale * global_scale", zero blocks guarded (safe_eff).
+ *        solid": NVFP4 two-level global + FP8-block scaling, the effective
+ *        scale being the block scale times the global scale, zero blocks
+ *        guarded (safe_eff).
  *  The E8M0 rule (scale = 2^(floor(log2 amax) - 8), biased byte clamped to
  *  [0,254], all-zero group -> 127), the E4M3 cast (RNE, saturate to +-448,
  *  NaN propagated) and the NVFP4 global scale amax/(448*6) are the statement
@@ -318,7 +319,7 @@ float orc_nvfp4_global_amax(const void* x, int dt, int64_t M, int64_t N, int64_t
  *                                         of x_i's sign when eff == 0;
  *   packed[r, k] = q[r, 2k] | q[r, 2k+1] << 4.
  * Readings: the order of the fp32 operations is the one written above (the
- * pages give only "effective = block_scale * global_scale"); a zero global
+ * pages give only that the effective scale is block scale times global scale); a zero global
  * scale gives s_b = 0 and zero codes with no division; the zero-block guard
  * writes sign-kept zero codes. Non-finite inputs are outside the method's
  * contract: the same fp32 operations are applied, with no further meaning. */
@@ -512,6 +513,45 @@ int orc_mxfp4_dequantize(const uint8_t* packed, const uint8_t* scale, int64_t M,
       double d = orc_e2m1_decode(code) * orc_e8m0_value(scale[r * S + c / 32]);
       store_out(y, out_dt, r * N + c, d);
     }
+  }
+  return ORC_OK;
+}
+
+/* ------------------------------------------ NVFP4 with per-slice global scale */
+
+/* NVFP4 quantize of x [M, N] cut into n_slices consecutive row ranges
+ * (slice s holds slice_rows[s] rows, the ranges following each other and
+ * covering all M rows), each with its own global scale ("Add FP8, NVFP4, and
+ * QARL training and export", review: _nvfp4_block_quantize_per_slice and
+ * weight_scale_2 per expert; non-blocking item 3: a fused gate/up weight
+ * takes one global scale per half during QAT, one shared scale per expert at
+ * export). Each slice is quantized exactly as orc_nvfp4_quantize quantizes a
+ * tensor holding only that slice's rows, with g_io[s] as its global scale
+ * (read when g_given, else written as slice amax / 2688; an empty slice has
+ * amax 0 and g 0).
+ * Reading: a slice is a range of rows (dim -2 of the stacked [E, R, N]
+ * weight): an expert, or one half (gate: first R/2 rows, up: last R/2) of an
+ * expert's fused gate/up rows. Blocks of 16 run along the last dim and so
+ * never cross a slice. */
+int orc_nvfp4_quantize_sliced(const void* x, int dt, int64_t M, int64_t N, int64_t ld_x,
+                              int32_t n_slices, const int64_t* slice_rows, uint8_t* packed,
+                              uint8_t* block_scale, float* g_io, int g_given) {
+  if (dt != ORC_BF16 && dt != ORC_FP32) return ORC_ERR_DTYPE;
+  if (M < 0 || N < 0 || N % 16 != 0 || ld_x < N || n_slices < 1) return ORC_ERR_SHAPE;
+  int64_t total = 0;
+  for (int32_t s = 0; s < n_slices; s++) {
+    if (slice_rows[s] < 0) return ORC_ERR_SHAPE;
+    total += slice_rows[s];
+  }
+  if (total != M) return ORC_ERR_SHAPE;
+  size_t esz = (dt == ORC_BF16) ? 2 : 4;
+  int64_t r0 = 0;
+  for (int32_t s = 0; s < n_slices; s++) {
+    const char* xs = (const char*)x + (size_t)(r0 * ld_x) * esz;
+    int rc = orc_nvfp4_quantize(xs, dt, slice_rows[s], N, ld_x, packed + r0 * (N / 2),
+                                block_scale + r0 * (N / 16), &g_io[s], g_given);
+    if (rc != ORC_OK) return rc;
+    r0 += slice_rows[s];
   }
   return ORC_OK;
 }

@@ -32,7 +32,9 @@ def declared_functions():
 def test_header_declares_expected_entry_points():
     names = declared_functions()
     for f in ("mxfp8_quantize", "mxfp8_dequantize", "mxfp8_quantize_grouped", "nvfp4_quantize",
-              "nvfp4_dequantize", "nvfp4_amax", "mxq_abi_version", "mxq_status_string"):
+              "nvfp4_dequantize", "nvfp4_amax", "mxq_abi_version", "mxq_status_string",
+              "mxfp4_quantize", "mxfp4_dequantize", "mxfp4_quantize_grouped", "mx_fake_quantize",
+              "nvfp4_quantize_sliced", "nvfp4_amax_sliced"):
         assert f in names
 
 
@@ -83,6 +85,43 @@ def test_mxfp8_dequantize_validation():
     assert L.mxfp8_dequantize(A + 4, A, 4, 64, A, 0, None) == ALIGN
     assert L.mxfp8_dequantize(A, A, 4, 64, A + 2, 1, None) == ALIGN
     assert L.mxfp8_dequantize(None, None, 0, 64, None, 0, None) == OK
+
+
+def test_mxfp4_validation():
+    L = mxq.lib
+    assert L.mxfp4_quantize(A, 2, 4, 64, 64, A, A, None, None) == DTYPE
+    assert L.mxfp4_quantize(A, 0, 4, 48, 48, A, A, None, None) == SHAPE
+    assert L.mxfp4_quantize(A, 0, 4, 64, 32, A, A, None, None) == SHAPE
+    assert L.mxfp4_quantize(None, 0, 4, 64, 64, A, A, None, None) == NULL
+    assert L.mxfp4_quantize(A, 0, 4, 64, 64, None, A, None, None) == NULL
+    assert L.mxfp4_quantize(A + 4, 0, 4, 64, 64, A, A, None, None) == ALIGN
+    assert L.mxfp4_quantize(A, 0, 4, 64, 64, A + 8, A, None, None) == ALIGN
+    assert L.mxfp4_quantize(None, 0, 0, 64, 64, None, None, None, None) == OK
+    assert L.mxfp4_dequantize(A, A, 4, 64, A, 5, None) == DTYPE
+    assert L.mxfp4_dequantize(A, A, 4, 80, A, 0, None) == SHAPE
+    assert L.mxfp4_dequantize(A, None, 4, 64, A, 0, None) == NULL
+    assert L.mxfp4_dequantize(A, A, 4, 64, A + 2, 0, None) == ALIGN
+    rows = (ctypes.c_int64 * 2)(4, 0)
+    ptrs = (ctypes.c_void_p * 2)(A, None)
+    assert L.mxfp4_quantize_grouped(0, ptrs, rows, 64, 0, A, A, None) == SHAPE
+    assert L.mxfp4_quantize_grouped(2, ptrs, rows, 40, 0, A, A, None) == SHAPE
+    assert L.mxfp4_quantize_grouped(2, ptrs, rows, 64, 0, None, A, None) == NULL
+
+
+def test_fake_quantize_validation():
+    L = mxq.lib
+    assert L.mx_fake_quantize(2, A, 0, 4, 64, 64, A, 0, None) == ARG
+    assert L.mx_fake_quantize(-1, A, 0, 4, 64, 64, A, 0, None) == ARG
+    assert L.mx_fake_quantize(1, A, 3, 4, 64, 64, A, 0, None) == DTYPE
+    assert L.mx_fake_quantize(1, A, 0, 4, 64, 64, A, 3, None) == DTYPE
+    assert L.mx_fake_quantize(0, A, 0, 4, 40, 40, A, 0, None) == SHAPE
+    assert L.mx_fake_quantize(0, A, 0, 4, 64, 32, A, 0, None) == SHAPE
+    assert L.mx_fake_quantize(0, None, 0, 4, 64, 64, A, 0, None) == NULL
+    assert L.mx_fake_quantize(1, A, 0, 4, 64, 64, None, 1, None) == NULL
+    assert L.mx_fake_quantize(1, A + 2, 0, 4, 64, 64, A, 0, None) == ALIGN
+    assert L.mx_fake_quantize(1, A, 0, 4, 64, 66, A, 0, None) == ALIGN
+    assert L.mx_fake_quantize(1, A, 0, 4, 64, 64, A + 4, 1, None) == ALIGN
+    assert L.mx_fake_quantize(0, None, 1, 0, 64, 64, None, 1, None) == OK
 
 
 def test_grouped_validation():
@@ -151,6 +190,37 @@ def test_nvfp4_noalloc_validation():
     assert f(A, 0, 4, 64, 64, A, A, None, None, 0, None) == NULL
     assert f(A, 0, 4, 64, 64, A + 4, A, A, None, 0, None) == ALIGN
     assert f(None, 0, 0, 64, 64, None, None, None, None, 0, None) == OK
+
+
+def test_nvfp4_sliced_validation():
+    L = mxq.lib
+    ws = mxq.lib.mxq_nvfp4_sliced_workspace_bytes(3)
+    assert ws == 4 * (2048 + 3)
+    assert mxq.lib.mxq_nvfp4_sliced_workspace_bytes(0) == 0
+    assert mxq.lib.mxq_nvfp4_sliced_workspace_bytes(1025) == 0
+    rows = (ctypes.c_int64 * 3)(4, 0, 12)
+    bad_sum = (ctypes.c_int64 * 3)(4, 0, 11)
+    neg = (ctypes.c_int64 * 3)(20, -4, 0)
+    Q = L.nvfp4_quantize_sliced
+    assert Q(A, 0, 16, 64, 64, 3, bad_sum, A, A, A, None, 0, A, ws, None) == SHAPE
+    assert Q(A, 0, 16, 64, 64, 3, neg, A, A, A, None, 0, A, ws, None) == SHAPE
+    assert Q(A, 0, 16, 64, 64, 0, rows, A, A, A, None, 0, A, ws, None) == SHAPE
+    assert Q(A, 0, 16, 64, 64, 1025, rows, A, A, A, None, 0, A, ws, None) == SHAPE
+    assert Q(A, 0, 16, 64, 64, 3, None, A, A, A, None, 0, A, ws, None) == NULL
+    assert Q(A, 0, 16, 72, 72, 3, rows, A, A, A, None, 0, A, ws, None) == SHAPE
+    assert Q(A, 0, 16, 64, 64, 3, rows, A, A, None, None, 0, A, ws, None) == NULL
+    assert Q(A, 0, 16, 64, 64, 3, rows, A, A, A, None, 0, None, ws, None) == WORKSPACE
+    assert Q(A, 0, 16, 64, 64, 3, rows, A, A, A, None, 0, A, ws - 4, None) == WORKSPACE
+    assert Q(A, 0, 16, 64, 64, 3, rows, A, A, A, A, 1, None, 0, None) == ARG
+    assert Q(A, 0, 16, 64, 64, 3, rows, A, A, A, None, 2, None, 0, None) == ARG
+    assert Q(A, 0, 16, 64, 64, 3, rows, A + 8, A, A, None, 0, A, ws, None) == ALIGN
+    assert Q(A, 5, 16, 64, 64, 3, rows, A, A, A, None, 0, A, ws, None) == DTYPE
+    zero = (ctypes.c_int64 * 2)(0, 0)
+    assert Q(None, 0, 0, 64, 64, 2, zero, None, None, None, None, 0, None, 0, None) == OK
+    X = L.nvfp4_amax_sliced
+    assert X(A, 0, 16, 64, 64, 3, bad_sum, A, A, ws, None) == SHAPE
+    assert X(A, 0, 16, 64, 64, 3, rows, None, A, ws, None) == NULL
+    assert X(A, 0, 16, 64, 64, 3, rows, A, A, 16, None) == WORKSPACE
 
 
 def test_python_binding_rejects_cpu_tensors():

@@ -178,6 +178,48 @@ def mxfp8_every_value_every_scale() -> np.ndarray:
     return out.reshape(rows, per_row * 32)
 
 
+def mx_every_value_every_exponent() -> np.ndarray:
+    """bf16 [M, 1024] pairing every bf16 pattern with every group-amax
+    exponent field e in 0..255 that can hold it: for e in 1..254 the groups
+    start with 1.5 * 2^(e - 127) (for e == 0 with the largest subnormal,
+    for e == 255 with +inf) followed by every pattern whose exponent field is
+    at most e, and every NaN pattern. Covers every scale byte of any MX
+    element format. Groups are 1 planted + 31 swept elements."""
+    allp = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    mag_e = (allp >> 7) & 0xFF
+    is_nan = ((allp & 0x7FFF) > 0x7F80)
+    groups = []
+    for e in range(256):
+        if e == 0:
+            lead = 0x007F
+        elif e == 255:
+            lead = 0x7F80
+        else:
+            lead = (e << 7) | 0x40
+        vals = allp[((mag_e <= e) & ~is_nan) | is_nan] if e < 255 else allp
+        n = (len(vals) + 30) // 31
+        g = np.zeros((n, 32), np.uint16)
+        g[:, 0] = lead
+        flat = np.zeros(n * 31, np.uint16)
+        flat[:len(vals)] = vals
+        g[:, 1:] = flat.reshape(n, 31)
+        groups.append(g)
+    allg = np.concatenate(groups, 0)
+    rows = (allg.shape[0] + 31) // 32
+    out = np.zeros((rows * 32, 32), np.uint16)
+    out[:allg.shape[0]] = allg
+    return out.reshape(rows, 1024)
+
+
+def mx_all_packed_scale_pairs():
+    """(packed [256, 256], scale [256, 16]): row r carries scale byte r on
+    every group of 32 elements and the 256 byte values (every pair of E2M1
+    codes) once, so every (code, byte) pair is dequantized."""
+    q = np.tile(np.arange(256, dtype=np.uint8), (256, 1))
+    s = np.repeat(np.arange(256, dtype=np.uint8)[:, None], 16, axis=1)
+    return q, s
+
+
 def mxfp8_all_code_scale_pairs():
     """(qweight [256, 8192], scale [256, 256]): row r carries scale byte r on
     every group and the 256 E4M3 codes repeated, so every (code, byte) pair
