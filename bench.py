@@ -59,6 +59,22 @@ def mxfp8_dequant_bytes(M, N, out_bytes=2):
     return E + E // 32 + E * out_bytes
 
 
+def mxfp4_quant_bytes(M, N, in_bytes=2, swizzled=False):
+    E = M * N
+    S = N // 32
+    swz = ((M + 127) // 128 * 128) * ((S + 3) // 4 * 4) if swizzled else 0
+    return E * in_bytes + E // 2 + E // 32 + swz
+
+
+def mxfp4_dequant_bytes(M, N, out_bytes=2):
+    E = M * N
+    return E // 2 + E // 32 + E * out_bytes
+
+
+def fake_quant_bytes(M, N, in_bytes=2, out_bytes=2):
+    return M * N * (in_bytes + out_bytes)
+
+
 def nvfp4_quant_bytes(M, N, in_bytes=2, two_pass=True):
     E = M * N
     return E * in_bytes * (2 if two_pass else 1) + E // 2 + E // 16 + 4
@@ -76,8 +92,10 @@ def hbm_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-KERNEL_SOURCES = {"mxfp8_quant_kernel": ("common.cuh", "mxfp8.cu"),
-                  "mxfp8_dequant_kernel": ("common.cuh", "mxfp8.cu"),
+KERNEL_SOURCES = {"mx_quant_kernel": ("common.cuh", "mx_rowwise.cu"),
+                  "mx_dequant_kernel": ("common.cuh", "mx_rowwise.cu"),
+                  "mx_fake_quant_kernel": ("common.cuh", "mx_rowwise.cu"),
+                  "mxfp8_colwise_kernel": ("common.cuh", "colwise.cu"),
                   "nvfp4_amax_kernel": ("common.cuh", "nvfp4.cu"),
                   "nvfp4_quant_kernel": ("common.cuh", "nvfp4.cu"),
                   "nvfp4_dequant_kernel": ("common.cuh", "nvfp4.cu")}
@@ -379,8 +397,8 @@ def run(args):
     peak, peak_kind = hbm_peak()
     q_avg, d_avg = statistics.fmean(q_ms), statistics.fmean(d_ms)
     kernels = {
-        "mxfp8_quant_kernel": {"avg_us": q_avg * 1e3, "bytes": qb, "gbs": qb / (q_avg / 1e3) / 1e9},
-        "mxfp8_dequant_kernel": {"avg_us": d_avg * 1e3, "bytes": db, "gbs": db / (d_avg / 1e3) / 1e9},
+        "mx_quant_kernel": {"avg_us": q_avg * 1e3, "bytes": qb, "gbs": qb / (q_avg / 1e3) / 1e9},
+        "mx_dequant_kernel": {"avg_us": d_avg * 1e3, "bytes": db, "gbs": db / (d_avg / 1e3) / 1e9},
     }
     for k in kernels.values():
         k["frac_of_measured"] = k["gbs"] / peak
@@ -490,11 +508,36 @@ def run_suite(device, only=None):
              mxfp8_quant_bytes(M_ROWS, N_COLS, in_bytes=4, swizzled=False),
              time_kernel(lambda: mxq.mxfp8_quantize(xf), 30))
 
+    def mxfp4_activation():
+        x = bf(W.activation())
+        emit("mxfp4_quantize activation 16384x7168", mxfp4_quant_bytes(M_ROWS, N_COLS),
+             time_kernel(lambda: mxq.mxfp4_quantize(x), 30))
+        p, s = mxq.mxfp4_quantize(x)
+        emit("mxfp4_dequantize->bf16 activation 16384x7168", mxfp4_dequant_bytes(M_ROWS, N_COLS),
+             time_kernel(lambda: mxq.mxfp4_dequantize(p, s), 30))
+
+    def fake_activation():
+        x = bf(W.activation())
+        for fmt in ("mxfp8", "mxfp4"):
+            emit(f"mx_fake_quantize {fmt} bf16->bf16 activation 16384x7168",
+                 fake_quant_bytes(M_ROWS, N_COLS),
+                 time_kernel(lambda: mxq.mx_fake_quantize(x, fmt), 30))
+
     def experts():
         x = bf(W.experts())
         emit("mxfp8_quantize_grouped experts 64x2048x7168",
              mxfp8_quant_bytes(64 * 2048, 7168, swizzled=False),
              time_kernel(lambda: mxq.mxfp8_quantize_grouped(x), 10))
+        emit("mxfp4_quantize_grouped experts 64x2048x7168",
+             mxfp4_quant_bytes(64 * 2048, 7168),
+             time_kernel(lambda: mxq.mxfp4_quantize_grouped(x), 10))
+        ws = torch.empty(int(mxq.lib.mxq_nvfp4_sliced_workspace_bytes(128)), dtype=torch.uint8,
+                         device=device)
+        for per_half in (False, True):
+            rows = [1024] * 128 if per_half else [2048] * 64
+            emit(f"nvfp4_quantize_sliced (two passes, {'per gate/up half' if per_half else 'per expert'})"
+                 " experts 64x2048x7168", nvfp4_quant_bytes(64 * 2048, 7168),
+                 time_kernel(lambda: mxq.nvfp4_quantize_sliced(x, rows, workspace=ws), 10))
 
     def nvfp4():
         x = bf(W.nvfp4_tensor())
@@ -508,6 +551,7 @@ def run_suite(device, only=None):
              time_kernel(lambda: mxq.nvfp4_dequantize(p, b, g), 30))
 
     for name, fn in (("linear_weight", linear_weight), ("activation", activation),
+                     ("mxfp4 activation", mxfp4_activation), ("fake activation", fake_activation),
                      ("experts", experts), ("nvfp4", nvfp4)):
         if only is None or only in name:
             fn()
