@@ -290,6 +290,31 @@ def fake_quantize(x: np.ndarray, fmt: str, out: str = "bf16") -> np.ndarray:
     raise ValueError(fmt)
 
 
+# --------------------------------------------------------------------- GEMM
+
+def e4m3_decode_table() -> np.ndarray:
+    """float64 values of the 256 E4M3 codes (NaN for 0x7F and 0xFF)."""
+    return np.array([lib().orc_e4m3_decode(c) for c in range(256)], np.float64)
+
+
+def mxfp8_gemm(qa: np.ndarray, sa: np.ndarray, qb: np.ndarray, sb: np.ndarray) -> np.ndarray:
+    """The block-scaled product written out in float64: D = A B^T with
+    A[m, k] = decode(qa[m, k]) * 2^(sa[m, k/32] - 127) and B likewise from
+    (qb, sb). qa [M, K], qb [N, K] E4M3 codes; sa [M, K/32], sb [N, K/32]
+    compact E8M0 bytes. Products are exact; the float64 sums are exact for
+    the test inputs on a coarse grid and within K * 2^-53 of the exact sum
+    otherwise."""
+    qa = np.ascontiguousarray(qa, np.uint8)
+    qb = np.ascontiguousarray(qb, np.uint8)
+    t = e4m3_decode_table()
+    K = qa.shape[1]
+    ea = np.repeat(np.asarray(sa, np.int64) - 127, 32, axis=1)[:, :K]
+    eb = np.repeat(np.asarray(sb, np.int64) - 127, 32, axis=1)[:, :K]
+    A = np.ldexp(t[qa], ea)
+    B = np.ldexp(t[qb], eb)
+    return A @ B.T
+
+
 # -------------------------------------------------------------------- NVFP4
 
 def nvfp4_global_amax(x: np.ndarray) -> np.float32:
