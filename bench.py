@@ -92,6 +92,17 @@ def hbm_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+def tensor_peak():
+    """fp8 dense peak for a kernel timed alone: the measured bf16 burst
+    figure times the nominal fp8 / bf16 ratio of 2."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            return 2.0 * float(json.load(f)["bf16_tflops"]), "measured bf16 burst x 2"
+    except Exception:
+        return 2.0 * 1590.0, "fallback bf16 x 2"
+
+
 KERNEL_SOURCES = {"mx_quant_kernel": ("common.cuh", "mx_rowwise.cu"),
                   "mx_dequant_kernel": ("common.cuh", "mx_rowwise.cu"),
                   "mx_fake_quant_kernel": ("common.cuh", "mx_rowwise.cu"),
@@ -523,6 +534,22 @@ def run_suite(device, only=None):
                  fake_quant_bytes(M_ROWS, N_COLS),
                  time_kernel(lambda: mxq.mx_fake_quantize(x, fmt), 30))
 
+    def gemm():
+        xa = bf(W.activation())
+        xb = bf(W.linear_weight(seed=111, M=7168, N=7168))
+        qa, _, za = mxq.mxfp8_quantize(xa, swizzled=True)
+        qb, _, zb = mxq.mxfp8_quantize(xb, swizzled=True)
+        del xa, xb
+        flops = 2 * M_ROWS * 7168 * N_COLS
+        t = time_kernel(lambda: mxq.mxfp8_gemm(qa, za, qb, zb), 20)
+        med, p10, p90 = t
+        bf16_peak = tensor_peak()
+        print(json.dumps({"suite": "mxfp8_gemm activation 16384x7168 x weight 7168x7168 -> bf16",
+                          "median_us": med * 1e3, "p10_us": p10 * 1e3, "p90_us": p90 * 1e3,
+                          "tflops": flops / med / 1e9,
+                          "frac_of_fp8_peak": flops / med / 1e9 / bf16_peak[0],
+                          "fp8_peak_tflops": bf16_peak[0], "peak_kind": bf16_peak[1]}), flush=True)
+
     def experts():
         x = bf(W.experts())
         emit("mxfp8_quantize_grouped experts 64x2048x7168",
@@ -550,7 +577,7 @@ def run_suite(device, only=None):
         emit("nvfp4_dequantize->bf16 8192x8192", 8192 * 8192 // 2 + 8192 * 512 + 8192 * 8192 * 2,
              time_kernel(lambda: mxq.nvfp4_dequantize(p, b, g), 30))
 
-    for name, fn in (("linear_weight", linear_weight), ("activation", activation),
+    for name, fn in (("gemm", gemm), ("linear_weight", linear_weight), ("activation", activation),
                      ("mxfp4 activation", mxfp4_activation), ("fake activation", fake_activation),
                      ("experts", experts), ("nvfp4", nvfp4)):
         if only is None or only in name:

@@ -212,6 +212,32 @@ mxq_status mxfp4_quantize_grouped(int32_t E, const void* const* xs, const int64_
 mxq_status mx_fake_quantize(int fmt, const void* x, int dt, int64_t M, int64_t N, int64_t ld_x,
                             void* y, int out_dt, mxq_stream_t stream);
 
+/* ------------------------------------------------ block-scaled MXFP8 GEMM */
+
+/* D = A * B^T on the tensor cores (tcgen05 kind::mxf8f6f4.block_scale), the
+ * consumer of mxfp8_quantize's codes and swizzled scales:
+ *   D[m, n] = sum_k decode(qa[m, k]) 2^(sa[m, k/32] - 127)
+ *                 * decode(qb[n, k]) 2^(sb[n, k/32] - 127),
+ * products exact, accumulated in fp32 in an order of the hardware's choosing.
+ * (The pages quantize weights and activations for block-scaled GEMMs: "V4
+ * mxfp4 #1372", description; "PR #1935 完整报告 ...", 功能与动机. This entry
+ * point is the consumer that reads the swizzled scale layout.)
+ *  qa      [M, K] uint8 E4M3 codes, row-major (mxfp8_quantize of A).
+ *  sa_swz  mxq_swizzled_scale_bytes(M, K/32) bytes: A's scales in the
+ *          128x4-tile layout (mxfp8_quantize's scale_swz).
+ *  qb      [N, K] uint8 E4M3 codes, row-major (B as a linear layer's
+ *          [out, in] weight), sb_swz its swizzled scales.
+ *  d       [M, N] row-major, bf16 (RNE of the fp32 sum) or fp32 (out_dt).
+ *  error_flag  NULL, or a device int32 that the kernel sets to a non-zero
+ *          code if one of its waits gives up (after about one second); the
+ *          result is then undefined. It is never cleared by the library.
+ * K % 32 == 0, N % 16 == 0; all pointers 16-byte aligned. K == 0 writes
+ * zeros. One launch of ceil(M/128) x ceil(N/128) CTAs of 128 threads with
+ * about 200 KB of shared memory each. */
+mxq_status mxfp8_gemm(const uint8_t* qa, const uint8_t* sa_swz, const uint8_t* qb,
+                      const uint8_t* sb_swz, int64_t M, int64_t N, int64_t K, void* d,
+                      int out_dt, int32_t* error_flag, mxq_stream_t stream);
+
 /* ------------------------------------------------------------------ NVFP4 */
 
 /* Workspace bytes nvfp4_quantize / nvfp4_amax need (per-CTA partial maxima of

@@ -24,6 +24,7 @@ __all__ = [
     "MxqError", "lib", "library_path",
     "mxfp8_quantize", "mxfp8_dequantize", "mxfp8_quantize_grouped", "mxfp8_quantize_columnwise",
     "mxfp4_quantize", "mxfp4_dequantize", "mxfp4_quantize_grouped", "mx_fake_quantize",
+    "mxfp8_gemm",
     "nvfp4_amax", "nvfp4_quantize", "nvfp4_dequantize",
     "nvfp4_amax_sliced", "nvfp4_quantize_sliced", "nvfp4_quantize_experts",
     "swizzled_scale_bytes", "nvfp4_workspace_bytes",
@@ -67,6 +68,7 @@ def _load() -> ctypes.CDLL:
     L.mxfp4_dequantize.argtypes = [vp, vp, i64, i64, vp, i32, vp]
     L.mxfp4_quantize_grouped.argtypes = [i32, vp, vp, i64, i32, vp, vp, vp]
     L.mx_fake_quantize.argtypes = [i32, vp, i32, i64, i64, i64, vp, i32, vp]
+    L.mxfp8_gemm.argtypes = [vp, vp, vp, vp, i64, i64, i64, vp, i32, vp, vp]
     L.nvfp4_amax.argtypes = [vp, i32, i64, i64, i64, vp, vp, sz, vp]
     L.nvfp4_quantize.argtypes = [vp, i32, i64, i64, i64, vp, vp, vp, vp, u32, vp, sz, vp]
     L.nvfp4_dequantize.argtypes = [vp, vp, vp, i64, i64, vp, i32, vp]
@@ -77,7 +79,7 @@ def _load() -> ctypes.CDLL:
     L.nvfp4_amax_sliced.argtypes = [vp, i32, i64, i64, i64, i32, vp, vp, vp, sz, vp]
     for f in ("mxfp8_quantize", "mxfp8_dequantize", "mxfp8_quantize_grouped",
               "mxfp8_quantize_columnwise", "mxfp4_quantize", "mxfp4_dequantize",
-              "mxfp4_quantize_grouped", "mx_fake_quantize", "nvfp4_amax",
+              "mxfp4_quantize_grouped", "mx_fake_quantize", "mxfp8_gemm", "nvfp4_amax",
               "nvfp4_quantize_sliced", "nvfp4_amax_sliced",
               "nvfp4_quantize", "nvfp4_dequantize"):
         getattr(L, f).restype = i32
@@ -303,6 +305,37 @@ def mx_fake_quantize(x: torch.Tensor, fmt: str = "mxfp4",
     _check("mx_fake_quantize", lib.mx_fake_quantize(formats[fmt], _ptr(x), dt, M, N, ld, _ptr(y),
                                                     _dtype_code(dtype), _stream(x)))
     return y
+
+
+# ------------------------------------------------------------------- GEMM
+
+def mxfp8_gemm(qa: torch.Tensor, sa_swizzled: torch.Tensor, qb: torch.Tensor,
+               sb_swizzled: torch.Tensor, dtype: torch.dtype = torch.bfloat16,
+               error_flag: torch.Tensor | None = None) -> torch.Tensor:
+    """D = A B^T from MXFP8 operands on the tensor cores: ``qa`` [M, K] and
+    ``qb`` [N, K] uint8 E4M3 codes (as :func:`mxfp8_quantize` returns them)
+    and their swizzled scales (the third output of
+    ``mxfp8_quantize(..., swizzled=True)``). Returns D [M, N] as ``dtype``.
+    ``error_flag`` (a zeroed int32 CUDA tensor) receives a non-zero code if
+    a wait inside the kernel gave up."""
+    _require_cuda(qa, sa_swizzled, qb, sb_swizzled)
+    for t in (qa, qb, sa_swizzled, sb_swizzled):
+        if t.dtype != torch.uint8 or not t.is_contiguous():
+            raise TypeError("codes and scales must be contiguous uint8 tensors")
+    if qa.dim() != 2 or qb.dim() != 2 or qa.shape[1] != qb.shape[1]:
+        raise ValueError("expected qa [M, K] and qb [N, K]")
+    M, K = qa.shape
+    N = qb.shape[0]
+    if sa_swizzled.numel() < swizzled_scale_bytes(M, K // 32) or \
+            sb_swizzled.numel() < swizzled_scale_bytes(N, K // 32):
+        raise ValueError("swizzled scales are smaller than the operands need")
+    if error_flag is not None and (error_flag.dtype != torch.int32 or not error_flag.is_cuda):
+        raise TypeError("error_flag must be an int32 CUDA tensor")
+    d = torch.empty((M, N), dtype=dtype, device=qa.device)
+    _check("mxfp8_gemm", lib.mxfp8_gemm(_ptr(qa), _ptr(sa_swizzled), _ptr(qb), _ptr(sb_swizzled),
+                                        M, N, K, _ptr(d), _dtype_code(dtype), _ptr(error_flag),
+                                        _stream(qa)))
+    return d
 
 
 # ------------------------------------------------------------------ NVFP4

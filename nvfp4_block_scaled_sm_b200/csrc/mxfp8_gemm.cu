@@ -1,0 +1,414 @@
+// mxfp8_gemm.cu -- a block-scaled MXFP8 x MXFP8 GEMM on the 5th-generation
+// tensor cores (tcgen05, kind::mxf8f6f4.block_scale), the consumer of the
+// quantizer's codes and 128x4-tile swizzled E8M0 scales, for sm_100a.
+//
+//   D[m, n] = sum_k decode(A[m, k]) 2^(SA[m, k/32] - 127)
+//                 * decode(B[n, k]) 2^(SB[n, k/32] - 127)
+//
+// A [M, K] and B [N, K] are E4M3 codes as mxfp8_quantize writes them (rows of
+// K contiguous bytes: both operands K-major, B in the [out, in] layout of a
+// linear layer's weight), SA / SB their scales in the swizzled layout
+// (mxfp8_quantize's scale_swz). The products of two E4M3 values and two
+// power-of-two scales are exact; the tensor core accumulates them in fp32.
+// Context: "V4 mxfp4 #1372" (description: block-scaled low-precision GEMMs
+// reading E8M0 scales on Blackwell) and "PR #1935 完整报告 -- Use
+// TransformerEngine for MXFP8 quantization" (the quantized weights feed the
+// GEMM); the scale-tile layout is the one the block-scaled MMA reads.
+//
+// Structure (one CTA per 128 x 128 output tile, 128 threads):
+//  - warp 0, one lane: producer. Per K block of 128: TMA loads of the A and
+//    B tiles (128 rows x 128 bytes, 128-byte swizzle) and bulk copies of the
+//    two 512-byte scale tiles into one of kStages shared-memory stages;
+//    completion is counted in bytes on the stage's "full" mbarrier.
+//  - warp 1, one lane: MMA issuer. Copies the stage's scale tiles into tensor
+//    memory (tcgen05.cp 32x128b.warpx4, the 32 x 16-byte scale tile
+//    broadcast to the four lane quarters), issues four MMAs of K = 32 (one
+//    scale column each, selected by the scale-factor id), then commits the
+//    stage's "empty" mbarrier; after the last block it commits "accum".
+//  - all four warps: epilogue. Each warp reads its 32 accumulator lanes
+//    (tcgen05.ld 32x32b) and writes its rows of D as bf16 or fp32.
+// Tensor memory: 128 columns of fp32 accumulator plus 8 scale columns per
+// stage (4 for A, 4 for B), 256 columns allocated.
+//
+// Every wait on an mbarrier gives up after about one second (by %globaltimer)
+// or 2^30 polls; the kernel then records an error code in *err (when err is
+// not NULL), skips the remaining work, frees its tensor memory and returns.
+#include <cuda.h>
+
+#include "common.cuh"
+
+namespace mxq {
+namespace {
+
+constexpr int kBM = 128, kBN = 128, kBK = 128;  // kBK elements = bytes of E4M3
+constexpr int kStages = 6;
+constexpr int kGemmThreads = 128;
+constexpr uint32_t kTileBytes = kBM * kBK;                         // 16 KiB (A and B alike)
+constexpr uint32_t kSfTile = 512;                                  // one 128 x 4 scale tile
+constexpr uint32_t kStageBytes = 2 * kTileBytes + 2 * kSfTile;     // 33 KiB, a multiple of 1 KiB
+constexpr uint32_t kTmemCols = 256;
+constexpr uint32_t kSfCol0 = kBN;                                  // first scale column
+constexpr uint32_t kBarBytes = 256;
+constexpr uint32_t kSmemBytes = kStages * kStageBytes + kBarBytes + 1024;  // + alignment slack
+constexpr uint64_t kWaitNs = 1000000000ull;                        // one second
+
+enum GemmError : int32_t { kErrNone = 0, kErrFullWait = 1, kErrEmptyWait = 2, kErrAccumWait = 3 };
+
+struct GemmArgs {
+  const uint8_t* sfa;   // swizzled scales of A
+  const uint8_t* sfb;   // swizzled scales of B
+  void* d;              // [M, N] row-major
+  int32_t* err;         // device error word or NULL
+  uint32_t M, N;
+  uint32_t nk;          // K blocks of 128
+  uint32_t kp4;         // 4-column scale tiles per 128-row block: ceil(K / 128)
+};
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ uint64_t globaltimer() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+
+// Waits until the phase of parity `parity` has completed; false on timeout.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint64_t deadline) {
+  for (uint32_t it = 0; it < (1u << 30); ++it) {
+    uint32_t done;
+    asm volatile(
+        "{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"
+        : "=r"(done)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    if (done) return true;
+    if ((it & 15u) == 15u && globaltimer() > deadline) return false;
+  }
+  return false;
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
+                                            int32_t x, int32_t y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];"
+      ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y)
+      : "memory");
+}
+
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+      ::"r"(dst), "l"(src), "r"(bytes), "r"(bar)
+      : "memory");
+}
+
+// Shared-memory matrix descriptor (tcgen05): start address, leading and
+// stride byte offsets in 16-byte units, descriptor version 1, layout type.
+__device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint32_t sbo,
+                                              uint32_t layout) {
+  return uint64_t((addr >> 4) & 0x3fffu) | (uint64_t(lbo & 0x3fffu) << 16) |
+         (uint64_t(sbo & 0x3fffu) << 32) | (1ull << 46) | (uint64_t(layout) << 61);
+}
+
+// K-major operand tile, rows of 128 bytes with the 128-byte swizzle: 8-row
+// groups 1024 bytes apart (layout type 2).
+__device__ __forceinline__ uint64_t operand_desc(uint32_t addr) {
+  return smem_desc(addr, 1, 1024 >> 4, 2);
+}
+
+// The 512-byte scale tile seen as 32 rows of 16 bytes, no swizzle.
+__device__ __forceinline__ uint64_t scale_desc(uint32_t addr) {
+  return smem_desc(addr, 1, 128 >> 4, 0);
+}
+
+// Instruction descriptor of kind::mxf8f6f4.block_scale: E4M3 x E4M3, both
+// K-major, fp32 accumulator, M = 128, N = 128, E8M0 scales; the scale-factor
+// ids pick byte `k` (the scale column of the k-th MMA of a K block) of the
+// 32-bit scale columns of A and B.
+__device__ __forceinline__ uint32_t instr_desc(uint32_t k) {
+  return (k << 4) | (uint32_t(kBN >> 3) << 17) | (1u << 23) | (uint32_t(kBM >> 4) << 24) | (k << 29);
+}
+
+__device__ __forceinline__ void mma_mxf8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                         uint32_t idesc, uint32_t sfa_tmem, uint32_t sfb_tmem,
+                                         uint32_t accumulate) {
+  asm volatile(
+      "{ .reg .pred p; setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p; }"
+      ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_copy_scales(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
+__device__ __forceinline__ void mma_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+               : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// 32 consecutive fp32 accumulator columns of this thread's lane.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
+        "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]),
+        "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]),
+        "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void record_error(int32_t* err, int32_t code) {
+  if (err) atomicCAS(err, 0, code);
+}
+
+template <typename OutT>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+mxfp8_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_b,
+                  const __grid_constant__ GemmArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  // operand tiles need 1024-byte alignment (128-byte swizzle atoms)
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* smem = smem_raw + (base - raw);
+  const uint32_t bars = base + kStages * kStageBytes;  // full[s], empty[s], accum, tmem slot
+  auto full_bar = [&](int s) { return bars + 8u * s; };
+  auto empty_bar = [&](int s) { return bars + 8u * (kStages + s); };
+  const uint32_t accum_bar = bars + 8u * (2 * kStages);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kStages * kStageBytes + 8 * (2 * kStages + 1));
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t n_blk = blockIdx.x, m_blk = blockIdx.y;
+  const uint64_t deadline = globaltimer() + kWaitNs;
+
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                 ::"r"(smem_u32(tmem_slot)), "r"(kTmemCols) : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  if (threadIdx.x == 32) {
+    for (int s = 0; s < kStages; s++) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    mbar_init(accum_bar, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0 && lane == 0) {
+    // ---------------------------------------------------------- producer
+    const uint8_t* sfa = a.sfa + (uint64_t(m_blk) * a.kp4) * kSfTile;
+    const uint8_t* sfb = a.sfb + (uint64_t(n_blk) * a.kp4) * kSfTile;
+    for (uint32_t kb = 0; kb < a.nk; kb++) {
+      const int s = kb % kStages;
+      const uint32_t phase = (kb / kStages) & 1u;
+      if (!mbar_wait(empty_bar(s), phase ^ 1u, deadline)) {
+        record_error(a.err, kErrEmptyWait);
+        break;
+      }
+      const uint32_t st = base + s * kStageBytes;
+      mbar_expect_tx(full_bar(s), kStageBytes);
+      tma_load_2d(st, &tma_a, full_bar(s), int32_t(kb * kBK), int32_t(m_blk * kBM));
+      tma_load_2d(st + kTileBytes, &tma_b, full_bar(s), int32_t(kb * kBK), int32_t(n_blk * kBN));
+      bulk_load(st + 2 * kTileBytes, sfa + uint64_t(kb) * kSfTile, kSfTile, full_bar(s));
+      bulk_load(st + 2 * kTileBytes + kSfTile, sfb + uint64_t(kb) * kSfTile, kSfTile, full_bar(s));
+    }
+  } else if (warp == 1 && lane == 0) {
+    // ------------------------------------------------------- MMA issuer
+    bool ok = true;
+    for (uint32_t kb = 0; kb < a.nk; kb++) {
+      const int s = kb % kStages;
+      const uint32_t phase = (kb / kStages) & 1u;
+      if (!mbar_wait(full_bar(s), phase, deadline)) {
+        record_error(a.err, kErrFullWait);
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t st = base + s * kStageBytes;
+      const uint32_t sfa_t = tmem + kSfCol0 + 8u * s;
+      const uint32_t sfb_t = sfa_t + 4u;
+      tmem_copy_scales(sfa_t, scale_desc(st + 2 * kTileBytes));
+      tmem_copy_scales(sfb_t, scale_desc(st + 2 * kTileBytes + kSfTile));
+#pragma unroll
+      for (uint32_t k = 0; k < 4; k++) {
+        mma_mxf8(tmem, operand_desc(st + 32u * k), operand_desc(st + kTileBytes + 32u * k),
+                 instr_desc(k), sfa_t | (k << 30), sfb_t | (k << 30), (kb | k) != 0u);
+      }
+      mma_commit(empty_bar(s));
+    }
+    if (ok) mma_commit(accum_bar);
+  }
+  __syncwarp();
+
+  // ------------------------------------------------------------ epilogue
+  // the phase completes once for everyone: a lane that saw it lets the warp go
+  const bool have = __any_sync(0xffffffffu, a.nk > 0 && mbar_wait(accum_bar, 0, deadline));
+  if (a.nk > 0 && !have && lane == 0) record_error(a.err, kErrAccumWait);
+  tc_fence_after();
+  if (have) {
+    const uint32_t row = m_blk * kBM + warp * 32 + lane;
+    const uint32_t taddr = tmem + (uint32_t(warp * 32) << 16);
+    OutT* drow = static_cast<OutT*>(a.d) + uint64_t(row) * a.N + uint64_t(n_blk) * kBN;
+    const uint32_t ncols = min(uint32_t(kBN), a.N - n_blk * kBN);
+#pragma unroll 1
+    for (uint32_t c0 = 0; c0 < uint32_t(kBN); c0 += 32) {
+      uint32_t r[32];
+      tmem_ld32(taddr + c0, r);  // every lane of the warp takes part
+      if (row >= a.M || c0 >= ncols) continue;
+      if constexpr (sizeof(OutT) == 2) {
+        uint32_t w[16];
+#pragma unroll
+        for (int i = 0; i < 16; i++)
+          w[i] = cvt_bf16x2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
+        if (c0 + 32 <= ncols) {
+#pragma unroll
+          for (int i = 0; i < 4; i++)
+            st_v4(drow + c0 + 8 * i, make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]));
+        } else {
+#pragma unroll
+          for (uint32_t i = 0; i < 16; i++)
+            if (c0 + 2 * i < ncols) st_u32(drow + c0 + 2 * i, w[i]);
+        }
+      } else {
+        if (c0 + 32 <= ncols) {
+#pragma unroll
+          for (int i = 0; i < 8; i++)
+            st_v4(drow + c0 + 4 * i, make_uint4(r[4 * i], r[4 * i + 1], r[4 * i + 2], r[4 * i + 3]));
+        } else {
+#pragma unroll
+          for (uint32_t i = 0; i < 32; i++)
+            if (c0 + i < ncols) st_u32(drow + c0 + i, r[i]);
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols)
+                 : "memory");
+  }
+}
+
+// ------------------------------------------------------------------ host
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// [rows, K] bytes, row stride K, boxes of 128 rows x 128 bytes, 128-byte
+// swizzle; out-of-range rows and columns read as zero.
+bool make_operand_map(CUtensorMap* map, const uint8_t* p, uint64_t rows, uint64_t K) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {K, rows};
+  const cuuint64_t strides[1] = {K};
+  const cuuint32_t box[2] = {uint32_t(kBK), uint32_t(kBM)};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(p), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <typename OutT>
+mxq_status launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const GemmArgs& args,
+                       cudaStream_t s) {
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [] {
+    attr_err = cudaFuncSetAttribute(mxfp8_gemm_kernel<OutT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    int(kSmemBytes));
+  });
+  if (attr_err != cudaSuccess) {
+    record_cuda_error(attr_err);
+    return MXQ_ERR_CUDA;
+  }
+  const dim3 grid((args.N + kBN - 1) / kBN, (args.M + kBM - 1) / kBM);
+  mxfp8_gemm_kernel<OutT><<<grid, kGemmThreads, kSmemBytes, s>>>(ta, tb, args);
+  return check_launch();
+}
+
+}  // namespace
+}  // namespace mxq
+
+extern "C" mxq_status mxfp8_gemm(const uint8_t* qa, const uint8_t* sa_swz, const uint8_t* qb,
+                                 const uint8_t* sb_swz, int64_t M, int64_t N, int64_t K, void* d,
+                                 int out_dt, int32_t* error_flag, mxq_stream_t stream) {
+  using namespace mxq;
+  if (!valid_dtype(out_dt)) return MXQ_ERR_DTYPE;
+  if (M < 0 || N < 0 || K < 0 || K % 32 != 0 || N % 16 != 0) return MXQ_ERR_SHAPE;
+  if (M > 0x7fffff80ll || N > 0x7fffff80ll || K > 0x7fffff80ll) return MXQ_ERR_SHAPE;
+  if (M == 0 || N == 0) return MXQ_OK;
+  if (!d) return MXQ_ERR_NULL;
+  if (!aligned16(d)) return MXQ_ERR_ALIGN;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (K == 0) {
+    const cudaError_t e = cudaMemsetAsync(d, 0, size_t(M) * size_t(N) * elem_size(out_dt), s);
+    if (e != cudaSuccess) {
+      record_cuda_error(e);
+      return MXQ_ERR_CUDA;
+    }
+    return MXQ_OK;
+  }
+  if (!qa || !qb || !sa_swz || !sb_swz) return MXQ_ERR_NULL;
+  if (!aligned16(qa) || !aligned16(qb) || !aligned16(sa_swz) || !aligned16(sb_swz))
+    return MXQ_ERR_ALIGN;
+  CUtensorMap ta, tb;
+  if (!make_operand_map(&ta, qa, uint64_t(M), uint64_t(K)) ||
+      !make_operand_map(&tb, qb, uint64_t(N), uint64_t(K)))
+    return MXQ_ERR_CUDA;
+  GemmArgs args{};
+  args.sfa = sa_swz;
+  args.sfb = sb_swz;
+  args.d = d;
+  args.err = error_flag;
+  args.M = uint32_t(M);
+  args.N = uint32_t(N);
+  args.nk = uint32_t((K + kBK - 1) / kBK);
+  args.kp4 = args.nk;
+  if (out_dt == MXQ_BF16) return launch_gemm<uint16_t>(ta, tb, args, s);
+  return launch_gemm<float>(ta, tb, args, s);
+}

@@ -220,6 +220,19 @@ def mx_all_packed_scale_pairs():
     return q, s
 
 
+def gemm_pow2_operand(seed: int, rows: int, K: int) -> np.ndarray:
+    """bf16 [rows, K] for exact GEMM checks: each element is 0 or +-2^g with
+    g drawn per 32-element group from {-2, ..., 2} (about a quarter zeros), so
+    groups carry different power-of-two magnitudes, every element is exactly
+    representable after quantization, and all products and partial sums of
+    two such operands lie on the grid 2^-4 within 2^(log2 K + 4)."""
+    rng = np.random.default_rng(seed)
+    g = rng.integers(-2, 3, (rows, K // 32))
+    mag = np.repeat(np.ldexp(1.0, g), 32, axis=1)
+    sign = rng.choice(np.array([-1.0, 0.0, 1.0, 1.0]), (rows, K))
+    return to_bf16_bits((sign * mag).astype(np.float32))
+
+
 def mxfp8_all_code_scale_pairs():
     """(qweight [256, 8192], scale [256, 256]): row r carries scale byte r on
     every group and the 256 E4M3 codes repeated, so every (code, byte) pair
