@@ -15,20 +15,22 @@
 // TransformerEngine for MXFP8 quantization" (the quantized weights feed the
 // GEMM); the scale-tile layout is the one the block-scaled MMA reads.
 //
-// Structure (one CTA per 128 x 128 output tile, 128 threads):
-//  - warp 0, one lane: producer. Per K block of 128: TMA loads of the A and
-//    B tiles (128 rows x 128 bytes, 128-byte swizzle) and bulk copies of the
-//    two 512-byte scale tiles into one of kStages shared-memory stages;
-//    completion is counted in bytes on the stage's "full" mbarrier.
+// Structure (one CTA per 128 x BN output tile, BN = 128 or 256, 128 threads):
+//  - warp 0, one lane: producer. Per K block of 128: TMA loads of the A tile
+//    (128 rows x 128 bytes) and the B tile (BN rows x 128 bytes), both with
+//    the 128-byte swizzle, and bulk copies of the 512-byte scale tiles (one
+//    for A, BN / 128 for B) into one of the shared-memory stages; completion
+//    is counted in bytes on the stage's "full" mbarrier.
 //  - warp 1, one lane: MMA issuer. Copies the stage's scale tiles into tensor
 //    memory (tcgen05.cp 32x128b.warpx4, the 32 x 16-byte scale tile
 //    broadcast to the four lane quarters), issues four MMAs of K = 32 (one
-//    scale column each, selected by the scale-factor id), then commits the
+//    scale column each, selected by the scale-factor id; M = 128, N = BN),
+//    then commits the
 //    stage's "empty" mbarrier; after the last block it commits "accum".
 //  - all four warps: epilogue. Each warp reads its 32 accumulator lanes
 //    (tcgen05.ld 32x32b) and writes its rows of D as bf16 or fp32.
-// Tensor memory: 128 columns of fp32 accumulator plus 8 scale columns per
-// stage (4 for A, 4 for B), 256 columns allocated.
+// Tensor memory: BN columns of fp32 accumulator plus 4 scale columns per
+// 128-row scale tile and stage (4 for A, 4 or 8 for B).
 //
 // Every wait on an mbarrier gives up after about one second (by %globaltimer)
 // or 2^30 polls; the kernel then records an error code in *err (when err is
@@ -40,17 +42,26 @@
 namespace mxq {
 namespace {
 
-constexpr int kBM = 128, kBN = 128, kBK = 128;  // kBK elements = bytes of E4M3
-constexpr int kStages = 6;
+constexpr int kBM = 128, kBK = 128;  // kBK elements = bytes of E4M3
 constexpr int kGemmThreads = 128;
-constexpr uint32_t kTileBytes = kBM * kBK;                         // 16 KiB (A and B alike)
-constexpr uint32_t kSfTile = 512;                                  // one 128 x 4 scale tile
-constexpr uint32_t kStageBytes = 2 * kTileBytes + 2 * kSfTile;     // 33 KiB, a multiple of 1 KiB
-constexpr uint32_t kTmemCols = 256;
-constexpr uint32_t kSfCol0 = kBN;                                  // first scale column
+constexpr uint32_t kSfTile = 512;    // one 128 x 4 scale tile
 constexpr uint32_t kBarBytes = 256;
-constexpr uint32_t kSmemBytes = kStages * kStageBytes + kBarBytes + 1024;  // + alignment slack
-constexpr uint64_t kWaitNs = 1000000000ull;                        // one second
+constexpr uint64_t kWaitNs = 1000000000ull;  // one second
+
+template <int BN>
+struct GemmCfg {
+  static constexpr int kStages = BN == 128 ? 6 : 4;
+  static constexpr uint32_t kTileA = kBM * kBK;                   // 16 KiB
+  static constexpr uint32_t kTileB = BN * kBK;                    // 16 or 32 KiB
+  static constexpr uint32_t kSfbTiles = BN / 128;
+  static constexpr uint32_t kStageBytes =                         // a multiple of 1 KiB
+      (kTileA + kTileB + kSfTile * (1 + kSfbTiles) + 1023u) & ~1023u;
+  static constexpr uint32_t kSfColsPerStage = 4 * (1 + kSfbTiles);
+  static constexpr uint32_t kTmemCols = BN + kStages * kSfColsPerStage <= 256 ? 256 : 512;
+  static constexpr uint32_t kSmemBytes = kStages * kStageBytes + kBarBytes + 1024;  // + alignment slack
+  static_assert(BN + kStages * kSfColsPerStage <= 512, "tensor memory");
+  static_assert(kSmemBytes <= 232448, "shared memory");
+};
 
 enum GemmError : int32_t { kErrNone = 0, kErrFullWait = 1, kErrEmptyWait = 2, kErrAccumWait = 3 };
 
@@ -62,6 +73,7 @@ struct GemmArgs {
   uint32_t M, N;
   uint32_t nk;          // K blocks of 128
   uint32_t kp4;         // 4-column scale tiles per 128-row block: ceil(K / 128)
+  uint32_t nb128;       // 128-row blocks of B's scales: ceil(N / 128)
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -133,11 +145,12 @@ __device__ __forceinline__ uint64_t scale_desc(uint32_t addr) {
 }
 
 // Instruction descriptor of kind::mxf8f6f4.block_scale: E4M3 x E4M3, both
-// K-major, fp32 accumulator, M = 128, N = 128, E8M0 scales; the scale-factor
+// K-major, fp32 accumulator, M = 128, N = BN, E8M0 scales; the scale-factor
 // ids pick byte `k` (the scale column of the k-th MMA of a K block) of the
 // 32-bit scale columns of A and B.
+template <int BN>
 __device__ __forceinline__ uint32_t instr_desc(uint32_t k) {
-  return (k << 4) | (uint32_t(kBN >> 3) << 17) | (1u << 23) | (uint32_t(kBM >> 4) << 24) | (k << 29);
+  return (k << 4) | (uint32_t(BN >> 3) << 17) | (1u << 23) | (uint32_t(kBM >> 4) << 24) | (k << 29);
 }
 
 __device__ __forceinline__ void mma_mxf8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
@@ -184,10 +197,13 @@ __device__ __forceinline__ void record_error(int32_t* err, int32_t code) {
   if (err) atomicCAS(err, 0, code);
 }
 
-template <typename OutT>
+template <typename OutT, int BN>
 __global__ void __launch_bounds__(kGemmThreads, 1)
 mxfp8_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_b,
                   const __grid_constant__ GemmArgs a) {
+  using C = GemmCfg<BN>;
+  constexpr int kStages = C::kStages;
+  constexpr uint32_t kStageBytes = C::kStageBytes;
   extern __shared__ uint8_t smem_raw[];
   // operand tiles need 1024-byte alignment (128-byte swizzle atoms)
   const uint32_t raw = smem_u32(smem_raw);
@@ -205,7 +221,7 @@ mxfp8_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_consta
 
   if (warp == 0) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
-                 ::"r"(smem_u32(tmem_slot)), "r"(kTmemCols) : "memory");
+                 ::"r"(smem_u32(tmem_slot)), "r"(C::kTmemCols) : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
   if (threadIdx.x == 32) {
@@ -224,7 +240,11 @@ mxfp8_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_consta
   if (warp == 0 && lane == 0) {
     // ---------------------------------------------------------- producer
     const uint8_t* sfa = a.sfa + (uint64_t(m_blk) * a.kp4) * kSfTile;
-    const uint8_t* sfb = a.sfb + (uint64_t(n_blk) * a.kp4) * kSfTile;
+    // B's 128-row scale blocks of this tile that exist (the last tile of a
+    // ragged N may have fewer than BN / 128; its missing rows are never stored)
+    const uint32_t b0 = n_blk * C::kSfbTiles;
+    const uint32_t nsfb = min(C::kSfbTiles, a.nb128 - b0);
+    const uint32_t tx = C::kTileA + C::kTileB + kSfTile * (1 + nsfb);
     for (uint32_t kb = 0; kb < a.nk; kb++) {
       const int s = kb % kStages;
       const uint32_t phase = (kb / kStages) & 1u;
@@ -233,11 +253,14 @@ mxfp8_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_consta
         break;
       }
       const uint32_t st = base + s * kStageBytes;
-      mbar_expect_tx(full_bar(s), kStageBytes);
+      mbar_expect_tx(full_bar(s), tx);
       tma_load_2d(st, &tma_a, full_bar(s), int32_t(kb * kBK), int32_t(m_blk * kBM));
-      tma_load_2d(st + kTileBytes, &tma_b, full_bar(s), int32_t(kb * kBK), int32_t(n_blk * kBN));
-      bulk_load(st + 2 * kTileBytes, sfa + uint64_t(kb) * kSfTile, kSfTile, full_bar(s));
-      bulk_load(st + 2 * kTileBytes + kSfTile, sfb + uint64_t(kb) * kSfTile, kSfTile, full_bar(s));
+      tma_load_2d(st + C::kTileA, &tma_b, full_bar(s), int32_t(kb * kBK), int32_t(n_blk * BN));
+      const uint32_t sf = st + C::kTileA + C::kTileB;
+      bulk_load(sf, sfa + uint64_t(kb) * kSfTile, kSfTile, full_bar(s));
+      for (uint32_t j = 0; j < nsfb; j++)
+        bulk_load(sf + kSfTile * (1 + j), a.sfb + (uint64_t(b0 + j) * a.kp4 + kb) * kSfTile, kSfTile,
+                  full_bar(s));
     }
   } else if (warp == 1 && lane == 0) {
     // ------------------------------------------------------- MMA issuer
@@ -252,14 +275,17 @@ mxfp8_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_consta
       }
       tc_fence_after();
       const uint32_t st = base + s * kStageBytes;
-      const uint32_t sfa_t = tmem + kSfCol0 + 8u * s;
+      const uint32_t sfa_t = tmem + BN + C::kSfColsPerStage * s;
       const uint32_t sfb_t = sfa_t + 4u;
-      tmem_copy_scales(sfa_t, scale_desc(st + 2 * kTileBytes));
-      tmem_copy_scales(sfb_t, scale_desc(st + 2 * kTileBytes + kSfTile));
+      const uint32_t sf = st + C::kTileA + C::kTileB;
+      tmem_copy_scales(sfa_t, scale_desc(sf));
+#pragma unroll
+      for (uint32_t j = 0; j < C::kSfbTiles; j++)
+        tmem_copy_scales(sfb_t + 4u * j, scale_desc(sf + kSfTile * (1 + j)));
 #pragma unroll
       for (uint32_t k = 0; k < 4; k++) {
-        mma_mxf8(tmem, operand_desc(st + 32u * k), operand_desc(st + kTileBytes + 32u * k),
-                 instr_desc(k), sfa_t | (k << 30), sfb_t | (k << 30), (kb | k) != 0u);
+        mma_mxf8(tmem, operand_desc(st + 32u * k), operand_desc(st + C::kTileA + 32u * k),
+                 instr_desc<BN>(k), sfa_t | (k << 30), sfb_t | (k << 30), (kb | k) != 0u);
       }
       mma_commit(empty_bar(s));
     }
@@ -275,10 +301,10 @@ mxfp8_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_consta
   if (have) {
     const uint32_t row = m_blk * kBM + warp * 32 + lane;
     const uint32_t taddr = tmem + (uint32_t(warp * 32) << 16);
-    OutT* drow = static_cast<OutT*>(a.d) + uint64_t(row) * a.N + uint64_t(n_blk) * kBN;
-    const uint32_t ncols = min(uint32_t(kBN), a.N - n_blk * kBN);
+    OutT* drow = static_cast<OutT*>(a.d) + uint64_t(row) * a.N + uint64_t(n_blk) * BN;
+    const uint32_t ncols = min(uint32_t(BN), a.N - n_blk * BN);
 #pragma unroll 1
-    for (uint32_t c0 = 0; c0 < uint32_t(kBN); c0 += 32) {
+    for (uint32_t c0 = 0; c0 < uint32_t(BN); c0 += 32) {
       uint32_t r[32];
       tmem_ld32(taddr + c0, r);  // every lane of the warp takes part
       if (row >= a.M || c0 >= ncols) continue;
@@ -314,7 +340,7 @@ mxfp8_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_consta
   __syncthreads();
   if (warp == 0) {
     tc_fence_after();
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols)
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(C::kTmemCols)
                  : "memory");
   }
 }
@@ -339,35 +365,37 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// [rows, K] bytes, row stride K, boxes of 128 rows x 128 bytes, 128-byte
-// swizzle; out-of-range rows and columns read as zero.
-bool make_operand_map(CUtensorMap* map, const uint8_t* p, uint64_t rows, uint64_t K) {
+// [rows, K] bytes, row stride K, boxes of box_rows rows x 128 bytes,
+// 128-byte swizzle; out-of-range rows and columns read as zero.
+bool make_operand_map(CUtensorMap* map, const uint8_t* p, uint64_t rows, uint64_t K,
+                      uint32_t box_rows) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
   const cuuint64_t dims[2] = {K, rows};
   const cuuint64_t strides[1] = {K};
-  const cuuint32_t box[2] = {uint32_t(kBK), uint32_t(kBM)};
+  const cuuint32_t box[2] = {uint32_t(kBK), box_rows};
   const cuuint32_t estr[2] = {1, 1};
   return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(p), dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <typename OutT>
+template <typename OutT, int BN>
 mxq_status launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const GemmArgs& args,
                        cudaStream_t s) {
+  constexpr uint32_t kSmemBytes = GemmCfg<BN>::kSmemBytes;
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(once, [] {
-    attr_err = cudaFuncSetAttribute(mxfp8_gemm_kernel<OutT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    int(kSmemBytes));
+    attr_err = cudaFuncSetAttribute(mxfp8_gemm_kernel<OutT, BN>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmemBytes));
   });
   if (attr_err != cudaSuccess) {
     record_cuda_error(attr_err);
     return MXQ_ERR_CUDA;
   }
-  const dim3 grid((args.N + kBN - 1) / kBN, (args.M + kBM - 1) / kBM);
-  mxfp8_gemm_kernel<OutT><<<grid, kGemmThreads, kSmemBytes, s>>>(ta, tb, args);
+  const dim3 grid((args.N + BN - 1) / BN, (args.M + kBM - 1) / kBM);
+  mxfp8_gemm_kernel<OutT, BN><<<grid, kGemmThreads, kSmemBytes, s>>>(ta, tb, args);
   return check_launch();
 }
 
@@ -396,9 +424,12 @@ extern "C" mxq_status mxfp8_gemm(const uint8_t* qa, const uint8_t* sa_swz, const
   if (!qa || !qb || !sa_swz || !sb_swz) return MXQ_ERR_NULL;
   if (!aligned16(qa) || !aligned16(qb) || !aligned16(sa_swz) || !aligned16(sb_swz))
     return MXQ_ERR_ALIGN;
+  // 128 x 256 tiles halve the operand traffic per MMA; narrow outputs keep
+  // 128-wide tiles
+  const bool wide = N > 128;
   CUtensorMap ta, tb;
-  if (!make_operand_map(&ta, qa, uint64_t(M), uint64_t(K)) ||
-      !make_operand_map(&tb, qb, uint64_t(N), uint64_t(K)))
+  if (!make_operand_map(&ta, qa, uint64_t(M), uint64_t(K), kBM) ||
+      !make_operand_map(&tb, qb, uint64_t(N), uint64_t(K), wide ? 256u : 128u))
     return MXQ_ERR_CUDA;
   GemmArgs args{};
   args.sfa = sa_swz;
@@ -409,6 +440,8 @@ extern "C" mxq_status mxfp8_gemm(const uint8_t* qa, const uint8_t* sa_swz, const
   args.N = uint32_t(N);
   args.nk = uint32_t((K + kBK - 1) / kBK);
   args.kp4 = args.nk;
-  if (out_dt == MXQ_BF16) return launch_gemm<uint16_t>(ta, tb, args, s);
-  return launch_gemm<float>(ta, tb, args, s);
+  args.nb128 = uint32_t((N + 127) / 128);
+  if (out_dt == MXQ_BF16)
+    return wide ? launch_gemm<uint16_t, 256>(ta, tb, args, s) : launch_gemm<uint16_t, 128>(ta, tb, args, s);
+  return wide ? launch_gemm<float, 256>(ta, tb, args, s) : launch_gemm<float, 128>(ta, tb, args, s);
 }
