@@ -200,6 +200,22 @@ __device__ __forceinline__ uint32_t cvt_e2m1x2(float lo, float hi) {
   return r;
 }
 
+// Four bytes of E2M1 codes for eight values, two per byte, the first value of
+// each pair in the low nibble and pair p in byte p (one register pack, no
+// byte shuffles).
+__device__ __forceinline__ uint32_t cvt_e2m1x8(float2 p0, float2 p1, float2 p2, float2 p3) {
+  uint32_t r;
+  asm("{ .reg .b8 b0, b1, b2, b3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+      "mov.b32 %0, {b0, b1, b2, b3}; }"
+      : "=r"(r)
+      : "f"(p0.x), "f"(p0.y), "f"(p1.x), "f"(p1.y), "f"(p2.x), "f"(p2.y), "f"(p3.x), "f"(p3.y));
+  return r;
+}
+
 // One byte holding two E2M1 codes (low nibble first) -> f16x2 (exact).
 __device__ __forceinline__ uint32_t cvt_f16x2_from_e2m1x2(uint32_t byte) {
   uint32_t r;

@@ -203,9 +203,8 @@ __device__ __forceinline__ uint32_t e2m1_resolve(float x, float eff, uint32_t c)
 
 // Byte of two E2M1 codes for (x0, x1) when the bracket codes cl (from the
 // lower products) and ch (upper) disagree in at least one nibble: each
-// disagreeing nibble is decided exactly. Out of line so that the common path
-// only pays a predicted-not-taken branch per pair.
-__device__ __noinline__ uint32_t fix_pair(float x0, float x1, float eff, uint32_t cl, uint32_t ch) {
+// disagreeing nibble is decided exactly.
+__device__ __forceinline__ uint32_t fix_pair(float x0, float x1, float eff, uint32_t cl, uint32_t ch) {
   const bool fma_ok = (__float_as_uint(eff) & 0x7f800000u) >= (29u << 23);  // eff >= 2^-98
   uint32_t code = cl & 0xffu;
 #pragma unroll
@@ -219,6 +218,26 @@ __device__ __noinline__ uint32_t fix_pair(float x0, float x1, float eff, uint32_
     }
   }
   return code;
+}
+
+// The block's codes when the bracket words lo (lower products) and hi
+// (upper) differ: every pair whose bytes differ is decided exactly. Out of
+// line, so that the common path pays one predicted-not-taken branch per block
+// and the exact arithmetic is never evaluated speculatively.
+template <typename InT>
+__device__ __noinline__ uint2 fix_block(In16<InT> v, float eff, uint2 lo, uint2 hi) {
+  uint32_t w[2] = {lo.x, lo.y};
+  const uint32_t hw[2] = {hi.x, hi.y};
+#pragma unroll
+  for (int k = 0; k < 8; k++) {
+    const int sh = 8 * (k & 3);
+    const uint32_t cl = (w[k >> 2] >> sh) & 0xffu, ch = (hw[k >> 2] >> sh) & 0xffu;
+    if (cl != ch) {
+      const uint32_t b = fix_pair(v.lo(k), v.hi(k), eff, cl, ch);
+      w[k >> 2] = (w[k >> 2] & ~(0xffu << sh)) | (b << sh);
+    }
+  }
+  return make_uint2(w[0], w[1]);
 }
 
 // Packed E2M1 codes (8 bytes, element 2k in the low nibble of byte k) of the
@@ -239,18 +258,18 @@ __device__ __forceinline__ uint2 e2m1_codes(const In16<InT>& v, float eff) {
     const float r = rcp_approx(eff);
     const float rl = __fmul_rn(r, 0.99999904632568359375f);  // 1 - 2^-20
     const float rh = __fmul_rn(r, 1.00000095367431640625f);  // 1 + 2^-20
-    uint32_t b[8];
+    float2 l[8], h[8];
 #pragma unroll
     for (int k = 0; k < 8; k++) {
-      const float2 l = mul2(v.lo(k), v.hi(k), rl);
-      const float2 h = mul2(v.lo(k), v.hi(k), rh);
-      const uint32_t cl = cvt_e2m1x2(l.x, l.y), ch = cvt_e2m1x2(h.x, h.y);
-      // a code boundary inside the bracket (exact quotients such as 3.5 are
-      // common with bf16 inputs): decide those elements exactly
-      b[k] = __builtin_expect(cl != ch, 0) ? fix_pair(v.lo(k), v.hi(k), eff, cl, ch) : cl;
+      l[k] = mul2(v.lo(k), v.hi(k), rl);
+      h[k] = mul2(v.lo(k), v.hi(k), rh);
     }
-    const uint2 out = make_uint2(pack4(b[0], b[1], b[2], b[3]), pack4(b[4], b[5], b[6], b[7]));
-    return out;
+    const uint2 L = make_uint2(cvt_e2m1x8(l[0], l[1], l[2], l[3]), cvt_e2m1x8(l[4], l[5], l[6], l[7]));
+    const uint2 H = make_uint2(cvt_e2m1x8(h[0], h[1], h[2], h[3]), cvt_e2m1x8(h[4], h[5], h[6], h[7]));
+    // a code boundary inside some bracket (exact quotients such as 3.5 are
+    // common with bf16 inputs): decide those elements exactly
+    if (__builtin_expect(((L.x ^ H.x) | (L.y ^ H.y)) != 0u, 0)) return fix_block(v, eff, L, H);
+    return L;
   }
   float x[16];
 #pragma unroll
