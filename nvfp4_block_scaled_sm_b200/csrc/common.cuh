@@ -399,12 +399,12 @@ __device__ __forceinline__ void pdl_enter() {
 // Launches `kernel` with programmatic stream serialization, so its launch and
 // CTA scheduling overlap the tail of the previous grid in the stream.
 template <typename... KArgs, typename... Args>
-inline cudaError_t launch_pdl(void (*kernel)(KArgs...), uint32_t grid, cudaStream_t stream,
-                              Args&&... args) {
+inline cudaError_t launch_pdl_ex(void (*kernel)(KArgs...), uint32_t grid, uint32_t block,
+                                 size_t smem, cudaStream_t stream, Args&&... args) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = 0;
+  cfg.blockDim = dim3(block);
+  cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -412,6 +412,20 @@ inline cudaError_t launch_pdl(void (*kernel)(KArgs...), uint32_t grid, cudaStrea
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), uint32_t grid, cudaStream_t stream,
+                              Args&&... args) {
+  return launch_pdl_ex(kernel, grid, kThreads, 0, stream, std::forward<Args>(args)...);
+}
+
+// Multiprocessors of the current device (148 on B200 if the query fails).
+inline int sm_count() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 148;
 }
 
 // ----------------------------------------------------------- block reduce

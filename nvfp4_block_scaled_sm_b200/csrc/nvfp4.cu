@@ -544,12 +544,6 @@ nvfp4_dequant_kernel(const uint8_t* __restrict__ packed, const uint8_t* __restri
 
 // ------------------------------------------------------------------ host
 
-int sm_count() {
-  int dev = 0, n = 148;
-  if (cudaGetDevice(&dev) == cudaSuccess)
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-  return n > 0 ? n : 148;
-}
 
 template <typename InT, bool V8, bool STRIDED>
 cudaError_t launch_amax_kernel(uint32_t grid, const void* x, uint64_t nchunks, uint32_t cpr,
