@@ -21,20 +21,21 @@
 //    <= 1 ulp), the products lo = fl(x * fl(r (1 - 2^-20))) and
 //    hi = fl(x * fl(r (1 + 2^-20))) bracket f strictly (a few 2^-24 relative
 //    roundings against the 2^-20 margin; f lies within 2^-24 of x / eff). When
-//    E2M1(lo) == E2M1(hi) that is E2M1(f); a tie of f on a midpoint puts lo
-//    and hi on opposite sides of it. Elements whose brackets disagree (bf16
-//    inputs make exact quotients such as 3.5 common) are decided exactly from
-//    the fused-multiply-add residual |x| - eff * M against the midpoint M
-//    (see e2m1_resolve), or by IEEE division for divisors below 2^-98.
+//    E2M1(lo) == E2M1(hi) for all 16 elements, that is E2M1(f); a tie of f on
+//    a midpoint puts lo and hi on opposite sides of it.
 //  - E4M3 (per block): the product amax * rcp.approx(t) lies within a few
 //    ulps of f; every E4M3 midpoint has at most four significant bits, so the
 //    product rounds like f unless it is within 32 ulps of a value whose
-//    mantissa is zero below bit 19, in which case the block divides exactly.
-// Divisors outside [2^-125, 2^125) (whose approximate reciprocal would not be
-// normal) take the exact path. Products below the normal range are far below
-// the first midpoint and overflowing products far above the last, so neither
-// can change a code. The exact paths are out-of-line functions so that the
-// compiler cannot evaluate them speculatively.
+//    mantissa is zero below bit 19.
+// A block where either test fails (bf16 inputs make exact quotients such as
+// 3.5 common), or whose divisors lie outside [2^-125, 2^125) (where the
+// approximate reciprocal would not be normal), is put on a shared list and
+// recomputed by the definition, with IEEE divisions, after the tile's main
+// loop; the out-of-line exact path then costs the main loop one predicated
+// shared atomic. Blocks with eff == 0 (the zero-block guard) get sign-kept
+// zero codes inline. Products below the normal range are far below the first
+// midpoint and overflowing products far above the last, so neither can change
+// a code.
 //
 // Passes: the tensor amax must be known before any block can be quantized,
 // so a first kernel reduces |x| into per-CTA partial maxima (workspace), and
@@ -161,123 +162,69 @@ struct QuantArgs {
   uint32_t ntiles;
 };
 
-// Four bytes (low byte of each argument) into one word, first argument lowest.
-__device__ __forceinline__ uint32_t pack4(uint32_t b0, uint32_t b1, uint32_t b2, uint32_t b3) {
-  return __byte_perm(__byte_perm(b0, b1, 0x0040), __byte_perm(b2, b3, 0x0040), 0x5410);
-}
-
-// IEEE quotient, kept out of line so that the compiler cannot evaluate it
-// speculatively on the common path.
-__device__ __noinline__ float div_exact(float a, float b) { return __fdiv_rn(a, b); }
-
-// E2M1 codes of the 16 elements from correctly rounded quotients (the rare
-// path; out of line for the same reason).
-__device__ __noinline__ uint2 e2m1_exact(const float (&x)[16], float eff) {
-  uint32_t b[8];
-#pragma unroll
-  for (int k = 0; k < 8; k++) b[k] = cvt_e2m1x2(__fdiv_rn(x[2 * k], eff), __fdiv_rn(x[2 * k + 1], eff));
-  return make_uint2(pack4(b[0], b[1], b[2], b[3]), pack4(b[4], b[5], b[6], b[7]));
-}
-
-// Exact E2M1 code of fl(x / eff) when |x| / eff is known to lie within
-// 2^-19 (relative) of M, the midpoint between magnitude codes c and c + 1
-// (c in 0..6), for eff >= 2^-98. Then D = |x| - eff * M is a multiple of
-// 2^(e(eff) + e(M) - 25) of magnitude below 2^(e(eff) + e(M) - 17), i.e. a
-// number of at most 8 significant bits, so the fused multiply-add returns it
-// exactly. f = fl(|x| / eff) equals M exactly when -h_below <= D <= h_above
-// (h = eff times half an ulp of M on either side; the quotient of numbers of
-// at most 24 significant bits never falls exactly on an fp32 rounding
-// boundary, so the ends need no tie rule), is above M when D > h_above and
-// below when D < -h_below; on a tie the even code wins.
-__device__ __forceinline__ uint32_t e2m1_resolve(float x, float eff, uint32_t c) {
-  // midpoints 0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5 and their binade exponents
-  const float M = c == 0 ? 0.25f : c == 1 ? 0.75f : c == 2 ? 1.25f : c == 3 ? 1.75f
-                : c == 4 ? 2.5f : c == 5 ? 3.5f : 5.0f;
-  const int eM = c == 0 ? -2 : c == 1 ? -1 : c <= 3 ? 0 : c <= 5 ? 1 : 2;
-  const float h_above = __fmul_rn(eff, __uint_as_float(uint32_t(127 + eM - 24) << 23));
-  const float h_below = c == 0 ? __fmul_rn(h_above, 0.5f) : h_above;  // 0.25 is a power of two
-  const float D = __fmaf_rn(-eff, M, fabsf(x));
-  const uint32_t mag = D > h_above ? c + 1 : (D < -h_below ? c : ((c & 1u) ? c + 1 : c));
-  return mag | ((__float_as_uint(x) >> 31) << 3);
-}
-
-// Byte of two E2M1 codes for (x0, x1) when the bracket codes cl (from the
-// lower products) and ch (upper) disagree in at least one nibble: each
-// disagreeing nibble is decided exactly.
-__device__ __forceinline__ uint32_t fix_pair(float x0, float x1, float eff, uint32_t cl, uint32_t ch) {
-  const bool fma_ok = (__float_as_uint(eff) & 0x7f800000u) >= (29u << 23);  // eff >= 2^-98
-  uint32_t code = cl & 0xffu;
-#pragma unroll
-  for (int e = 0; e < 2; e++) {
-    const uint32_t nl = (cl >> (4 * e)) & 0xfu, nh = (ch >> (4 * e)) & 0xfu;
-    if (nl != nh) {
-      const float xe = e ? x1 : x0;
-      const uint32_t c = min(nl & 7u, nh & 7u);
-      const uint32_t q = fma_ok ? e2m1_resolve(xe, eff, c) : (cvt_e2m1x2(__fdiv_rn(xe, eff), 0.0f) & 0xfu);
-      code = (code & ~(0xfu << (4 * e))) | (q << (4 * e));
-    }
-  }
-  return code;
-}
-
-// The block's codes when the bracket words lo (lower products) and hi
-// (upper) differ: every pair whose bytes differ is decided exactly. Out of
-// line, so that the common path pays one predicted-not-taken branch per block
-// and the exact arithmetic is never evaluated speculatively.
+// Sign-kept zero codes of a block (zero-block guard, eff == 0).
 template <typename InT>
-__device__ __noinline__ uint2 fix_block(In16<InT> v, float eff, uint2 lo, uint2 hi) {
-  uint32_t w[2] = {lo.x, lo.y};
-  const uint32_t hw[2] = {hi.x, hi.y};
+__device__ __forceinline__ uint2 zero_codes(const In16<InT>& v) {
+  const uint32_t sg = v.signs();
+  uint32_t w0 = 0, w1 = 0;
+#pragma unroll
+  for (int i = 0; i < 8; i++) {
+    w0 |= ((sg >> i) & 1u) << (4 * i + 3);
+    w1 |= ((sg >> (i + 8)) & 1u) << (4 * i + 3);
+  }
+  return make_uint2(w0, w1);
+}
+
+// Scale byte and codes of one block by the definition, with IEEE divisions:
+// the path for the rare blocks whose fast-path decision is not certain. Out
+// of line and run after the tile's main loop, so that it costs the main loop
+// nothing.
+template <typename InT>
+__device__ __noinline__ void exact_block(const InT* p, float g, uint8_t* pk, uint8_t* sc) {
+  In16<InT> v;
+  v.template load<false>(p);
+  const float amax = fmaxf(v.absmax(), 0.0f);
+  uint32_t sb = 0;
+  float eff = 0.0f;
+  if (g != 0.0f) {
+    sb = cvt_e4m3x2(__fdiv_rn(amax, __fmul_rn(6.0f, g)), 0.0f) & 0xffu;
+    eff = __fmul_rn(decode_e4m3(sb), g);
+  }
+  uint2 codes;
+  if (eff == 0.0f) {
+    codes = zero_codes(v);
+  } else {
+    uint32_t b[8];
+#pragma unroll
+    for (int k = 0; k < 8; k++) b[k] = cvt_e2m1x2(__fdiv_rn(v.lo(k), eff), __fdiv_rn(v.hi(k), eff));
+    codes = make_uint2(b[0] | (b[1] << 8) | (b[2] << 16) | (b[3] << 24),
+                       b[4] | (b[5] << 8) | (b[6] << 16) | (b[7] << 24));
+  }
+  st_v2(pk, codes);
+  st_u8(sc, sb);
+}
+
+// Packed E2M1 codes (8 bytes, element 2k in the low nibble of byte k) of a
+// block for eff != 0, from the bracketing products x * r (1 -+ 2^-20); *sure
+// is cleared when the two brackets disagree anywhere or eff is outside the
+// range where the approximate reciprocal is normal.
+template <typename InT>
+__device__ __forceinline__ uint2 e2m1_codes(const In16<InT>& v, float eff, bool& sure) {
+  const float r = rcp_approx(eff);
+  const float rl = __fmul_rn(r, 0.99999904632568359375f);  // 1 - 2^-20
+  const float rh = __fmul_rn(r, 1.00000095367431640625f);  // 1 + 2^-20
+  float2 l[8], h[8];
 #pragma unroll
   for (int k = 0; k < 8; k++) {
-    const int sh = 8 * (k & 3);
-    const uint32_t cl = (w[k >> 2] >> sh) & 0xffu, ch = (hw[k >> 2] >> sh) & 0xffu;
-    if (cl != ch) {
-      const uint32_t b = fix_pair(v.lo(k), v.hi(k), eff, cl, ch);
-      w[k >> 2] = (w[k >> 2] & ~(0xffu << sh)) | (b << sh);
-    }
+    l[k] = mul2(v.lo(k), v.hi(k), rl);
+    h[k] = mul2(v.lo(k), v.hi(k), rh);
   }
-  return make_uint2(w[0], w[1]);
-}
-
-// Packed E2M1 codes (8 bytes, element 2k in the low nibble of byte k) of the
-// lane's block for a given eff.
-template <typename InT>
-__device__ __forceinline__ uint2 e2m1_codes(const In16<InT>& v, float eff) {
-  if (eff == 0.0f) {  // zero-block guard: zeros carrying the sign of x
-    const uint32_t sg = v.signs();
-    uint32_t w0 = 0, w1 = 0;
-#pragma unroll
-    for (int i = 0; i < 8; i++) {
-      w0 |= ((sg >> i) & 1u) << (4 * i + 3);
-      w1 |= ((sg >> (i + 8)) & 1u) << (4 * i + 3);
-    }
-    return make_uint2(w0, w1);
-  }
-  if (rcp_safe(eff)) {
-    const float r = rcp_approx(eff);
-    const float rl = __fmul_rn(r, 0.99999904632568359375f);  // 1 - 2^-20
-    const float rh = __fmul_rn(r, 1.00000095367431640625f);  // 1 + 2^-20
-    float2 l[8], h[8];
-#pragma unroll
-    for (int k = 0; k < 8; k++) {
-      l[k] = mul2(v.lo(k), v.hi(k), rl);
-      h[k] = mul2(v.lo(k), v.hi(k), rh);
-    }
-    const uint2 L = make_uint2(cvt_e2m1x8(l[0], l[1], l[2], l[3]), cvt_e2m1x8(l[4], l[5], l[6], l[7]));
-    const uint2 H = make_uint2(cvt_e2m1x8(h[0], h[1], h[2], h[3]), cvt_e2m1x8(h[4], h[5], h[6], h[7]));
-    // a code boundary inside some bracket (exact quotients such as 3.5 are
-    // common with bf16 inputs): decide those elements exactly
-    if (__builtin_expect(((L.x ^ H.x) | (L.y ^ H.y)) != 0u, 0)) return fix_block(v, eff, L, H);
-    return L;
-  }
-  float x[16];
-#pragma unroll
-  for (int k = 0; k < 8; k++) {
-    x[2 * k] = v.lo(k);
-    x[2 * k + 1] = v.hi(k);
-  }
-  return e2m1_exact(x, eff);
+  const uint2 L = make_uint2(cvt_e2m1x8(l[0], l[1], l[2], l[3]), cvt_e2m1x8(l[4], l[5], l[6], l[7]));
+  const uint2 H = make_uint2(cvt_e2m1x8(h[0], h[1], h[2], h[3]), cvt_e2m1x8(h[4], h[5], h[6], h[7]));
+  // a code boundary inside some bracket (exact quotients such as 3.5 are
+  // common with bf16 inputs) leaves the block to the exact path
+  sure = rcp_safe(eff) && ((L.x ^ H.x) | (L.y ^ H.y)) == 0u;
+  return L;
 }
 
 // Quantizes the tile of blocks [tb0, tb0 + nt) (block = 16 elements, row-
@@ -287,6 +234,10 @@ __device__ __forceinline__ uint2 e2m1_codes(const In16<InT>& v, float eff) {
 template <typename InT, bool V8, bool STRIDED, typename GetG>
 __device__ __forceinline__ void quant_tile(const QuantArgs& a, uint64_t tb0, uint32_t nt,
                                            GetG get_g) {
+  __shared__ uint16_t fix_list[kBlocksPerTile];  // tile-local blocks for the exact path
+  __shared__ uint32_t fix_count[1];
+  if (threadIdx.x == 0) *fix_count = 0;
+  __syncthreads();
   const bool full = nt == kBlocksPerTile;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const uint32_t lb0 = warp * kBlocksPerWarp + lane;
@@ -322,16 +273,42 @@ __device__ __forceinline__ void quant_tile(const QuantArgs& a, uint64_t tb0, uin
     const float amax = fmaxf(v[u].absmax(), 0.0f);  // a block holding only NaNs has amax 0
     uint32_t sb = 0;
     float eff = 0.0f;
+    bool sure = true;
     if (!gzero) {
       // E4M3 code of fl(amax / t); the approximate quotient decides unless it
       // is within 32 ulps of a value with four significant bits
-      float s = __fmul_rn(amax, rt);
-      if (__builtin_expect(!t_ok || grid_key<19>(s) <= 64u, 0)) s = div_exact(amax, t);
+      const float s = __fmul_rn(amax, rt);
+      sure = t_ok && grid_key<19>(s) > 64u;
       sb = cvt_e4m3x2(s, 0.0f) & 0xffu;  // NaN -> 0x7F
       eff = __fmul_rn(decode_e4m3(sb), g);
     }
-    st_v2(pk + lb * 8, e2m1_codes(v[u], eff));
+    uint2 codes;
+    if (eff == 0.0f) {
+      codes = zero_codes(v[u]);
+    } else {
+      bool sure_codes;
+      codes = e2m1_codes(v[u], eff, sure_codes);
+      sure = sure && sure_codes;
+    }
+    st_v2(pk + lb * 8, codes);
     st_u8(sc + lb, sb);
+    if (__builtin_expect(!sure, 0)) fix_list[atomicAdd(fix_count, 1u)] = uint16_t(lb);
+  }
+
+  // the blocks left undecided, by the definition (their input is read again)
+  __syncthreads();
+  const uint32_t nfix = *fix_count;
+  for (uint32_t i = threadIdx.x; i < nfix; i += kThreads) {
+    const uint32_t lb = fix_list[i];
+    const InT* p;
+    if constexpr (STRIDED) {
+      const uint64_t blk = tb0 + lb;
+      const uint64_t r = a.rowdiv.div(blk);
+      p = x + r * uint64_t(a.ld) + (blk - r * a.bpr) * 16;
+    } else {
+      p = x + (tb0 + lb) * 16;
+    }
+    exact_block(p, g, pk + lb * 8, sc + lb);
   }
 }
 
