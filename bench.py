@@ -248,6 +248,7 @@ def run_reference(args):
     if rank != 0:
         return
     x_all = W.activation(M=M_ROWS, N=N_COLS)
+    input_sha = hashlib.sha256(x_all.tobytes()).hexdigest()[:16]
     t_row, _, _ = time_oracle_round_trip(np.ascontiguousarray(x_all[:64]), 0.5)
     t_row /= 64
     budget = 150.0
@@ -270,7 +271,7 @@ def run_reference(args):
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": el / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-            "config": config_block(world),
+            "config": config_block(world, input_sha),
             "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle",
                              "sample": f"first {rows} rows per step of the {M_ROWS}x{N_COLS} "
                                        "activation workload, single-threaded scalar C"},
@@ -279,14 +280,17 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
-def config_block(world):
-    return {"workload": f"MXFP8 rowwise quantize (+128x4 swizzled scales) + dequantize round "
+def config_block(world, input_sha=None):
+    c = {"workload": f"MXFP8 rowwise quantize (+128x4 swizzled scales) + dequantize round "
                         f"trip of a bf16 activation {M_ROWS}x{N_COLS}, Student-t(df=3)*0.5, 1% "
                         f"zero groups, 0.5% groups x2^-120, seed 2",
             "shape": [M_ROWS, N_COLS], "input_dtype": "bf16", "group": 32,
             "outputs": "e4m3 u8 [M,N], e8m0 u8 [M,N/32], swizzled e8m0, bf16 [M,N]",
             "l2": "inputs larger than L2 (235 MB bf16 input per step), no flush",
             "parallelism": f"replicas x{world} (rows independent, no exchange)"}
+    if input_sha:
+        c["input_sha256_rank0"] = input_sha
+    return c
 
 
 # -------------------------------------------------------------------- main
@@ -304,6 +308,7 @@ def run(args):
     import ctypes
 
     xb = W.activation(seed=2 + 1000 * rank, M=M_ROWS, N=N_COLS)
+    input_sha = hashlib.sha256(xb.tobytes()).hexdigest()[:16] if rank == 0 else None
     x = torch.from_numpy(xb.view(np.int16)).view(torch.bfloat16).to(device)
     M, N = M_ROWS, N_COLS
     S = N // 32
@@ -421,7 +426,7 @@ def run(args):
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": max_ms / K, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-        "config": config_block(world),
+        "config": config_block(world, input_sha),
         "roofline": {"bound": "hbm", "kernel": dom, "achieved": kernels[dom]["gbs"], "peak": peak,
                      "peak_kind": peak_kind, "unit": "GB/s",
                      "frac": kernels[dom]["gbs"] / peak,
