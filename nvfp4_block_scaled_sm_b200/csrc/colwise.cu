@@ -12,11 +12,12 @@
 // q_t [N, M] (q_t[c, r] is the code of x[r, c]) and scale_t [N, ceil(M/32)].
 //
 // Work split (HBM-bound: 2 bytes read, 1 + 1/32 written per bf16 element;
-// the fused mode writes 2 + 2/32): a CTA stages a tile of 128 rows x 256
-// bytes (128 bf16 or 64 fp32 columns) in shared memory with coalesced
-// 16-byte loads, rows past M and columns past N zero-filled; row pitch 272
-// bytes so that both phases below read shared memory without bank
-// conflicts.
+// the fused mode writes 2 + 2/32): persistent CTAs (two per multiprocessor)
+// walk tiles of 128 rows x 256 bytes (128 bf16 or 64 fp32 columns). A tile is
+// staged in shared memory with 16-byte cp.async copies (rows past M and
+// columns past N zero-filled) into one of two buffers while the previous tile
+// is worked on, so loads overlap compute and stores; row pitch 272 bytes so
+// that both phases below read shared memory without bank conflicts.
 //  - Column phase: a thread owns one 4-byte word column (two bf16 columns or
 //    one fp32 column) and one 32-row group, reads its 32 words down the
 //    rows (consecutive lanes read consecutive words), reduces both bf16
@@ -29,10 +30,6 @@
 // consecutive lanes, and the tile's 4 scale bytes of a column as one word.
 #include "common.cuh"
 
-#ifndef MXQ_COLWISE_ROWS_FAST
-#define MXQ_COLWISE_ROWS_FAST false  // CTA order: column tiles vary fastest
-#endif
-
 namespace mxq {
 namespace {
 
@@ -41,6 +38,15 @@ constexpr int kRowBytes = 256;               // one tile row
 constexpr int kPitch = kRowBytes + 16;       // padded shared-memory row pitch
 constexpr int kWordCols = kRowBytes / 4;     // 64 word columns per tile
 constexpr int kOutPitch = kTileRows + 16;    // shared pitch of a transposed code row
+constexpr uint32_t kInBytes = kTileRows * kPitch;           // one staged input tile
+constexpr uint32_t kQsBytes = (kRowBytes / 2) * kOutPitch;  // transposed codes (bf16: 128 columns)
+constexpr uint32_t kColSmem = 2 * kInBytes + kQsBytes + (kRowBytes / 2) * 4;
+
+// 16-byte asynchronous copy global -> shared; src_bytes == 0 writes zeros.
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes)
+               : "memory");
+}
 
 __device__ __forceinline__ uint32_t lds32(const uint8_t* p) {
   uint32_t v;
@@ -68,7 +74,7 @@ struct ColArgs {
   int64_t ld_bytes;      // input row stride in bytes
   int64_t M, N;
   uint32_t n_ct;         // column tiles
-  uint32_t n_rt;         // row tiles
+  uint32_t ntiles;       // row tiles x column tiles
   uint32_t gt;           // groups per column: ceil(M / 32)
   uint8_t* q_t;          // [N, M]
   uint8_t* scale_t;      // [N, gt]
@@ -93,174 +99,196 @@ __device__ __forceinline__ void column_codes(const float (&f)[32], float mul, ui
                   __byte_perm(c[12], c[13], 0x5410), __byte_perm(c[14], c[15], 0x5410));
 }
 
-template <typename InT, bool ROW, bool ROWS_FAST>
-__global__ void __launch_bounds__(kThreads)
+template <typename InT, bool ROW>
+__global__ void __launch_bounds__(kThreads, 2)
 mxfp8_colwise_kernel(const __grid_constant__ ColArgs a) {
   pdl_enter();
-  __shared__ __align__(16) uint8_t tile[kTileRows * kPitch];
+  extern __shared__ __align__(16) uint8_t smem[];
   constexpr int kEsize = sizeof(InT);
   constexpr int kTileCols = kRowBytes / kEsize;
-  uint8_t* qs = tile;  // transposed codes, written once the input tile is consumed
-  static_assert(kTileCols * kOutPitch <= kTileRows * kPitch, "qs must fit in the tile");
-  __shared__ __align__(16) uint8_t ss[kTileCols * 4];          // scales [column][group]
+  uint8_t* const qs = smem + 2 * kInBytes;  // transposed codes [column][row]
+  uint8_t* const ss = qs + kQsBytes;        // scales [column][group]
   const int t = threadIdx.x;
-  const uint32_t ct = ROWS_FAST ? blockIdx.x / a.n_rt : blockIdx.x % a.n_ct;
-  const uint32_t rt = ROWS_FAST ? blockIdx.x % a.n_rt : blockIdx.x / a.n_ct;
-  const int64_t r0 = int64_t(rt) * kTileRows, c0 = int64_t(ct) * kTileCols;
-  const int rows = a.M - r0 < kTileRows ? int(a.M - r0) : kTileRows;
-  const int row_bytes = (a.N - c0 < kTileCols ? int(a.N - c0) : kTileCols) * kEsize;  // multiple of 32
 
-  // stage the tile: 128 rows x 16 chunks of 16 bytes, 8 chunks per thread
-  uint4 buf[8];
+  // stages tile `tile` into input buffer `b`: 128 rows x 16 chunks of 16
+  // bytes, 8 chunks per thread, zeros past M and N
+  auto stage = [&](uint32_t tile, int b) {
+    const uint32_t ct = tile % a.n_ct, rt = tile / a.n_ct;
+    const int64_t r0 = int64_t(rt) * kTileRows, c0 = int64_t(ct) * kTileCols;
+    const int rows = a.M - r0 < kTileRows ? int(a.M - r0) : kTileRows;
+    const int row_bytes = (a.N - c0 < kTileCols ? int(a.N - c0) : kTileCols) * kEsize;
+    const uint32_t dst = static_cast<uint32_t>(__cvta_generic_to_shared(smem + b * kInBytes));
 #pragma unroll
-  for (int i = 0; i < 8; i++) {
-    const int idx = i * kThreads + t, r = idx >> 4, ch = idx & 15;
-    if (r < rows && ch * 16 < row_bytes)
-      buf[i] = ld_nc_v4(a.x + (r0 + r) * a.ld_bytes + c0 * kEsize + ch * 16);
-    else
-      buf[i] = make_uint4(0, 0, 0, 0);
-  }
-#pragma unroll
-  for (int i = 0; i < 8; i++) {
-    const int idx = i * kThreads + t;
-    sts128(tile + (idx >> 4) * kPitch + (idx & 15) * 16, buf[i]);
-  }
-  __syncthreads();
+    for (int i = 0; i < 8; i++) {
+      const int idx = i * kThreads + t, r = idx >> 4, ch = idx & 15;
+      const bool ok = r < rows && ch * 16 < row_bytes;
+      const uint8_t* src = ok ? a.x + (r0 + r) * a.ld_bytes + c0 * kEsize + ch * 16 : a.x;
+      cp_async16(dst + r * kPitch + ch * 16, src, ok ? 16u : 0u);
+    }
+  };
 
-  // row phase (fused mode): (row, 32-column group) pairs of the tile
-  if constexpr (ROW) {
-    constexpr int kGroups = kTileCols / 32;             // 4 (bf16) or 2 (fp32)
-    constexpr int kPerThread = kTileRows * kGroups / kThreads;
-    const int64_t S = a.N / 32;
+  int b = 0;
+  if (blockIdx.x < a.ntiles) stage(blockIdx.x, 0);
+  asm volatile("cp.async.commit_group;" ::: "memory");
+  for (uint32_t tile = blockIdx.x; tile < a.ntiles; tile += gridDim.x, b ^= 1) {
+    // the next tile's copies go out before this one is worked on
+    if (tile + gridDim.x < a.ntiles) stage(tile + gridDim.x, b ^ 1);
+    asm volatile("cp.async.commit_group;" ::: "memory");
+    asm volatile("cp.async.wait_group 1;" ::: "memory");
+    __syncthreads();  // this tile is in shared memory; the previous one's outputs are written
+
+    const uint8_t* in = smem + b * kInBytes;
+    const uint32_t ct = tile % a.n_ct, rt = tile / a.n_ct;
+    const int64_t r0 = int64_t(rt) * kTileRows, c0 = int64_t(ct) * kTileCols;
+    const int rows = a.M - r0 < kTileRows ? int(a.M - r0) : kTileRows;
+    const int row_bytes = (a.N - c0 < kTileCols ? int(a.N - c0) : kTileCols) * kEsize;  // multiple of 32
+    // row phase (fused mode): (row, 32-column group) pairs of the tile
+    if constexpr (ROW) {
+      constexpr int kGroups = kTileCols / 32;             // 4 (bf16) or 2 (fp32)
+      constexpr int kPerThread = kTileRows * kGroups / kThreads;
+      const int64_t S = a.N / 32;
 #pragma unroll
-    for (int j = 0; j < kPerThread; j++) {
-      const int r = t & (kTileRows - 1);
-      const int k = (t >> 7) * kPerThread + j;
-      if (r < rows && k * 32 * kEsize < row_bytes) {
-        const uint8_t* src = tile + r * kPitch + k * 32 * kEsize;
+      for (int j = 0; j < kPerThread; j++) {
+        const int r = t & (kTileRows - 1);
+        const int k = (t >> 7) * kPerThread + j;
+        if (r < rows && k * 32 * kEsize < row_bytes) {
+          const uint8_t* src = in + r * kPitch + k * 32 * kEsize;
+          float f[32];
+          float amax;
+          if constexpr (kEsize == 2) {
+            uint32_t w[16];
+#pragma unroll
+            for (int i = 0; i < 4; i++) {
+              const uint4 q4 = lds128(src + 16 * i);
+              w[4 * i] = q4.x; w[4 * i + 1] = q4.y; w[4 * i + 2] = q4.z; w[4 * i + 3] = q4.w;
+            }
+            uint32_t m = absmax_bf16x2(w[0], w[1]);
+#pragma unroll
+            for (int i = 2; i < 16; i++) m = absmax_bf16x2(m, w[i]);
+            m &= 0x7fff7fffu;
+            amax = fmaxf(fmaxf(bf16_lo(m), bf16_hi(m)), 0.0f);
+#pragma unroll
+            for (int i = 0; i < 16; i++) {
+              f[2 * i] = bf16_lo(w[i]);
+              f[2 * i + 1] = bf16_hi(w[i]);
+            }
+          } else {
+            amax = 0.0f;
+#pragma unroll
+            for (int i = 0; i < 8; i++) {
+              const uint4 q4 = lds128(src + 16 * i);
+              f[4 * i] = __uint_as_float(q4.x); f[4 * i + 1] = __uint_as_float(q4.y);
+              f[4 * i + 2] = __uint_as_float(q4.z); f[4 * i + 3] = __uint_as_float(q4.w);
+            }
+#pragma unroll
+            for (int i = 0; i < 32; i++) amax = fmaxf(amax, fabsf(f[i]));
+          }
+          const uint32_t b = mx_scale_byte<8>(amax);
+          uint4 lo, hi;
+          column_codes(f, pow2_quant(b), lo, hi);
+          uint8_t* dst = a.q + (r0 + r) * a.N + c0 + 32 * k;
+          st_v4(dst, lo);
+          st_v4(dst + 16, hi);
+          st_u8(a.scale + (r0 + r) * S + c0 / 32 + k, b);
+        }
+      }
+    }
+    // column phase: word column w, group g (rows 32g .. 32g + 31 of the tile);
+    // the codes go to the transposed tile qs[column][row].
+    {
+      const int w = t & (kWordCols - 1), g = t >> 6;
+      const bool active = 32 * g < rows && w * 4 < row_bytes;
+      uint4 code[kEsize == 2 ? 4 : 2];
+      uint32_t sb[2] = {0, 0};
+      if (active) {
+        uint32_t v[32];
+#pragma unroll
+        for (int i = 0; i < 32; i++) v[i] = lds32(in + (32 * g + i) * kPitch + 4 * w);
         float f[32];
-        float amax;
         if constexpr (kEsize == 2) {
-          uint32_t w[16];
+          uint32_t m = absmax_bf16x2(v[0], v[1]);
 #pragma unroll
-          for (int i = 0; i < 4; i++) {
-            const uint4 q4 = lds128(src + 16 * i);
-            w[4 * i] = q4.x; w[4 * i + 1] = q4.y; w[4 * i + 2] = q4.z; w[4 * i + 3] = q4.w;
-          }
-          uint32_t m = absmax_bf16x2(w[0], w[1]);
-#pragma unroll
-          for (int i = 2; i < 16; i++) m = absmax_bf16x2(m, w[i]);
+          for (int i = 2; i < 32; i++) m = absmax_bf16x2(m, v[i]);
           m &= 0x7fff7fffu;
-          amax = fmaxf(fmaxf(bf16_lo(m), bf16_hi(m)), 0.0f);
+          sb[0] = mx_scale_byte<8>(fmaxf(bf16_lo(m), 0.0f));
+          sb[1] = mx_scale_byte<8>(fmaxf(bf16_hi(m), 0.0f));
 #pragma unroll
-          for (int i = 0; i < 16; i++) {
-            f[2 * i] = bf16_lo(w[i]);
-            f[2 * i + 1] = bf16_hi(w[i]);
-          }
+          for (int i = 0; i < 32; i++) f[i] = bf16_lo(v[i]);
+          column_codes(f, pow2_quant(sb[0]), code[0], code[1]);
+#pragma unroll
+          for (int i = 0; i < 32; i++) f[i] = bf16_hi(v[i]);
+          column_codes(f, pow2_quant(sb[1]), code[2], code[3]);
         } else {
-          amax = 0.0f;
+          float amax = 0.0f;
 #pragma unroll
-          for (int i = 0; i < 8; i++) {
-            const uint4 q4 = lds128(src + 16 * i);
-            f[4 * i] = __uint_as_float(q4.x); f[4 * i + 1] = __uint_as_float(q4.y);
-            f[4 * i + 2] = __uint_as_float(q4.z); f[4 * i + 3] = __uint_as_float(q4.w);
+          for (int i = 0; i < 32; i++) {
+            f[i] = __uint_as_float(v[i]);
+            amax = fmaxf(amax, fabsf(f[i]));
           }
-#pragma unroll
-          for (int i = 0; i < 32; i++) amax = fmaxf(amax, fabsf(f[i]));
+          sb[0] = mx_scale_byte<8>(amax);
+          column_codes(f, pow2_quant(sb[0]), code[0], code[1]);
         }
-        const uint32_t b = mx_scale_byte<8>(amax);
-        uint4 lo, hi;
-        column_codes(f, pow2_quant(b), lo, hi);
-        uint8_t* dst = a.q + (r0 + r) * a.N + c0 + 32 * k;
-        st_v4(dst, lo);
-        st_v4(dst + 16, hi);
-        st_u8(a.scale + (r0 + r) * S + c0 / 32 + k, b);
       }
-    }
-  }
-  // column phase: word column w, group g (rows 32g .. 32g + 31 of the tile).
-  // The codes stay in registers until every thread has read the input tile;
-  // then they go to the transposed tile qs[column][row], which reuses the
-  // input tile's shared memory.
-  {
-    const int w = t & (kWordCols - 1), g = t >> 6;
-    const bool active = 32 * g < rows && w * 4 < row_bytes;
-    uint4 code[kEsize == 2 ? 4 : 2];
-    uint32_t sb[2] = {0, 0};
-    if (active) {
-      uint32_t v[32];
+      if (active) {
+        constexpr int kCols = 4 / kEsize;  // columns per word
 #pragma unroll
-      for (int i = 0; i < 32; i++) v[i] = lds32(tile + (32 * g + i) * kPitch + 4 * w);
-      float f[32];
-      if constexpr (kEsize == 2) {
-        uint32_t m = absmax_bf16x2(v[0], v[1]);
-#pragma unroll
-        for (int i = 2; i < 32; i++) m = absmax_bf16x2(m, v[i]);
-        m &= 0x7fff7fffu;
-        sb[0] = mx_scale_byte<8>(fmaxf(bf16_lo(m), 0.0f));
-        sb[1] = mx_scale_byte<8>(fmaxf(bf16_hi(m), 0.0f));
-#pragma unroll
-        for (int i = 0; i < 32; i++) f[i] = bf16_lo(v[i]);
-        column_codes(f, pow2_quant(sb[0]), code[0], code[1]);
-#pragma unroll
-        for (int i = 0; i < 32; i++) f[i] = bf16_hi(v[i]);
-        column_codes(f, pow2_quant(sb[1]), code[2], code[3]);
-      } else {
-        float amax = 0.0f;
-#pragma unroll
-        for (int i = 0; i < 32; i++) {
-          f[i] = __uint_as_float(v[i]);
-          amax = fmaxf(amax, fabsf(f[i]));
+        for (int e = 0; e < kCols; e++) {
+          const int col = kCols * w + e;
+          sts128(qs + col * kOutPitch + 32 * g, code[2 * e]);
+          sts128(qs + col * kOutPitch + 32 * g + 16, code[2 * e + 1]);
+          ss[col * 4 + g] = uint8_t(sb[e]);
         }
-        sb[0] = mx_scale_byte<8>(amax);
-        column_codes(f, pow2_quant(sb[0]), code[0], code[1]);
       }
     }
-    __syncthreads();  // the input tile is dead from here on
-    if (active) {
-      constexpr int kCols = 4 / kEsize;  // columns per word
-#pragma unroll
-      for (int e = 0; e < kCols; e++) {
-        const int col = kCols * w + e;
-        sts128(qs + col * kOutPitch + 32 * g, code[2 * e]);
-        sts128(qs + col * kOutPitch + 32 * g + 16, code[2 * e + 1]);
-        ss[col * 4 + g] = uint8_t(sb[e]);
-      }
-    }
-  }
-  __syncthreads();
+    __syncthreads();
 
-  // write the transposed tile: 8 consecutive lanes write one q_t row's
-  // 128-byte segment (rows of the tile past M are not written)
-  {
-    const int cols = row_bytes / kEsize;
+    // write the transposed tile: 8 consecutive lanes write one q_t row's
+    // 128-byte segment (rows of the tile past M are not written)
+    {
+      const int cols = row_bytes / kEsize;
 #pragma unroll
-    for (int i = 0; i < kTileCols * 8 / kThreads; i++) {
-      const int idx = i * kThreads + t, col = idx >> 3, ch = idx & 7;
-      const int nbytes = rows - 16 * ch;  // valid bytes of this 16-byte chunk
-      if (col < cols && nbytes > 0) {
-        uint8_t* dst = a.q_t + (c0 + col) * a.M + r0 + 16 * ch;
-        const uint4 val = lds128(qs + col * kOutPitch + 16 * ch);
-        if (a.q_t_aligned && nbytes >= 16) {
-          st_v4(dst, val);
+      for (int i = 0; i < kTileCols * 8 / kThreads; i++) {
+        const int idx = i * kThreads + t, col = idx >> 3, ch = idx & 7;
+        const int nbytes = rows - 16 * ch;  // valid bytes of this 16-byte chunk
+        if (col < cols && nbytes > 0) {
+          uint8_t* dst = a.q_t + (c0 + col) * a.M + r0 + 16 * ch;
+          const uint4 val = lds128(qs + col * kOutPitch + 16 * ch);
+          if (a.q_t_aligned && nbytes >= 16) {
+            st_v4(dst, val);
+          } else {
+            const uint32_t wv[4] = {val.x, val.y, val.z, val.w};
+            for (int j = 0; j < (nbytes < 16 ? nbytes : 16); j++)
+              st_u8(dst + j, (wv[j >> 2] >> (8 * (j & 3))) & 0xffu);
+          }
+        }
+      }
+      // scales: the tile's 4 groups of a column are 4 consecutive bytes of scale_t
+      if (t < cols) {
+        const int ng = (rows + 31) / 32;
+        uint8_t* dst = a.scale_t + (c0 + t) * a.gt + r0 / 32;
+        if (ng == 4 && a.scale_words) {
+          st_u32(dst, *reinterpret_cast<const uint32_t*>(ss + 4 * t));
         } else {
-          const uint32_t wv[4] = {val.x, val.y, val.z, val.w};
-          for (int j = 0; j < (nbytes < 16 ? nbytes : 16); j++)
-            st_u8(dst + j, (wv[j >> 2] >> (8 * (j & 3))) & 0xffu);
+          for (int j = 0; j < ng; j++) st_u8(dst + j, ss[4 * t + j]);
         }
       }
     }
-    // scales: the tile's 4 groups of a column are 4 consecutive bytes of scale_t
-    if (t < cols) {
-      const int ng = (rows + 31) / 32;
-      uint8_t* dst = a.scale_t + (c0 + t) * a.gt + r0 / 32;
-      if (ng == 4 && a.scale_words) {
-        st_u32(dst, *reinterpret_cast<const uint32_t*>(ss + 4 * t));
-      } else {
-        for (int j = 0; j < ng; j++) st_u8(dst + j, ss[4 * t + j]);
-      }
-    }
   }
+}
+
+template <typename InT, bool ROW>
+mxq_status launch_colwise(const ColArgs& a, uint32_t grid, cudaStream_t s) {
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [] {
+    attr_err = cudaFuncSetAttribute(mxfp8_colwise_kernel<InT, ROW>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, int(kColSmem));
+  });
+  if (attr_err != cudaSuccess) {
+    record_cuda_error(attr_err);
+    return MXQ_ERR_CUDA;
+  }
+  return launched(launch_pdl_ex(mxfp8_colwise_kernel<InT, ROW>, grid, kThreads, kColSmem, s, a));
 }
 
 }  // namespace
@@ -291,7 +319,7 @@ extern "C" mxq_status mxfp8_quantize_columnwise(const void* x, int dt, int64_t M
   a.M = M;
   a.N = N;
   a.n_ct = uint32_t(n_ct);
-  a.n_rt = uint32_t(n_rt);
+  a.ntiles = uint32_t(n_rt * n_ct);
   a.gt = uint32_t((uint64_t(M) + 31) / 32);
   a.q_t = qweight_t;
   a.scale_t = scale_t;
@@ -300,11 +328,9 @@ extern "C" mxq_status mxfp8_quantize_columnwise(const void* x, int dt, int64_t M
   a.q_t_aligned = (M % 16) == 0;
   a.scale_words = (reinterpret_cast<uintptr_t>(scale_t) & 3u) == 0 && (a.gt & 3u) == 0;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  const uint32_t grid = uint32_t(n_rt * n_ct);
-  if (dt == MXQ_BF16) {
-    return launched(fused ? launch_pdl(mxfp8_colwise_kernel<uint16_t, true, MXQ_COLWISE_ROWS_FAST>, grid, s, a)
-                          : launch_pdl(mxfp8_colwise_kernel<uint16_t, false, MXQ_COLWISE_ROWS_FAST>, grid, s, a));
-  }
-  return launched(fused ? launch_pdl(mxfp8_colwise_kernel<float, true, MXQ_COLWISE_ROWS_FAST>, grid, s, a)
-                        : launch_pdl(mxfp8_colwise_kernel<float, false, MXQ_COLWISE_ROWS_FAST>, grid, s, a));
+  const uint64_t resident = uint64_t(sm_count()) * 2;
+  const uint32_t grid = uint32_t(a.ntiles < resident ? a.ntiles : resident);
+  if (dt == MXQ_BF16)
+    return fused ? launch_colwise<uint16_t, true>(a, grid, s) : launch_colwise<uint16_t, false>(a, grid, s);
+  return fused ? launch_colwise<float, true>(a, grid, s) : launch_colwise<float, false>(a, grid, s);
 }
