@@ -40,7 +40,12 @@ constexpr int kWordCols = kRowBytes / 4;     // 64 word columns per tile
 constexpr int kOutPitch = kTileRows + 16;    // shared pitch of a transposed code row
 constexpr uint32_t kInBytes = kTileRows * kPitch;           // one staged input tile
 constexpr uint32_t kQsBytes = (kRowBytes / 2) * kOutPitch;  // transposed codes (bf16: 128 columns)
-constexpr uint32_t kColSmem = 2 * kInBytes + kQsBytes + (kRowBytes / 2) * 4;
+constexpr uint32_t kSsBytes = (kRowBytes / 2) * 4;           // column scales of a tile
+constexpr int kRowPitch = kRowBytes / 2 + 16;                // shared pitch of a row of codes
+constexpr uint32_t kQrBytes = kTileRows * kRowPitch;          // rowwise codes (fused mode)
+constexpr uint32_t kSrBytes = kTileRows * 4;                  // rowwise scales (fused mode)
+constexpr uint32_t kColSmem = 2 * kInBytes + kQsBytes + kSsBytes;
+constexpr uint32_t kFusedSmem = kColSmem + kQrBytes + kSrBytes;
 
 // 16-byte asynchronous copy global -> shared; src_bytes == 0 writes zeros.
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
@@ -108,6 +113,8 @@ mxfp8_colwise_kernel(const __grid_constant__ ColArgs a) {
   constexpr int kTileCols = kRowBytes / kEsize;
   uint8_t* const qs = smem + 2 * kInBytes;  // transposed codes [column][row]
   uint8_t* const ss = qs + kQsBytes;        // scales [column][group]
+  uint8_t* const qr = ss + kSsBytes;        // fused mode: rowwise codes [row][column]
+  uint8_t* const sr = qr + kQrBytes;        // fused mode: rowwise scales [row][group]
   const int t = threadIdx.x;
 
   // stages tile `tile` into input buffer `b`: 128 rows x 16 chunks of 16
@@ -146,7 +153,6 @@ mxfp8_colwise_kernel(const __grid_constant__ ColArgs a) {
     if constexpr (ROW) {
       constexpr int kGroups = kTileCols / 32;             // 4 (bf16) or 2 (fp32)
       constexpr int kPerThread = kTileRows * kGroups / kThreads;
-      const int64_t S = a.N / 32;
 #pragma unroll
       for (int j = 0; j < kPerThread; j++) {
         const int r = t & (kTileRows - 1);
@@ -186,10 +192,9 @@ mxfp8_colwise_kernel(const __grid_constant__ ColArgs a) {
           const uint32_t b = mx_scale_byte<8>(amax);
           uint4 lo, hi;
           column_codes(f, pow2_quant(b), lo, hi);
-          uint8_t* dst = a.q + (r0 + r) * a.N + c0 + 32 * k;
-          st_v4(dst, lo);
-          st_v4(dst + 16, hi);
-          st_u8(a.scale + (r0 + r) * S + c0 / 32 + k, b);
+          sts128(qr + r * kRowPitch + 32 * k, lo);
+          sts128(qr + r * kRowPitch + 32 * k + 16, hi);
+          sr[4 * r + k] = uint8_t(b);
         }
       }
     }
@@ -273,22 +278,42 @@ mxfp8_colwise_kernel(const __grid_constant__ ColArgs a) {
         }
       }
     }
+    // fused mode: the rowwise codes of the tile, one row's segment (128 or 64
+    // bytes) written by 8 or 4 consecutive lanes, and its scale bytes
+    if constexpr (ROW) {
+      constexpr int kChunks = kTileCols / 16;  // 16-byte chunks of a row's codes
+      const int64_t S = a.N / 32;
+#pragma unroll
+      for (int i = 0; i < kTileRows * kChunks / kThreads; i++) {
+        const int idx = i * kThreads + t, r = idx / kChunks, ch = idx % kChunks;
+        if (r < rows && ch * 16 < row_bytes / kEsize)
+          st_v4(a.q + (r0 + r) * a.N + c0 + 16 * ch, lds128(qr + r * kRowPitch + 16 * ch));
+      }
+      if (t < rows) {
+        constexpr int kGroups = kTileCols / 32;
+        const int ng = row_bytes / kEsize / 32;
+        uint8_t* dst = a.scale + (r0 + t) * S + c0 / 32;
+        for (int j = 0; j < ng; j++) st_u8(dst + j, sr[4 * t + j]);
+        (void)kGroups;
+      }
+    }
   }
 }
 
 template <typename InT, bool ROW>
 mxq_status launch_colwise(const ColArgs& a, uint32_t grid, cudaStream_t s) {
+  constexpr uint32_t kSmem = ROW ? kFusedSmem : kColSmem;
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(once, [] {
     attr_err = cudaFuncSetAttribute(mxfp8_colwise_kernel<InT, ROW>,
-                                    cudaFuncAttributeMaxDynamicSharedMemorySize, int(kColSmem));
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmem));
   });
   if (attr_err != cudaSuccess) {
     record_cuda_error(attr_err);
     return MXQ_ERR_CUDA;
   }
-  return launched(launch_pdl_ex(mxfp8_colwise_kernel<InT, ROW>, grid, kThreads, kColSmem, s, a));
+  return launched(launch_pdl_ex(mxfp8_colwise_kernel<InT, ROW>, grid, kThreads, kSmem, s, a));
 }
 
 }  // namespace
