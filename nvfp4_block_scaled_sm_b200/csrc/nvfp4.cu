@@ -58,6 +58,9 @@ constexpr int kAmaxCtasPerSm = 8;   // one resident wave: grid = SMs x 8
 constexpr int kSteps = 2;
 constexpr int kBlocksPerWarp = 32 * kSteps;
 constexpr int kBlocksPerTile = kBlocksPerWarp * (kThreads / 32);
+constexpr int kDqSteps = 2;  // dequantize: blocks per lane
+constexpr int kDqBlocksPerWarp = 32 * kDqSteps;
+constexpr int kDqBlocksPerTile = kDqBlocksPerWarp * (kThreads / 32);
 
 enum GMode { kFromPartials = 0, kGiven = 1, kFromAmax = 2 };
 
@@ -444,16 +447,16 @@ __global__ void __launch_bounds__(kThreads)
 nvfp4_dequant_kernel(const uint8_t* __restrict__ packed, const uint8_t* __restrict__ bscale,
                      const float* __restrict__ gs, OutT* __restrict__ y, uint64_t nblocks) {
   pdl_enter();
-  const uint64_t tb0 = uint64_t(blockIdx.x) * kBlocksPerTile;
+  const uint64_t tb0 = uint64_t(blockIdx.x) * kDqBlocksPerTile;
   const uint64_t left = nblocks - tb0;
-  const uint32_t nt = left < kBlocksPerTile ? uint32_t(left) : uint32_t(kBlocksPerTile);
-  const bool full = nt == kBlocksPerTile;
+  const uint32_t nt = left < kDqBlocksPerTile ? uint32_t(left) : uint32_t(kDqBlocksPerTile);
+  const bool full = nt == kDqBlocksPerTile;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const uint32_t lb0 = warp * kBlocksPerWarp + lane;
-  uint2 w[kSteps];
-  uint32_t sb[kSteps];
+  const uint32_t lb0 = warp * kDqBlocksPerWarp + lane;
+  uint2 w[kDqSteps];
+  uint32_t sb[kDqSteps];
 #pragma unroll
-  for (int u = 0; u < kSteps; u++) {
+  for (int u = 0; u < kDqSteps; u++) {
     const uint32_t lb = lb0 + 32 * u;
     if (full || lb < nt) {
       w[u] = ld_nc_v2(packed + (tb0 + lb) * 8);
@@ -465,7 +468,7 @@ nvfp4_dequant_kernel(const uint8_t* __restrict__ packed, const uint8_t* __restri
   }
   const float g = *gs;
 #pragma unroll
-  for (int u = 0; u < kSteps; u++) {
+  for (int u = 0; u < kDqSteps; u++) {
     const uint32_t lb = lb0 + 32 * u;
     if (!(full || lb < nt)) continue;
     const float eff = __fmul_rn(decode_e4m3(sb[u]), g);
@@ -861,7 +864,7 @@ mxq_status nvfp4_dequantize(const uint8_t* packed, const uint8_t* block_scale,
   if (!packed || !block_scale || !global_scale || !y) return MXQ_ERR_NULL;
   if (!aligned16(packed) || !aligned16(y)) return MXQ_ERR_ALIGN;
   const uint64_t nblocks = uint64_t(M) * (uint64_t(N) / 16);
-  const uint64_t tiles = (nblocks + kBlocksPerTile - 1) / kBlocksPerTile;
+  const uint64_t tiles = (nblocks + kDqBlocksPerTile - 1) / kDqBlocksPerTile;
   if (tiles > 0x7fffffffull) return MXQ_ERR_SHAPE;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const uint32_t grid = uint32_t(tiles);
