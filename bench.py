@@ -355,6 +355,10 @@ def run(args):
             if e:
                 e[2].record(stream)
         t_end.record(stream)
+        # wait by polling so that the sampler thread gets the interpreter while
+        # the GPU works through the queued steps
+        while not t_end.query():
+            time.sleep(0.0002)
         torch.cuda.synchronize(device)
     if world > 1:
         torch.distributed.barrier()
