@@ -15,26 +15,32 @@
 // TransformerEngine for MXFP8 quantization" (the quantized weights feed the
 // GEMM); the scale-tile layout is the one the block-scaled MMA reads.
 //
-// Structure (one CTA per 128 x BN output tile, BN = 128 or 256, 128 threads):
+// Structure: persistent CTAs (one per multiprocessor) walk 128 x BN output
+// tiles (BN = 256, or 128 when N <= 128) with six warps:
 //  - warp 0, one lane: producer. Per K block of 128: TMA loads of the A tile
 //    (128 rows x 128 bytes) and the B tile (BN rows x 128 bytes), both with
 //    the 128-byte swizzle, and bulk copies of the 512-byte scale tiles (one
-//    for A, BN / 128 for B) into one of the shared-memory stages; completion
-//    is counted in bytes on the stage's "full" mbarrier.
-//  - warp 1, one lane: MMA issuer. Copies the stage's scale tiles into tensor
-//    memory (tcgen05.cp 32x128b.warpx4, the 32 x 16-byte scale tile
-//    broadcast to the four lane quarters), issues four MMAs of K = 32 (one
-//    scale column each, selected by the scale-factor id; M = 128, N = BN),
-//    then commits the
-//    stage's "empty" mbarrier; after the last block it commits "accum".
-//  - all four warps: epilogue. Each warp reads its 32 accumulator lanes
-//    (tcgen05.ld 32x32b) and writes its rows of D as bf16 or fp32.
+//    for A, BN / 128 for B) into the next shared-memory stage; completion is
+//    counted in bytes on the stage's "full" mbarrier. The stages run on
+//    across tiles, so the next tile's loads overlap this tile's epilogue.
+//  - warp 1, one lane: MMA issuer. Waits until the epilogue has read the
+//    previous tile's accumulator ("acc_empty"), then per stage copies the
+//    scale tiles into tensor memory (tcgen05.cp 32x128b.warpx4, the 32 x
+//    16-byte scale tile broadcast to the four lane quarters), issues four
+//    MMAs of K = 32 (one scale column each, selected by the scale-factor id;
+//    M = 128, N = BN) and commits the stage's "empty" mbarrier; after the
+//    tile's last stage it commits "acc_full".
+//  - warps 2-5: epilogue. Each reads its quarter of the accumulator lanes
+//    (tcgen05.ld 32x32b, warp w takes lanes 32 (w % 4) ..), hands the
+//    accumulator back once the last columns are in registers, and writes its
+//    rows of D as bf16 or fp32 while the next tile's MMAs run.
 // Tensor memory: BN columns of fp32 accumulator plus 4 scale columns per
 // 128-row scale tile and stage (4 for A, 4 or 8 for B).
 //
-// Every wait on an mbarrier gives up after about one second (by %globaltimer)
-// or 2^30 polls; the kernel then records an error code in *err (when err is
-// not NULL), skips the remaining work, frees its tensor memory and returns.
+// Every wait on an mbarrier gives up after about one second (by %globaltimer,
+// from the start of that wait) or 2^30 polls; the kernel then records an
+// error code in *err (when err is not NULL), skips the remaining work, frees
+// its tensor memory and returns.
 #include "common.cuh"
 #include "tma.cuh"
 
@@ -42,7 +48,8 @@ namespace mxq {
 namespace {
 
 constexpr int kBM = 128, kBK = 128;  // kBK elements = bytes of E4M3
-constexpr int kGemmThreads = 128;
+constexpr int kEpilogueWarps = 4;
+constexpr int kGemmThreads = 32 * (2 + kEpilogueWarps);  // producer, MMA, epilogue warps
 constexpr uint32_t kSfTile = 512;    // one 128 x 4 scale tile
 constexpr uint32_t kBarBytes = 256;
 constexpr uint64_t kWaitNs = 1000000000ull;  // one second
@@ -73,6 +80,8 @@ struct GemmArgs {
   uint32_t nk;          // K blocks of 128
   uint32_t kp4;         // 4-column scale tiles per 128-row block: ceil(K / 128)
   uint32_t nb128;       // 128-row blocks of B's scales: ceil(N / 128)
+  uint32_t n_tiles_n;   // output tiles along N
+  uint32_t ntiles;      // output tiles
 };
 
 // Shared-memory matrix descriptor (tcgen05): start address, leading and
@@ -159,15 +168,16 @@ mxfp8_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_consta
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
   uint8_t* smem = smem_raw + (base - raw);
-  const uint32_t bars = base + kStages * kStageBytes;  // full[s], empty[s], accum, tmem slot
+  // full[s], empty[s], acc_full, acc_empty, tmem slot
+  const uint32_t bars = base + kStages * kStageBytes;
   auto full_bar = [&](int s) { return bars + 8u * s; };
   auto empty_bar = [&](int s) { return bars + 8u * (kStages + s); };
-  const uint32_t accum_bar = bars + 8u * (2 * kStages);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kStages * kStageBytes + 8 * (2 * kStages + 1));
+  const uint32_t acc_full = bars + 8u * (2 * kStages);
+  const uint32_t acc_empty = acc_full + 8u;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kStages * kStageBytes + 8 * (2 * kStages + 2));
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const uint32_t n_blk = blockIdx.x, m_blk = blockIdx.y;
-  const uint64_t deadline = globaltimer() + kWaitNs;
+  const uint32_t n_my = (a.ntiles - blockIdx.x + gridDim.x - 1) / gridDim.x;  // grid <= tiles
 
   if (warp == 0) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
@@ -179,7 +189,8 @@ mxfp8_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_consta
       mbar_init(full_bar(s), 1);
       mbar_init(empty_bar(s), 1);
     }
-    mbar_init(accum_bar, 1);
+    mbar_init(acc_full, 1);
+    mbar_init(acc_empty, kEpilogueWarps);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   tc_fence_before();
@@ -189,103 +200,136 @@ mxfp8_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_consta
 
   if (warp == 0 && lane == 0) {
     // ---------------------------------------------------------- producer
-    const uint8_t* sfa = a.sfa + (uint64_t(m_blk) * a.kp4) * kSfTile;
-    // B's 128-row scale blocks of this tile that exist (the last tile of a
-    // ragged N may have fewer than BN / 128; its missing rows are never stored)
-    const uint32_t b0 = n_blk * C::kSfbTiles;
-    const uint32_t nsfb = min(C::kSfbTiles, a.nb128 - b0);
-    const uint32_t tx = C::kTileA + C::kTileB + kSfTile * (1 + nsfb);
-    for (uint32_t kb = 0; kb < a.nk; kb++) {
-      const int s = kb % kStages;
-      const uint32_t phase = (kb / kStages) & 1u;
-      if (!mbar_wait(empty_bar(s), phase ^ 1u, deadline)) {
-        record_error(a.err, kErrEmptyWait);
-        break;
+    // stages run on across tiles, so the next tile's loads overlap this
+    // tile's last MMAs and its epilogue
+    uint32_t it = 0;
+    for (uint32_t i = 0; i < n_my; i++) {
+      const uint32_t tile = blockIdx.x + i * gridDim.x;
+      const uint32_t m_blk = tile / a.n_tiles_n, n_blk = tile % a.n_tiles_n;
+      const uint8_t* sfa = a.sfa + (uint64_t(m_blk) * a.kp4) * kSfTile;
+      // B's 128-row scale blocks of this tile that exist (the last tile of a
+      // ragged N may have fewer than BN / 128; its missing rows are never stored)
+      const uint32_t b0 = n_blk * C::kSfbTiles;
+      const uint32_t nsfb = min(C::kSfbTiles, a.nb128 - b0);
+      const uint32_t tx = C::kTileA + C::kTileB + kSfTile * (1 + nsfb);
+      bool ok = true;
+      for (uint32_t kb = 0; kb < a.nk; kb++, it++) {
+        const int s = it % kStages;
+        const uint32_t phase = (it / kStages) & 1u;
+        if (!mbar_wait(empty_bar(s), phase ^ 1u, kWaitNs)) {
+          record_error(a.err, kErrEmptyWait);
+          ok = false;
+          break;
+        }
+        const uint32_t st = base + s * kStageBytes;
+        mbar_expect_tx(full_bar(s), tx);
+        tma_load_2d(st, &tma_a, full_bar(s), int32_t(kb * kBK), int32_t(m_blk * kBM));
+        tma_load_2d(st + C::kTileA, &tma_b, full_bar(s), int32_t(kb * kBK), int32_t(n_blk * BN));
+        const uint32_t sf = st + C::kTileA + C::kTileB;
+        bulk_load(sf, sfa + uint64_t(kb) * kSfTile, kSfTile, full_bar(s));
+        for (uint32_t j = 0; j < nsfb; j++)
+          bulk_load(sf + kSfTile * (1 + j), a.sfb + (uint64_t(b0 + j) * a.kp4 + kb) * kSfTile, kSfTile,
+                    full_bar(s));
       }
-      const uint32_t st = base + s * kStageBytes;
-      mbar_expect_tx(full_bar(s), tx);
-      tma_load_2d(st, &tma_a, full_bar(s), int32_t(kb * kBK), int32_t(m_blk * kBM));
-      tma_load_2d(st + C::kTileA, &tma_b, full_bar(s), int32_t(kb * kBK), int32_t(n_blk * BN));
-      const uint32_t sf = st + C::kTileA + C::kTileB;
-      bulk_load(sf, sfa + uint64_t(kb) * kSfTile, kSfTile, full_bar(s));
-      for (uint32_t j = 0; j < nsfb; j++)
-        bulk_load(sf + kSfTile * (1 + j), a.sfb + (uint64_t(b0 + j) * a.kp4 + kb) * kSfTile, kSfTile,
-                  full_bar(s));
+      if (!ok) break;
     }
   } else if (warp == 1 && lane == 0) {
     // ------------------------------------------------------- MMA issuer
-    bool ok = true;
-    for (uint32_t kb = 0; kb < a.nk; kb++) {
-      const int s = kb % kStages;
-      const uint32_t phase = (kb / kStages) & 1u;
-      if (!mbar_wait(full_bar(s), phase, deadline)) {
-        record_error(a.err, kErrFullWait);
-        ok = false;
+    uint32_t it = 0;
+    for (uint32_t i = 0; i < n_my; i++) {
+      // the epilogue must have read the previous tile's accumulator
+      if (i > 0 && !mbar_wait(acc_empty, (i - 1) & 1u, kWaitNs)) {
+        record_error(a.err, kErrAccumWait);
         break;
       }
       tc_fence_after();
-      const uint32_t st = base + s * kStageBytes;
-      const uint32_t sfa_t = tmem + BN + C::kSfColsPerStage * s;
-      const uint32_t sfb_t = sfa_t + 4u;
-      const uint32_t sf = st + C::kTileA + C::kTileB;
-      tmem_copy_scales(sfa_t, scale_desc(sf));
+      bool ok = true;
+      for (uint32_t kb = 0; kb < a.nk; kb++, it++) {
+        const int s = it % kStages;
+        const uint32_t phase = (it / kStages) & 1u;
+        if (!mbar_wait(full_bar(s), phase, kWaitNs)) {
+          record_error(a.err, kErrFullWait);
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t st = base + s * kStageBytes;
+        const uint32_t sfa_t = tmem + BN + C::kSfColsPerStage * s;
+        const uint32_t sfb_t = sfa_t + 4u;
+        const uint32_t sf = st + C::kTileA + C::kTileB;
+        tmem_copy_scales(sfa_t, scale_desc(sf));
 #pragma unroll
-      for (uint32_t j = 0; j < C::kSfbTiles; j++)
-        tmem_copy_scales(sfb_t + 4u * j, scale_desc(sf + kSfTile * (1 + j)));
+        for (uint32_t j = 0; j < C::kSfbTiles; j++)
+          tmem_copy_scales(sfb_t + 4u * j, scale_desc(sf + kSfTile * (1 + j)));
 #pragma unroll
-      for (uint32_t k = 0; k < 4; k++) {
-        mma_mxf8(tmem, operand_desc(st + 32u * k), operand_desc(st + C::kTileA + 32u * k),
-                 instr_desc<BN>(k), sfa_t | (k << 30), sfb_t | (k << 30), (kb | k) != 0u);
+        for (uint32_t k = 0; k < 4; k++) {
+          mma_mxf8(tmem, operand_desc(st + 32u * k), operand_desc(st + C::kTileA + 32u * k),
+                   instr_desc<BN>(k), sfa_t | (k << 30), sfb_t | (k << 30), (kb | k) != 0u);
+        }
+        mma_commit(empty_bar(s));
       }
-      mma_commit(empty_bar(s));
+      if (!ok) break;
+      mma_commit(acc_full);
     }
-    if (ok) mma_commit(accum_bar);
-  }
-  __syncwarp();
-
-  // ------------------------------------------------------------ epilogue
-  // the phase completes once for everyone: a lane that saw it lets the warp go
-  const bool have = __any_sync(0xffffffffu, a.nk > 0 && mbar_wait(accum_bar, 0, deadline));
-  if (a.nk > 0 && !have && lane == 0) record_error(a.err, kErrAccumWait);
-  tc_fence_after();
-  if (have) {
-    const uint32_t row = m_blk * kBM + warp * 32 + lane;
-    const uint32_t taddr = tmem + (uint32_t(warp * 32) << 16);
-    OutT* drow = static_cast<OutT*>(a.d) + uint64_t(row) * a.N + uint64_t(n_blk) * BN;
-    const uint32_t ncols = min(uint32_t(BN), a.N - n_blk * BN);
+  } else if (warp >= 2) {
+    // ------------------------------------------------------------ epilogue
+    // warp w reads accumulator lanes (rows) 32 (w % 4) .. 32 (w % 4) + 31
+    const uint32_t quarter = uint32_t(warp & 3);
+    const uint32_t taddr = tmem + ((quarter * 32) << 16);
+    for (uint32_t i = 0; i < n_my; i++) {
+      const uint32_t tile = blockIdx.x + i * gridDim.x;
+      const uint32_t m_blk = tile / a.n_tiles_n, n_blk = tile % a.n_tiles_n;
+      // the phase completes once for everyone: a lane that saw it lets the warp go
+      const bool have = __any_sync(0xffffffffu, mbar_wait(acc_full, i & 1u, kWaitNs));
+      if (!have) {
+        if (lane == 0) record_error(a.err, kErrAccumWait);
+        break;
+      }
+      tc_fence_after();
+      const uint32_t row = m_blk * kBM + quarter * 32 + lane;
+      OutT* drow = static_cast<OutT*>(a.d) + uint64_t(row) * a.N + uint64_t(n_blk) * BN;
+      const uint32_t ncols = min(uint32_t(BN), a.N - n_blk * BN);
 #pragma unroll 1
-    for (uint32_t c0 = 0; c0 < uint32_t(BN); c0 += 32) {
-      uint32_t r[32];
-      tmem_ld32(taddr + c0, r);  // every lane of the warp takes part
-      if (row >= a.M || c0 >= ncols) continue;
-      if constexpr (sizeof(OutT) == 2) {
-        uint32_t w[16];
-#pragma unroll
-        for (int i = 0; i < 16; i++)
-          w[i] = cvt_bf16x2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
-        if (c0 + 32 <= ncols) {
-#pragma unroll
-          for (int i = 0; i < 4; i++)
-            st_v4(drow + c0 + 8 * i, make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]));
-        } else {
-#pragma unroll
-          for (uint32_t i = 0; i < 16; i++)
-            if (c0 + 2 * i < ncols) st_u32(drow + c0 + 2 * i, w[i]);
+      for (uint32_t c0 = 0; c0 < uint32_t(BN); c0 += 32) {
+        uint32_t r[32];
+        tmem_ld32(taddr + c0, r);  // every lane of the warp takes part
+        if (c0 + 32 >= uint32_t(BN)) {
+          // the whole accumulator is in registers: hand it back to the MMA
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(acc_empty);
         }
-      } else {
-        if (c0 + 32 <= ncols) {
+        if (row >= a.M || c0 >= ncols) continue;
+        if constexpr (sizeof(OutT) == 2) {
+          uint32_t w[16];
 #pragma unroll
-          for (int i = 0; i < 8; i++)
-            st_v4(drow + c0 + 4 * i, make_uint4(r[4 * i], r[4 * i + 1], r[4 * i + 2], r[4 * i + 3]));
+          for (int q = 0; q < 16; q++)
+            w[q] = cvt_bf16x2(__uint_as_float(r[2 * q]), __uint_as_float(r[2 * q + 1]));
+          if (c0 + 32 <= ncols) {
+#pragma unroll
+            for (int q = 0; q < 4; q++)
+              st_v4(drow + c0 + 8 * q, make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]));
+          } else {
+#pragma unroll
+            for (uint32_t q = 0; q < 16; q++)
+              if (c0 + 2 * q < ncols) st_u32(drow + c0 + 2 * q, w[q]);
+          }
         } else {
+          if (c0 + 32 <= ncols) {
 #pragma unroll
-          for (uint32_t i = 0; i < 32; i++)
-            if (c0 + i < ncols) st_u32(drow + c0 + i, r[i]);
+            for (int q = 0; q < 8; q++)
+              st_v4(drow + c0 + 4 * q, make_uint4(r[4 * q], r[4 * q + 1], r[4 * q + 2], r[4 * q + 3]));
+          } else {
+#pragma unroll
+            for (uint32_t q = 0; q < 32; q++)
+              if (c0 + q < ncols) st_u32(drow + c0 + q, r[q]);
+          }
         }
       }
     }
   }
 
+  __syncwarp();
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {
@@ -326,8 +370,12 @@ mxq_status launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const GemmA
     record_cuda_error(attr_err);
     return MXQ_ERR_CUDA;
   }
-  const dim3 grid((args.N + BN - 1) / BN, (args.M + kBM - 1) / kBM);
-  mxfp8_gemm_kernel<OutT, BN><<<grid, kGemmThreads, kSmemBytes, s>>>(ta, tb, args);
+  GemmArgs a2 = args;
+  a2.n_tiles_n = (args.N + BN - 1) / BN;
+  a2.ntiles = a2.n_tiles_n * ((args.M + kBM - 1) / kBM);
+  const uint32_t sms = uint32_t(sm_count());
+  const uint32_t grid = a2.ntiles < sms ? a2.ntiles : sms;
+  mxfp8_gemm_kernel<OutT, BN><<<grid, kGemmThreads, kSmemBytes, s>>>(ta, tb, a2);
   return check_launch();
 }
 

@@ -31,9 +31,11 @@ __device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
                : "memory");
 }
 
-// Waits until the phase of parity `parity` has completed; false once the
-// deadline (%globaltimer, ns) has passed or after 2^30 polls.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint64_t deadline) {
+// Waits until the phase of parity `parity` has completed; false once
+// timeout_ns (by %globaltimer) have passed since the call, or after 2^30
+// polls.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint64_t timeout_ns) {
+  uint64_t deadline = 0;
   for (uint32_t it = 0; it < (1u << 30); ++it) {
     uint32_t done;
     asm volatile(
@@ -42,7 +44,11 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint64_
         : "r"(bar), "r"(parity)
         : "memory");
     if (done) return true;
-    if ((it & 15u) == 15u && globaltimer() > deadline) return false;
+    if ((it & 15u) == 15u) {
+      const uint64_t now = globaltimer();
+      if (deadline == 0) deadline = now + timeout_ns;
+      else if (now > deadline) return false;
+    }
   }
   return false;
 }

@@ -64,7 +64,8 @@ def check_tol(d, exact, absum, K, bf16, what):
 
 
 @pytest.mark.parametrize("M,N,K", [(128, 128, 128), (256, 384, 1024), (33, 48, 96), (1, 16, 32),
-                                   (200, 144, 2048), (300, 272, 160)])
+                                   (200, 144, 2048), (300, 272, 160),
+                                   (2048, 4096, 256), (3000, 3008, 96)])  # more tiles than SMs
 def test_power_of_two_grid_is_exact(M, N, K):
     xa = W.gemm_pow2_operand(1000 + M, M, K)
     xb = W.gemm_pow2_operand(2000 + N, N, K)
