@@ -499,6 +499,15 @@ def run_suite(device, only=None):
     def bf(a):
         return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(device)
 
+    def planted():
+        x = bf(W.planted())
+        emit("mxfp8_quantize planted 256x1024 (L2-flushed, launch-bound)",
+             mxfp8_quant_bytes(256, 1024, swizzled=False),
+             time_kernel(lambda: mxq.mxfp8_quantize(x), 50, flush))
+        q, s = mxq.mxfp8_quantize(x)
+        emit("mxfp8_dequantize->bf16 planted 256x1024 (L2-flushed, launch-bound)",
+             mxfp8_dequant_bytes(256, 1024), time_kernel(lambda: mxq.mxfp8_dequantize(q, s), 50, flush))
+
     def linear_weight():
         x = bf(W.linear_weight())
         emit("mxfp8_quantize linear_weight 4096x4096", mxfp8_quant_bytes(4096, 4096, swizzled=False),
@@ -586,7 +595,8 @@ def run_suite(device, only=None):
         emit("nvfp4_dequantize->bf16 8192x8192", 8192 * 8192 // 2 + 8192 * 512 + 8192 * 8192 * 2,
              time_kernel(lambda: mxq.nvfp4_dequantize(p, b, g), 30))
 
-    for name, fn in (("gemm", gemm), ("linear_weight", linear_weight), ("activation", activation),
+    for name, fn in (("planted", planted), ("gemm", gemm), ("linear_weight", linear_weight),
+                     ("activation", activation),
                      ("mxfp4 activation", mxfp4_activation), ("fake activation", fake_activation),
                      ("experts", experts), ("nvfp4", nvfp4)):
         if only is None or only in name:
