@@ -485,6 +485,8 @@ def run_suite(device, only=None):
     """One JSON line per workload kernel: median device time over repeated
     launches (L2 flushed between launches for the 50 MB workload, the others
     exceed L2), algorithmic bytes, GB/s and fraction of the HBM peak."""
+    import ctypes
+
     import nvfp4_block_scaled_sm_b200 as mxq
     peak, kind = hbm_peak()
     flush = torch.empty(64 * 2**20, dtype=torch.float32, device=device)  # 256 MB > L2
@@ -510,8 +512,26 @@ def run_suite(device, only=None):
 
     def linear_weight():
         x = bf(W.linear_weight())
-        emit("mxfp8_quantize linear_weight 4096x4096", mxfp8_quant_bytes(4096, 4096, swizzled=False),
+        emit("mxfp8_quantize linear_weight 4096x4096 (L2 flushed by a 256 MB write)",
+             mxfp8_quant_bytes(4096, 4096, swizzled=False),
              time_kernel(lambda: mxq.mxfp8_quantize(x), 50, flush))
+        # rotating inputs and outputs: 8 sets of 34 MB in, 17 MB out (> 2x L2),
+        # so no launch finds its input in L2 and no flush's dirty lines compete
+        xs = [x.clone() for _ in range(8)]
+        qs = [torch.empty((4096, 4096), dtype=torch.uint8, device=device) for _ in range(8)]
+        ss = [torch.empty((4096, 128), dtype=torch.uint8, device=device) for _ in range(8)]
+        L = mxq.lib
+        sp = ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+        P = [[ctypes.c_void_p(t.data_ptr()) for t in (xs[i], qs[i], ss[i])] for i in range(8)]
+        k = [0]
+
+        def rotating():
+            p = P[k[0] % 8]
+            k[0] += 1
+            L.mxfp8_quantize(p[0], 0, 4096, 4096, 4096, p[1], p[2], None, sp)
+
+        emit("mxfp8_quantize linear_weight 4096x4096 (8 rotating input/output sets)",
+             mxfp8_quant_bytes(4096, 4096, swizzled=False), time_kernel(rotating, 48))
 
     def activation():
         x = bf(W.activation())
@@ -567,6 +587,23 @@ def run_suite(device, only=None):
                           "tflops": flops / med / 1e9,
                           "frac_of_fp8_peak": flops / med / 1e9 / bf16_peak[0],
                           "fp8_peak_tflops": bf16_peak[0], "peak_kind": bf16_peak[1]}), flush=True)
+        # context: NVIDIA's library MX GEMM (through torch) on the same codes and scales
+        F = torch.nn.functional
+        try:
+            lib_mm = lambda: F.scaled_mm(
+                qa.view(torch.float8_e4m3fn), qb.view(torch.float8_e4m3fn).t(),
+                za.view(torch.float8_e8m0fnu), F.ScalingType.BlockWise1x32,
+                zb.view(torch.float8_e8m0fnu), F.ScalingType.BlockWise1x32,
+                swizzle_a=F.SwizzleType.SWIZZLE_32_4_4, swizzle_b=F.SwizzleType.SWIZZLE_32_4_4,
+                output_dtype=torch.bfloat16)
+            med, p10, p90 = time_kernel(lib_mm, 20)
+            print(json.dumps({"suite": "library MX GEMM (torch scaled_mm, same operands), for context",
+                              "median_us": med * 1e3, "p10_us": p10 * 1e3, "p90_us": p90 * 1e3,
+                              "tflops": flops / med / 1e9,
+                              "frac_of_fp8_peak": flops / med / 1e9 / bf16_peak[0]}), flush=True)
+        except Exception as e:  # not every torch build exposes the MX recipe
+            print(json.dumps({"suite": "library MX GEMM (torch scaled_mm)", "unavailable": str(e)[:200]}),
+                  flush=True)
 
     def experts():
         x = bf(W.experts())

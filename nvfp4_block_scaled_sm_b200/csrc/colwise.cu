@@ -303,12 +303,7 @@ mxfp8_colwise_kernel(const __grid_constant__ ColArgs a) {
 template <typename InT, bool ROW>
 mxq_status launch_colwise(const ColArgs& a, uint32_t grid, cudaStream_t s) {
   constexpr uint32_t kSmem = ROW ? kFusedSmem : kColSmem;
-  static std::once_flag once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(once, [] {
-    attr_err = cudaFuncSetAttribute(mxfp8_colwise_kernel<InT, ROW>,
-                                    cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmem));
-  });
+  const cudaError_t attr_err = ensure_smem_limit<mxfp8_colwise_kernel<InT, ROW>>(int(kSmem));
   if (attr_err != cudaSuccess) {
     record_cuda_error(attr_err);
     return MXQ_ERR_CUDA;

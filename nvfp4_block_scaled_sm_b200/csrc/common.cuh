@@ -12,6 +12,7 @@
 #include <cuda_runtime.h>
 #include <algorithm>
 #include <cstring>
+#include <atomic>
 #include <mutex>
 #include <utility>
 
@@ -418,6 +419,21 @@ template <typename... KArgs, typename... Args>
 inline cudaError_t launch_pdl(void (*kernel)(KArgs...), uint32_t grid, cudaStream_t stream,
                               Args&&... args) {
   return launch_pdl_ex(kernel, grid, kThreads, 0, stream, std::forward<Args>(args)...);
+}
+
+// Raises Kernel's dynamic shared memory limit to `bytes` on the current
+// device, the first time a call reaches it there (the attribute belongs to the
+// device's context, so each device needs its own call).
+template <auto Kernel>
+inline cudaError_t ensure_smem_limit(int bytes) {
+  static std::atomic<unsigned char> done[256];
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev >= 0 && dev < 256 && done[dev].load(std::memory_order_acquire)) return cudaSuccess;
+  e = cudaFuncSetAttribute(Kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && dev >= 0 && dev < 256) done[dev].store(1, std::memory_order_release);
+  return e;
 }
 
 // Multiprocessors of the current device (148 on B200 if the query fails).

@@ -360,12 +360,7 @@ template <typename OutT, int BN>
 mxq_status launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const GemmArgs& args,
                        cudaStream_t s) {
   constexpr uint32_t kSmemBytes = GemmCfg<BN>::kSmemBytes;
-  static std::once_flag once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(once, [] {
-    attr_err = cudaFuncSetAttribute(mxfp8_gemm_kernel<OutT, BN>,
-                                    cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmemBytes));
-  });
+  const cudaError_t attr_err = ensure_smem_limit<mxfp8_gemm_kernel<OutT, BN>>(int(kSmemBytes));
   if (attr_err != cudaSuccess) {
     record_cuda_error(attr_err);
     return MXQ_ERR_CUDA;
