@@ -55,7 +55,7 @@ namespace {
 constexpr int kMaxPartials = 2048;  // CTAs of the amax pass (workspace floats)
 constexpr int kAmaxSteps = 2;       // 16-element bf16 chunks per thread per iteration (fp32: 1)
 constexpr int kAmaxCtasPerSm = 8;   // one resident wave: grid = SMs x 8
-constexpr int kSteps = 2;
+constexpr int kSteps = 4;
 constexpr int kBlocksPerWarp = 32 * kSteps;
 constexpr int kBlocksPerTile = kBlocksPerWarp * (kThreads / 32);
 constexpr int kDqSteps = 2;  // dequantize: blocks per lane
