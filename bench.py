@@ -336,7 +336,10 @@ def run(args):
     # Per-kernel durations come from events around the two kernels of every
     # SAMPLE_EVERY-th step only: an event recorded between two kernels ends
     # their programmatic overlap, so events on every step would slow the step.
-    sampled = [k for k in range(K) if k % SAMPLE_EVERY == SAMPLE_EVERY - 1] or [K - 1]
+    # A short run samples more often (every step at K < 16) so that the
+    # average still rests on about eight launches or more.
+    every = min(SAMPLE_EVERY, max(1, K // 8))
+    sampled = [k for k in range(K) if k % every == every - 1] or [K - 1]
     ev = {k: [torch.cuda.Event(enable_timing=True) for _ in range(3)] for k in sampled}
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if world > 1:
@@ -442,7 +445,7 @@ def run(args):
                 "ms_per_step": e2e_ms, "steps": e2e_steps,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": 2 * K,
-        "kernel_time_sampling": f"events around both kernels on every {SAMPLE_EVERY}th step "
+        "kernel_time_sampling": f"events around both kernels on every {every}th step "
                                 f"({len(sampled)} of {K} steps)",
         "clocks": clk.summary(),
     }

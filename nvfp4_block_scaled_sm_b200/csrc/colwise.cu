@@ -2,7 +2,7 @@
 // one column, the operand layout of a backward GEMM), optionally fused with
 // the rowwise quantize so that the input is read once, for sm_100a.
 //
-// Method: each column group is quantized by the rowwise rule of mxfp8.cu
+// Method: each column group is quantized by the rowwise rule of mx_rowwise.cu
 // (NaN-ignoring amax, E8M0 byte = 127 / 254 / clamp(E(amax) - 8, 0, 254),
 // E4M3 RNE with saturation). Following the adapter contract of "PR #1935
 // 完整报告 -- Use TransformerEngine for MXFP8 quantization" (实现拆解 item 1:
@@ -89,8 +89,15 @@ struct ColArgs {
   bool scale_words;      // scale_t 4-byte aligned and ceil(M/32) % 4 == 0
 };
 
-// 32 E4M3 codes (as two 16-byte halves) of one column of 32 values given as
-// fp32, times the power-of-two multiplier `mul`.
+// Sixteen code pairs (first code in the low byte) as two 16-byte halves.
+__device__ __forceinline__ void pack_codes(const uint32_t (&c)[16], uint4& lo, uint4& hi) {
+  lo = make_uint4(__byte_perm(c[0], c[1], 0x5410), __byte_perm(c[2], c[3], 0x5410),
+                  __byte_perm(c[4], c[5], 0x5410), __byte_perm(c[6], c[7], 0x5410));
+  hi = make_uint4(__byte_perm(c[8], c[9], 0x5410), __byte_perm(c[10], c[11], 0x5410),
+                  __byte_perm(c[12], c[13], 0x5410), __byte_perm(c[14], c[15], 0x5410));
+}
+
+// 32 E4M3 codes of 32 fp32 values times the power-of-two multiplier `mul`.
 __device__ __forceinline__ void column_codes(const float (&f)[32], float mul, uint4& lo, uint4& hi) {
   uint32_t c[16];
 #pragma unroll
@@ -98,10 +105,32 @@ __device__ __forceinline__ void column_codes(const float (&f)[32], float mul, ui
     const float2 p = mul2(f[2 * k], f[2 * k + 1], mul);
     c[k] = cvt_e4m3x2(p.x, p.y);
   }
-  lo = make_uint4(__byte_perm(c[0], c[1], 0x5410), __byte_perm(c[2], c[3], 0x5410),
-                  __byte_perm(c[4], c[5], 0x5410), __byte_perm(c[6], c[7], 0x5410));
-  hi = make_uint4(__byte_perm(c[8], c[9], 0x5410), __byte_perm(c[10], c[11], 0x5410),
-                  __byte_perm(c[12], c[13], 0x5410), __byte_perm(c[14], c[15], 0x5410));
+  pack_codes(c, lo, hi);
+}
+
+// 32 E4M3 codes of 32 consecutive bf16 elements of a row (16 packed words)
+// times the power of two `mul`.
+__device__ __forceinline__ void row_codes_bf16(const uint32_t (&w)[16], float mul, uint4& lo, uint4& hi) {
+  uint32_t c[16];
+#pragma unroll
+  for (int k = 0; k < 16; k++) {
+    const float2 p = mul_bf16x2_pow2(w[k], mul);
+    c[k] = cvt_e4m3x2(p.x, p.y);
+  }
+  pack_codes(c, lo, hi);
+}
+
+// 32 E4M3 codes of one bf16 column: half H of the words v[0..31] (one word
+// per row) times the power of two `mul`.
+template <int H>
+__device__ __forceinline__ void column_codes_bf16(const uint32_t (&v)[32], float mul, uint4& lo, uint4& hi) {
+  uint32_t c[16];
+#pragma unroll
+  for (int k = 0; k < 16; k++) {
+    const float2 p = mul_bf16_pow2<H, H>(v[2 * k], v[2 * k + 1], mul);
+    c[k] = cvt_e4m3x2(p.x, p.y);
+  }
+  pack_codes(c, lo, hi);
 }
 
 template <typename InT, bool ROW>
@@ -159,8 +188,8 @@ mxfp8_colwise_kernel(const __grid_constant__ ColArgs a) {
         const int k = (t >> 7) * kPerThread + j;
         if (r < rows && k * 32 * kEsize < row_bytes) {
           const uint8_t* src = in + r * kPitch + k * 32 * kEsize;
-          float f[32];
-          float amax;
+          uint32_t b;
+          uint4 lo, hi;
           if constexpr (kEsize == 2) {
             uint32_t w[16];
 #pragma unroll
@@ -172,14 +201,11 @@ mxfp8_colwise_kernel(const __grid_constant__ ColArgs a) {
 #pragma unroll
             for (int i = 2; i < 16; i++) m = absmax_bf16x2(m, w[i]);
             m &= 0x7fff7fffu;
-            amax = fmaxf(fmaxf(bf16_lo(m), bf16_hi(m)), 0.0f);
-#pragma unroll
-            for (int i = 0; i < 16; i++) {
-              f[2 * i] = bf16_lo(w[i]);
-              f[2 * i + 1] = bf16_hi(w[i]);
-            }
+            b = mx_scale_byte<8>(fmaxf(fmaxf(bf16_lo(m), bf16_hi(m)), 0.0f));
+            row_codes_bf16(w, pow2_quant(b), lo, hi);
           } else {
-            amax = 0.0f;
+            float f[32];
+            float amax = 0.0f;
 #pragma unroll
             for (int i = 0; i < 8; i++) {
               const uint4 q4 = lds128(src + 16 * i);
@@ -188,10 +214,9 @@ mxfp8_colwise_kernel(const __grid_constant__ ColArgs a) {
             }
 #pragma unroll
             for (int i = 0; i < 32; i++) amax = fmaxf(amax, fabsf(f[i]));
+            b = mx_scale_byte<8>(amax);
+            column_codes(f, pow2_quant(b), lo, hi);
           }
-          const uint32_t b = mx_scale_byte<8>(amax);
-          uint4 lo, hi;
-          column_codes(f, pow2_quant(b), lo, hi);
           sts128(qr + r * kRowPitch + 32 * k, lo);
           sts128(qr + r * kRowPitch + 32 * k + 16, hi);
           sr[4 * r + k] = uint8_t(b);
@@ -209,7 +234,6 @@ mxfp8_colwise_kernel(const __grid_constant__ ColArgs a) {
         uint32_t v[32];
 #pragma unroll
         for (int i = 0; i < 32; i++) v[i] = lds32(in + (32 * g + i) * kPitch + 4 * w);
-        float f[32];
         if constexpr (kEsize == 2) {
           uint32_t m = absmax_bf16x2(v[0], v[1]);
 #pragma unroll
@@ -217,13 +241,10 @@ mxfp8_colwise_kernel(const __grid_constant__ ColArgs a) {
           m &= 0x7fff7fffu;
           sb[0] = mx_scale_byte<8>(fmaxf(bf16_lo(m), 0.0f));
           sb[1] = mx_scale_byte<8>(fmaxf(bf16_hi(m), 0.0f));
-#pragma unroll
-          for (int i = 0; i < 32; i++) f[i] = bf16_lo(v[i]);
-          column_codes(f, pow2_quant(sb[0]), code[0], code[1]);
-#pragma unroll
-          for (int i = 0; i < 32; i++) f[i] = bf16_hi(v[i]);
-          column_codes(f, pow2_quant(sb[1]), code[2], code[3]);
+          column_codes_bf16<0>(v, pow2_quant(sb[0]), code[0], code[1]);
+          column_codes_bf16<1>(v, pow2_quant(sb[1]), code[2], code[3]);
         } else {
+          float f[32];
           float amax = 0.0f;
 #pragma unroll
           for (int i = 0; i < 32; i++) {

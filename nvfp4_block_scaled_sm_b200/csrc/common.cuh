@@ -161,6 +161,40 @@ __device__ __forceinline__ float2 mul2(float a0, float a1, float b) {
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
 
+// (x0 * m, x1 * m) for bf16 elements x0 (selected half SA of word a) and x1
+// (half SB of word b) and a power of two m whose fp32 bit pattern has a zero
+// low half (every MX multiplier 2^(127 - byte), the subnormal 2^-127
+// included, is also a bf16). sm_100 mixed-precision fma: the bf16 product is
+// formed exactly and rounded once to fp32, which makes it equal to the fp32
+// product of the widened operands; the addend is -0 so that a zero product
+// keeps its sign. Saves widening each bf16 element first.
+template <int SA, int SB>
+__device__ __forceinline__ float2 mul_bf16_pow2(uint32_t a, uint32_t b, float m) {
+  const uint32_t mb = __float_as_uint(m) >> 16;
+  float r0, r1;
+  if constexpr (SA == 0 && SB == 0)
+    asm("{ .reg .b16 a0, a1, b0, b1, s, z; mov.b32 {a0, a1}, %2; mov.b32 {b0, b1}, %3;\n\t"
+        "mov.b32 {s, z}, %4; fma.rn.f32.bf16 %0, a0, s, 0f80000000;\n\t"
+        "fma.rn.f32.bf16 %1, b0, s, 0f80000000; }"
+        : "=f"(r0), "=f"(r1) : "r"(a), "r"(b), "r"(mb));
+  else if constexpr (SA == 1 && SB == 1)
+    asm("{ .reg .b16 a0, a1, b0, b1, s, z; mov.b32 {a0, a1}, %2; mov.b32 {b0, b1}, %3;\n\t"
+        "mov.b32 {s, z}, %4; fma.rn.f32.bf16 %0, a1, s, 0f80000000;\n\t"
+        "fma.rn.f32.bf16 %1, b1, s, 0f80000000; }"
+        : "=f"(r0), "=f"(r1) : "r"(a), "r"(b), "r"(mb));
+  else
+    asm("{ .reg .b16 a0, a1, b0, b1, s, z; mov.b32 {a0, a1}, %2; mov.b32 {b0, b1}, %3;\n\t"
+        "mov.b32 {s, z}, %4; fma.rn.f32.bf16 %0, a0, s, 0f80000000;\n\t"
+        "fma.rn.f32.bf16 %1, b1, s, 0f80000000; }"
+        : "=f"(r0), "=f"(r1) : "r"(a), "r"(b), "r"(mb));
+  return make_float2(r0, r1);
+}
+
+// Both bf16 elements of one word times the power of two m (as above).
+__device__ __forceinline__ float2 mul_bf16x2_pow2(uint32_t w, float m) {
+  return mul_bf16_pow2<0, 1>(w, w, m);
+}
+
 // Two fp32 -> E4M3 codes (round to nearest even, |v| > 448 -> 448, NaN ->
 // NaN); `lo` lands in the low byte.
 __device__ __forceinline__ uint32_t cvt_e4m3x2(float lo, float hi) {
@@ -339,6 +373,8 @@ struct In16<uint16_t> {
   }
   __device__ __forceinline__ float lo(int k) const { return bf16_lo(w[k]); }  // element 2k
   __device__ __forceinline__ float hi(int k) const { return bf16_hi(w[k]); }  // element 2k+1
+  // (element 2k, element 2k+1) times a power of two m, in fp32
+  __device__ __forceinline__ float2 scaled(int k, float m) const { return mul_bf16x2_pow2(w[k], m); }
   __device__ __forceinline__ uint32_t signs() const {  // bit i = sign of element i
     uint32_t r = 0;
 #pragma unroll
@@ -377,6 +413,7 @@ struct In16<float> {
   }
   __device__ __forceinline__ float lo(int k) const { return __uint_as_float(w[2 * k]); }
   __device__ __forceinline__ float hi(int k) const { return __uint_as_float(w[2 * k + 1]); }
+  __device__ __forceinline__ float2 scaled(int k, float m) const { return mul2(lo(k), hi(k), m); }
   __device__ __forceinline__ uint32_t signs() const {
     uint32_t r = 0;
 #pragma unroll

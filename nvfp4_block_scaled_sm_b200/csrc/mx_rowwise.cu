@@ -67,7 +67,7 @@ __device__ __forceinline__ uint4 to_e4m3(const In16<InT>& v, float mul) {
   uint32_t c[8];
 #pragma unroll
   for (int k = 0; k < 8; k++) {
-    const float2 p = mul2(v.lo(k), v.hi(k), mul);
+    const float2 p = v.scaled(k, mul);
     c[k] = cvt_e4m3x2(p.x, p.y);
   }
   return make_uint4(__byte_perm(c[0], c[1], 0x5410), __byte_perm(c[2], c[3], 0x5410),
@@ -81,7 +81,7 @@ __device__ __forceinline__ uint2 to_e2m1(const In16<InT>& v, float mul) {
   uint32_t c[8];
 #pragma unroll
   for (int k = 0; k < 8; k++) {
-    const float2 p = mul2(v.lo(k), v.hi(k), mul);
+    const float2 p = v.scaled(k, mul);
     c[k] = cvt_e2m1x2(p.x, p.y);
   }
   return make_uint2(c[0] | (c[1] << 8) | (c[2] << 16) | (c[3] << 24),
