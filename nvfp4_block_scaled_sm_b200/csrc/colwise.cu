@@ -87,7 +87,23 @@ struct ColArgs {
   uint8_t* scale;        // [M, N / 32] (fused mode)
   bool q_t_aligned;      // every q_t row start is 16-byte aligned (M % 16 == 0)
   bool scale_words;      // scale_t 4-byte aligned and ceil(M/32) % 4 == 0
+  bool row_scale_words;  // fused mode: scale 4-byte aligned and (N / 32) % 4 == 0
 };
+
+// max.xorsign.abs over N bf16 pairs as a pairwise tree (depth log2 N rather
+// than a chain of N - 1 dependent maxima); the result's sign bits are junk.
+template <int N>
+__device__ __forceinline__ uint32_t absmax_tree(const uint32_t (&v)[N]) {
+  uint32_t m[N / 2];
+#pragma unroll
+  for (int i = 0; i < N / 2; i++) m[i] = absmax_bf16x2(v[2 * i], v[2 * i + 1]);
+#pragma unroll
+  for (int n = N / 4; n >= 1; n /= 2) {
+#pragma unroll
+    for (int i = 0; i < n; i++) m[i] = absmax_bf16x2(m[2 * i], m[2 * i + 1]);
+  }
+  return m[0];
+}
 
 // Sixteen code pairs (first code in the low byte) as two 16-byte halves.
 __device__ __forceinline__ void pack_codes(const uint32_t (&c)[16], uint4& lo, uint4& hi) {
@@ -197,10 +213,7 @@ mxfp8_colwise_kernel(const __grid_constant__ ColArgs a) {
               const uint4 q4 = lds128(src + 16 * i);
               w[4 * i] = q4.x; w[4 * i + 1] = q4.y; w[4 * i + 2] = q4.z; w[4 * i + 3] = q4.w;
             }
-            uint32_t m = absmax_bf16x2(w[0], w[1]);
-#pragma unroll
-            for (int i = 2; i < 16; i++) m = absmax_bf16x2(m, w[i]);
-            m &= 0x7fff7fffu;
+            const uint32_t m = absmax_tree(w) & 0x7fff7fffu;
             b = mx_scale_byte<8>(fmaxf(fmaxf(bf16_lo(m), bf16_hi(m)), 0.0f));
             row_codes_bf16(w, pow2_quant(b), lo, hi);
           } else {
@@ -235,10 +248,7 @@ mxfp8_colwise_kernel(const __grid_constant__ ColArgs a) {
 #pragma unroll
         for (int i = 0; i < 32; i++) v[i] = lds32(in + (32 * g + i) * kPitch + 4 * w);
         if constexpr (kEsize == 2) {
-          uint32_t m = absmax_bf16x2(v[0], v[1]);
-#pragma unroll
-          for (int i = 2; i < 32; i++) m = absmax_bf16x2(m, v[i]);
-          m &= 0x7fff7fffu;
+          const uint32_t m = absmax_tree(v) & 0x7fff7fffu;
           sb[0] = mx_scale_byte<8>(fmaxf(bf16_lo(m), 0.0f));
           sb[1] = mx_scale_byte<8>(fmaxf(bf16_hi(m), 0.0f));
           column_codes_bf16<0>(v, pow2_quant(sb[0]), code[0], code[1]);
@@ -311,11 +321,14 @@ mxfp8_colwise_kernel(const __grid_constant__ ColArgs a) {
           st_v4(a.q + (r0 + r) * a.N + c0 + 16 * ch, lds128(qr + r * kRowPitch + 16 * ch));
       }
       if (t < rows) {
-        constexpr int kGroups = kTileCols / 32;
+        constexpr int kGroups = kTileCols / 32;  // 4 (bf16) or 2 (fp32)
         const int ng = row_bytes / kEsize / 32;
         uint8_t* dst = a.scale + (r0 + t) * S + c0 / 32;
-        for (int j = 0; j < ng; j++) st_u8(dst + j, sr[4 * t + j]);
-        (void)kGroups;
+        if (kGroups == 4 && ng == 4 && a.row_scale_words) {
+          st_u32(dst, *reinterpret_cast<const uint32_t*>(sr + 4 * t));
+        } else {
+          for (int j = 0; j < ng; j++) st_u8(dst + j, sr[4 * t + j]);
+        }
       }
     }
   }
@@ -368,6 +381,7 @@ extern "C" mxq_status mxfp8_quantize_columnwise(const void* x, int dt, int64_t M
   a.scale = scale;
   a.q_t_aligned = (M % 16) == 0;
   a.scale_words = (reinterpret_cast<uintptr_t>(scale_t) & 3u) == 0 && (a.gt & 3u) == 0;
+  a.row_scale_words = (reinterpret_cast<uintptr_t>(scale) & 3u) == 0 && ((N / 32) & 3) == 0;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const uint64_t resident = uint64_t(sm_count()) * 2;
   const uint32_t grid = uint32_t(a.ntiles < resident ? a.ntiles : resident);
