@@ -52,6 +52,9 @@ constexpr int kEpilogueWarps = 4;
 constexpr int kGemmThreads = 32 * (2 + kEpilogueWarps);  // producer, MMA, epilogue warps
 constexpr uint32_t kSfTile = 512;    // one 128 x 4 scale tile
 constexpr uint32_t kBarBytes = 256;
+// bf16 epilogue staging per warp: 32 rows x 64 columns (128 bytes), pitch 144
+constexpr uint32_t kEpiPitch = 144;
+constexpr uint32_t kEpiStageBytes = 32 * kEpiPitch;
 constexpr uint64_t kWaitNs = 1000000000ull;  // one second
 
 template <int BN>
@@ -64,7 +67,8 @@ struct GemmCfg {
       (kTileA + kTileB + kSfTile * (1 + kSfbTiles) + 1023u) & ~1023u;
   static constexpr uint32_t kSfColsPerStage = 4 * (1 + kSfbTiles);
   static constexpr uint32_t kTmemCols = BN + kStages * kSfColsPerStage <= 256 ? 256 : 512;
-  static constexpr uint32_t kSmemBytes = kStages * kStageBytes + kBarBytes + 1024;  // + alignment slack
+  static constexpr uint32_t kSmemBytes =
+      kStages * kStageBytes + kBarBytes + kEpiStageBytes * kEpilogueWarps + 1024;  // + alignment slack
   static_assert(BN + kStages * kSfColsPerStage <= 512, "tensor memory");
   static_assert(kSmemBytes <= 232448, "shared memory");
 };
@@ -152,6 +156,21 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
+__device__ __forceinline__ void sts128_u32(uint32_t addr, uint4 v) {
+  asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z),
+               "r"(v.w)
+               : "memory");
+}
+
+__device__ __forceinline__ uint4 lds128_u32(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(addr)
+               : "memory");
+  return v;
+}
+
 __device__ __forceinline__ void record_error(int32_t* err, int32_t code) {
   if (err) atomicCAS(err, 0, code);
 }
@@ -177,6 +196,8 @@ mxfp8_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_consta
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kStages * kStageBytes + 8 * (2 * kStages + 2));
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // bf16 epilogue staging rows of this warp (epilogue warps only)
+  const uint32_t epi = bars + kBarBytes + kEpiStageBytes * uint32_t(warp >= 2 ? warp - 2 : 0);
   const uint32_t n_my = (a.ntiles - blockIdx.x + gridDim.x - 1) / gridDim.x;  // grid <= tiles
 
   if (warp == 0) {
@@ -287,34 +308,57 @@ mxfp8_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_consta
       }
       tc_fence_after();
       const uint32_t row = m_blk * kBM + quarter * 32 + lane;
-      OutT* drow = static_cast<OutT*>(a.d) + uint64_t(row) * a.N + uint64_t(n_blk) * BN;
       const uint32_t ncols = min(uint32_t(BN), a.N - n_blk * BN);
-#pragma unroll 1
-      for (uint32_t c0 = 0; c0 < uint32_t(BN); c0 += 32) {
-        uint32_t r[32];
-        tmem_ld32(taddr + c0, r);  // every lane of the warp takes part
-        if (c0 + 32 >= uint32_t(BN)) {
-          // the whole accumulator is in registers: hand it back to the MMA
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(acc_empty);
-        }
-        if (row >= a.M || c0 >= ncols) continue;
-        if constexpr (sizeof(OutT) == 2) {
-          uint32_t w[16];
+      if constexpr (sizeof(OutT) == 2) {
+        // the whole row of the accumulator into registers as bf16 pairs, the
+        // accumulator handed back, then the stores
+        uint32_t w[BN / 2];
+#pragma unroll
+        for (uint32_t c0 = 0; c0 < uint32_t(BN); c0 += 32) {
+          uint32_t r[32];
+          tmem_ld32(taddr + c0, r);
 #pragma unroll
           for (int q = 0; q < 16; q++)
-            w[q] = cvt_bf16x2(__uint_as_float(r[2 * q]), __uint_as_float(r[2 * q + 1]));
-          if (c0 + 32 <= ncols) {
+            w[c0 / 2 + q] = cvt_bf16x2(__uint_as_float(r[2 * q]), __uint_as_float(r[2 * q + 1]));
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(acc_empty);
+        // 64-column slices through this warp's staging rows, so that each
+        // store instruction writes four rows' 128-byte segments
+        const uint32_t row0 = m_blk * kBM + quarter * 32;
+        const uint32_t rsub = lane >> 3, ch = lane & 7;
 #pragma unroll
-            for (int q = 0; q < 4; q++)
-              st_v4(drow + c0 + 8 * q, make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]));
-          } else {
+        for (uint32_t c0 = 0; c0 < uint32_t(BN); c0 += 64) {
 #pragma unroll
-            for (uint32_t q = 0; q < 16; q++)
-              if (c0 + 2 * q < ncols) st_u32(drow + c0 + 2 * q, w[q]);
+          for (int q = 0; q < 8; q++)
+            sts128_u32(epi + lane * kEpiPitch + 16 * q,
+                       make_uint4(w[c0 / 2 + 4 * q], w[c0 / 2 + 4 * q + 1], w[c0 / 2 + 4 * q + 2],
+                                  w[c0 / 2 + 4 * q + 3]));
+          __syncwarp();
+          const uint32_t col = c0 + 8 * ch;  // first of this lane's 8 columns
+#pragma unroll
+          for (uint32_t i = 0; i < 8; i++) {
+            const uint32_t rr = 4 * i + rsub;
+            const uint4 v = lds128_u32(epi + rr * kEpiPitch + 16 * ch);
+            if (row0 + rr < a.M && col < ncols)
+              st_v4(static_cast<OutT*>(a.d) + uint64_t(row0 + rr) * a.N + uint64_t(n_blk) * BN + col, v);
           }
-        } else {
+          __syncwarp();
+        }
+      } else {
+        OutT* drow = static_cast<OutT*>(a.d) + uint64_t(row) * a.N + uint64_t(n_blk) * BN;
+#pragma unroll 1
+        for (uint32_t c0 = 0; c0 < uint32_t(BN); c0 += 32) {
+          uint32_t r[32];
+          tmem_ld32(taddr + c0, r);  // every lane of the warp takes part
+          if (c0 + 32 >= uint32_t(BN)) {
+            // the whole accumulator is in registers: hand it back to the MMA
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(acc_empty);
+          }
+          if (row >= a.M || c0 >= ncols) continue;
           if (c0 + 32 <= ncols) {
 #pragma unroll
             for (int q = 0; q < 8; q++)
