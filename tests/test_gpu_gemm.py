@@ -76,6 +76,22 @@ def test_power_of_two_grid_is_exact(M, N, K):
     assert not bad.any(), f"{int(bad.sum())} of {bad.size} differ; first {np.argwhere(bad)[:4].tolist()}"
 
 
+@pytest.mark.parametrize("M,N,K", [(128, 256, 128), (33, 48, 96), (1, 16, 32), (300, 272, 160),
+                                   (129, 400, 224), (3000, 3008, 96)])
+def test_power_of_two_grid_bf16_is_rounded_exact(M, N, K):
+    """bf16 output on the power-of-two grid: the fp32 sum is exact there, so
+    each output must be that value rounded to nearest even bf16 (the
+    epilogue's row and column edges included)."""
+    xa = W.gemm_pow2_operand(3000 + M, M, K)
+    xb = W.gemm_pow2_operand(4000 + N, N, K)
+    d = run(xa, xb, torch.bfloat16)
+    exact, _ = oracle_product(xa, xb)
+    want = torch.from_numpy(exact.astype(np.float32)).to(torch.bfloat16).view(torch.int16).numpy()
+    got = d.view(torch.int16).cpu().numpy()
+    bad = got != want
+    assert not bad.any(), f"{int(bad.sum())} of {bad.size} differ; first {np.argwhere(bad)[:4].tolist()}"
+
+
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
 def test_activation_times_weight(dtype):
     xa = W.activation(seed=105, M=512, N=2048)
