@@ -15,8 +15,13 @@
 // TransformerEngine for MXFP8 quantization" (the quantized weights feed the
 // GEMM); the scale-tile layout is the one the block-scaled MMA reads.
 //
-// Structure: persistent CTAs (one per multiprocessor) walk 128 x BN output
-// tiles (BN = 256, or 128 when N <= 128) with six warps:
+// Two kernels. When M and N both exceed 128, CTA pairs (clusters of two, one
+// CTA per SM) walk 256 x 256 output tiles with the pair form of the MMA; it is
+// described with mxfp8_gemm_pair_kernel below. Otherwise the single-CTA
+// kernel runs.
+//
+// Single-CTA structure: persistent CTAs (one per multiprocessor) walk
+// 128 x BN output tiles (BN = 256, or 128 when N <= 128) with six warps:
 //  - warp 0, one lane: producer. Per K block of 128: TMA loads of the A tile
 //    (128 rows x 128 bytes) and the B tile (BN rows x 128 bytes), both with
 //    the 128-byte swizzle, and bulk copies of the 512-byte scale tiles (one
@@ -383,6 +388,295 @@ mxfp8_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_consta
   }
 }
 
+// ------------------------------------------------------ CTA-pair kernel
+//
+// Two CTAs of a cluster (one per SM) share one 256 x 256 output tile through
+// the pair form of the block-scaled MMA (tcgen05.mma.cta_group::2, M = 256):
+// CTA r of the pair holds A rows 128 r .. 128 r + 127 of the tile and B rows
+// 128 r .. 128 r + 127, and the MMA, issued by the even CTA, reads B from
+// both. Each CTA therefore loads 32 KiB of operands per K block for the work
+// that takes 48 KiB in the single-CTA kernel, and six stages fit. Scales: each
+// CTA holds its own A scale tile and both B scale tiles of the pair tile in
+// shared memory; the even CTA copies them into both CTAs' tensor memory
+// (tcgen05.cp.cta_group::2). Every TMA load of both CTAs completes on the even
+// CTA's "full" barrier; the even CTA's commits arrive on the "empty" and
+// "acc_full" barriers of both CTAs; both CTAs' epilogue warps arrive on the
+// even CTA's "acc_empty". Each CTA's accumulator (its 128 rows x 256 columns)
+// is in its own tensor memory and is written out by its own epilogue warps.
+
+constexpr int kPairStages = 6;
+constexpr uint32_t kPairTileA = kBM * kBK;                    // 16 KiB: this CTA's A rows
+constexpr uint32_t kPairTileB = 128 * kBK;                    // 16 KiB: this CTA's half of B
+constexpr uint32_t kPairStageBytes =
+    (kPairTileA + kPairTileB + 3 * kSfTile + 1023u) & ~1023u;  // + A scales + both B scale tiles
+constexpr uint32_t kPairStageTx = kPairTileA + kPairTileB + 3 * kSfTile;  // one CTA's bytes
+constexpr uint32_t kPairSfCols = 12;                          // tensor-memory scale columns a stage
+constexpr uint32_t kPairTmemCols = 512;
+constexpr uint32_t kPairSmemBytes =
+    kPairStages * kPairStageBytes + kBarBytes + kEpiStageBytes * kEpilogueWarps + 1024;
+static_assert(256 + kPairStages * kPairSfCols <= kPairTmemCols, "tensor memory");
+static_assert(kPairSmemBytes <= 232448, "shared memory");
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+// All threads of both CTAs of the cluster.
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
+                   : "memory");
+}
+
+// Shared::cluster address of the same shared variable in CTA `rank`.
+__device__ __forceinline__ uint32_t cluster_addr(uint32_t local, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local), "r"(rank));
+  return r;
+}
+
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_bar) {
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar) : "memory");
+}
+
+// TMA load into this CTA's shared memory whose completion is counted on a
+// barrier of the pair (given by its shared::cluster address).
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* map,
+                                                 uint32_t cluster_bar, int32_t x, int32_t y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];"
+      ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(cluster_bar), "r"(x), "r"(y)
+      : "memory");
+}
+
+__device__ __forceinline__ void mma_mxf8_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                              uint32_t idesc, uint32_t sfa_tmem, uint32_t sfb_tmem,
+                                              uint32_t accumulate) {
+  asm volatile(
+      "{ .reg .pred p; setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p; }"
+      ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_copy_scales_pair(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
+// Arrives on the barrier at this shared offset in both CTAs of the pair once
+// the MMAs issued so far have completed.
+__device__ __forceinline__ void mma_commit_pair(uint32_t bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;"
+      ::"r"(bar), "h"(uint16_t(3))
+      : "memory");
+}
+
+// Instruction descriptor as instr_desc<256> but for the pair's M = 256.
+__device__ __forceinline__ uint32_t instr_desc_pair(uint32_t k) {
+  return (k << 4) | (uint32_t(256 >> 3) << 17) | (1u << 23) | (uint32_t(256 >> 4) << 24) | (k << 29);
+}
+
+template <typename OutT>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
+mxfp8_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_b,
+                       const __grid_constant__ CUtensorMap tma_sfa,
+                       const __grid_constant__ CUtensorMap tma_sfb, const __grid_constant__ GemmArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* smem = smem_raw + (base - raw);
+  const uint32_t bars = base + kPairStages * kPairStageBytes;
+  auto full_bar = [&](int s) { return bars + 8u * s; };
+  auto empty_bar = [&](int s) { return bars + 8u * (kPairStages + s); };
+  const uint32_t acc_full = bars + 8u * (2 * kPairStages);
+  const uint32_t acc_empty = acc_full + 8u;
+  uint32_t* tmem_slot =
+      reinterpret_cast<uint32_t*>(smem + kPairStages * kPairStageBytes + 8 * (2 * kPairStages + 2));
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();  // 0: issues the MMAs
+  const uint32_t pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+  const uint32_t n_my = (a.ntiles - pair + npairs - 1) / npairs;  // npairs <= tiles
+  const uint32_t epi = bars + kBarBytes + kEpiStageBytes * uint32_t(warp >= 2 ? warp - 2 : 0);
+
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;"
+                 ::"r"(smem_u32(tmem_slot)), "r"(kPairTmemCols) : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+  }
+  if (threadIdx.x == 32) {
+    for (int s = 0; s < kPairStages; s++) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    mbar_init(acc_full, 1);
+    mbar_init(acc_empty, 2 * kEpilogueWarps);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // the peer's barriers are initialised before any remote arrival
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0 && lane == 0) {
+    // ---------------------------------------------------------- producer
+    const uint32_t lead_full0 = cluster_addr(full_bar(0), 0);
+    uint32_t it = 0;
+    bool ok = true;
+    for (uint32_t i = 0; i < n_my && ok; i++) {
+      const uint32_t tile = pair + i * npairs;
+      const uint32_t m_blk = tile / a.n_tiles_n, n_blk = tile % a.n_tiles_n;
+      const int32_t a_row = int32_t(m_blk * 256 + 128 * rank);
+      const int32_t b_row = int32_t(n_blk * 256 + 128 * rank);
+      // rows of 128 bytes in the scale maps: tile (row block, K block) at 4 (rb kp4 + kb)
+      const uint32_t sfa_rb = m_blk * 2 + rank, sfb_rb = n_blk * 2;
+      for (uint32_t kb = 0; kb < a.nk; kb++, it++) {
+        const int s = it % kPairStages;
+        const uint32_t phase = (it / kPairStages) & 1u;
+        if (!mbar_wait(empty_bar(s), phase ^ 1u, kWaitNs)) {
+          record_error(a.err, kErrEmptyWait);
+          ok = false;
+          break;
+        }
+        if (rank == 0) mbar_expect_tx(full_bar(s), 2 * kPairStageTx);
+        const uint32_t bar = lead_full0 + 8u * s;
+        const uint32_t st = base + s * kPairStageBytes;
+        tma_load_2d_pair(st, &tma_a, bar, int32_t(kb * kBK), a_row);
+        tma_load_2d_pair(st + kPairTileA, &tma_b, bar, int32_t(kb * kBK), b_row);
+        const uint32_t sf = st + kPairTileA + kPairTileB;
+        tma_load_2d_pair(sf, &tma_sfa, bar, 0, int32_t(4 * (sfa_rb * a.kp4 + kb)));
+        tma_load_2d_pair(sf + kSfTile, &tma_sfb, bar, 0, int32_t(4 * (sfb_rb * a.kp4 + kb)));
+        tma_load_2d_pair(sf + 2 * kSfTile, &tma_sfb, bar, 0, int32_t(4 * ((sfb_rb + 1) * a.kp4 + kb)));
+      }
+    }
+  } else if (warp == 1 && lane == 0 && rank == 0) {
+    // ------------------------------------------------------- MMA issuer
+    uint32_t it = 0;
+    for (uint32_t i = 0; i < n_my; i++) {
+      if (i > 0 && !mbar_wait(acc_empty, (i - 1) & 1u, kWaitNs)) {
+        record_error(a.err, kErrAccumWait);
+        break;
+      }
+      tc_fence_after();
+      bool ok = true;
+      for (uint32_t kb = 0; kb < a.nk; kb++, it++) {
+        const int s = it % kPairStages;
+        const uint32_t phase = (it / kPairStages) & 1u;
+        if (!mbar_wait(full_bar(s), phase, kWaitNs)) {
+          record_error(a.err, kErrFullWait);
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t st = base + s * kPairStageBytes;
+        const uint32_t sfa_t = tmem + 256 + kPairSfCols * s;
+        const uint32_t sfb_t = sfa_t + 4u;
+        const uint32_t sf = st + kPairTileA + kPairTileB;
+        tmem_copy_scales_pair(sfa_t, scale_desc(sf));
+        tmem_copy_scales_pair(sfb_t, scale_desc(sf + kSfTile));
+        tmem_copy_scales_pair(sfb_t + 4u, scale_desc(sf + 2 * kSfTile));
+#pragma unroll
+        for (uint32_t k = 0; k < 4; k++) {
+          mma_mxf8_pair(tmem, operand_desc(st + 32u * k), operand_desc(st + kPairTileA + 32u * k),
+                        instr_desc_pair(k), sfa_t | (k << 30), sfb_t | (k << 30), (kb | k) != 0u);
+        }
+        mma_commit_pair(empty_bar(s));
+      }
+      if (!ok) break;
+      mma_commit_pair(acc_full);
+    }
+  } else if (warp >= 2) {
+    // ------------------------------------------------------------ epilogue
+    const uint32_t quarter = uint32_t(warp & 3);
+    const uint32_t taddr = tmem + ((quarter * 32) << 16);
+    const uint32_t lead_acc_empty = cluster_addr(acc_empty, 0);
+    for (uint32_t i = 0; i < n_my; i++) {
+      const uint32_t tile = pair + i * npairs;
+      const uint32_t m_blk = tile / a.n_tiles_n, n_blk = tile % a.n_tiles_n;
+      const bool have = __any_sync(0xffffffffu, mbar_wait(acc_full, i & 1u, kWaitNs));
+      if (!have) {
+        if (lane == 0) record_error(a.err, kErrAccumWait);
+        break;
+      }
+      tc_fence_after();
+      const uint32_t row0 = m_blk * 256 + 128 * rank + quarter * 32;
+      const uint32_t ncols = min(256u, a.N - n_blk * 256);
+      if constexpr (sizeof(OutT) == 2) {
+        uint32_t w[128];
+#pragma unroll
+        for (uint32_t c0 = 0; c0 < 256u; c0 += 32) {
+          uint32_t r[32];
+          tmem_ld32(taddr + c0, r);
+#pragma unroll
+          for (int q = 0; q < 16; q++)
+            w[c0 / 2 + q] = cvt_bf16x2(__uint_as_float(r[2 * q]), __uint_as_float(r[2 * q + 1]));
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_remote(lead_acc_empty);
+        const uint32_t rsub = lane >> 3, ch = lane & 7;
+#pragma unroll
+        for (uint32_t c0 = 0; c0 < 256u; c0 += 64) {
+#pragma unroll
+          for (int q = 0; q < 8; q++)
+            sts128_u32(epi + lane * kEpiPitch + 16 * q,
+                       make_uint4(w[c0 / 2 + 4 * q], w[c0 / 2 + 4 * q + 1], w[c0 / 2 + 4 * q + 2],
+                                  w[c0 / 2 + 4 * q + 3]));
+          __syncwarp();
+          const uint32_t col = c0 + 8 * ch;
+#pragma unroll
+          for (uint32_t j = 0; j < 8; j++) {
+            const uint32_t rr = 4 * j + rsub;
+            const uint4 v = lds128_u32(epi + rr * kEpiPitch + 16 * ch);
+            if (row0 + rr < a.M && col < ncols)
+              st_v4(static_cast<OutT*>(a.d) + uint64_t(row0 + rr) * a.N + uint64_t(n_blk) * 256 + col, v);
+          }
+          __syncwarp();
+        }
+      } else {
+        const uint32_t row = row0 + lane;
+        OutT* drow = static_cast<OutT*>(a.d) + uint64_t(row) * a.N + uint64_t(n_blk) * 256;
+#pragma unroll 1
+        for (uint32_t c0 = 0; c0 < 256u; c0 += 32) {
+          uint32_t r[32];
+          tmem_ld32(taddr + c0, r);
+          if (c0 + 32 >= 256u) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_remote(lead_acc_empty);
+          }
+          if (row >= a.M || c0 >= ncols) continue;
+          if (c0 + 32 <= ncols) {
+#pragma unroll
+            for (int q = 0; q < 8; q++)
+              st_v4(drow + c0 + 4 * q, make_uint4(r[4 * q], r[4 * q + 1], r[4 * q + 2], r[4 * q + 3]));
+          } else {
+#pragma unroll
+            for (uint32_t q = 0; q < 32; q++)
+              if (c0 + q < ncols) st_u32(drow + c0 + q, r[q]);
+          }
+        }
+      }
+    }
+  }
+
+  // neither CTA leaves while the other may still reach its shared memory or
+  // tensor memory (barrier arrivals, MMA operand reads, scale copies)
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();
+  if (warp == 0) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kPairTmemCols)
+                 : "memory");
+  }
+}
+
 // ------------------------------------------------------------------ host
 
 // [rows, K] bytes, row stride K, boxes of box_rows rows x 128 bytes,
@@ -398,6 +692,66 @@ bool make_operand_map(CUtensorMap* map, const uint8_t* p, uint64_t rows, uint64_
   return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(p), dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// A swizzled scale array seen as rows of 128 bytes; one load takes a 512-byte
+// 128 x 4 scale tile (4 rows), no swizzle.
+bool make_scale_map(CUtensorMap* map, const uint8_t* p, uint64_t bytes) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {128, bytes / 128};
+  const cuuint64_t strides[1] = {128};
+  const cuuint32_t box[2] = {128, 4};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(p), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+             CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Clusters of two that can be resident at once on the current device (at
+// least one), for the CTA-pair kernel's persistent grid.
+template <typename OutT>
+uint32_t max_pair_clusters() {
+  static std::atomic<int> cached[256];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 256) dev = 0;
+  int n = cached[dev].load(std::memory_order_relaxed);
+  if (n > 0) return uint32_t(n);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * 256);
+  cfg.blockDim = dim3(kGemmThreads);
+  cfg.dynamicSmemBytes = kPairSmemBytes;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int c = 0;
+  if (cudaOccupancyMaxActiveClusters(&c, mxfp8_gemm_pair_kernel<OutT>, &cfg) != cudaSuccess || c <= 0) {
+    (void)cudaGetLastError();
+    c = sm_count() / 2;
+  }
+  cached[dev].store(c, std::memory_order_relaxed);
+  return uint32_t(c);
+}
+
+template <typename OutT>
+mxq_status launch_gemm_pair(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tsa,
+                            const CUtensorMap& tsb, const GemmArgs& args, cudaStream_t s) {
+  const cudaError_t attr_err = ensure_smem_limit<mxfp8_gemm_pair_kernel<OutT>>(int(kPairSmemBytes));
+  if (attr_err != cudaSuccess) {
+    record_cuda_error(attr_err);
+    return MXQ_ERR_CUDA;
+  }
+  GemmArgs a2 = args;
+  a2.n_tiles_n = (args.N + 255) / 256;
+  a2.ntiles = a2.n_tiles_n * ((args.M + 255) / 256);
+  const uint32_t clusters = max_pair_clusters<OutT>();
+  const uint32_t pairs = a2.ntiles < clusters ? a2.ntiles : clusters;
+  mxfp8_gemm_pair_kernel<OutT><<<2 * pairs, kGemmThreads, kPairSmemBytes, s>>>(ta, tb, tsa, tsb, a2);
+  return check_launch();
 }
 
 template <typename OutT, int BN>
@@ -443,12 +797,13 @@ extern "C" mxq_status mxfp8_gemm(const uint8_t* qa, const uint8_t* sa_swz, const
   if (!qa || !qb || !sa_swz || !sb_swz) return MXQ_ERR_NULL;
   if (!aligned16(qa) || !aligned16(qb) || !aligned16(sa_swz) || !aligned16(sb_swz))
     return MXQ_ERR_ALIGN;
-  // 128 x 256 tiles halve the operand traffic per MMA; narrow outputs keep
-  // 128-wide tiles
+  // 256 x 256 tiles over a CTA pair when both sides exceed one 128-row
+  // block; otherwise one CTA per tile, 128 x 256 (128 x 128 when N <= 128)
   const bool wide = N > 128;
-  CUtensorMap ta, tb;
+  const bool paired = wide && M > 128;
+  CUtensorMap ta, tb, tsa, tsb;
   if (!make_operand_map(&ta, qa, uint64_t(M), uint64_t(K), kBM) ||
-      !make_operand_map(&tb, qb, uint64_t(N), uint64_t(K), wide ? 256u : 128u))
+      !make_operand_map(&tb, qb, uint64_t(N), uint64_t(K), (wide && !paired) ? 256u : 128u))
     return MXQ_ERR_CUDA;
   GemmArgs args{};
   args.sfa = sa_swz;
@@ -460,6 +815,14 @@ extern "C" mxq_status mxfp8_gemm(const uint8_t* qa, const uint8_t* sa_swz, const
   args.nk = uint32_t((K + kBK - 1) / kBK);
   args.kp4 = args.nk;
   args.nb128 = uint32_t((N + 127) / 128);
+  if (paired) {
+    const uint64_t sa_bytes = (uint64_t(M) + 127) / 128 * args.kp4 * kSfTile;
+    const uint64_t sb_bytes = (uint64_t(N) + 127) / 128 * args.kp4 * kSfTile;
+    if (!make_scale_map(&tsa, sa_swz, sa_bytes) || !make_scale_map(&tsb, sb_swz, sb_bytes))
+      return MXQ_ERR_CUDA;
+    return out_dt == MXQ_BF16 ? launch_gemm_pair<uint16_t>(ta, tb, tsa, tsb, args, s)
+                              : launch_gemm_pair<float>(ta, tb, tsa, tsb, args, s);
+  }
   if (out_dt == MXQ_BF16)
     return wide ? launch_gemm<uint16_t, 256>(ta, tb, args, s) : launch_gemm<uint16_t, 128>(ta, tb, args, s);
   return wide ? launch_gemm<float, 256>(ta, tb, args, s) : launch_gemm<float, 128>(ta, tb, args, s);
