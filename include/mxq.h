@@ -233,8 +233,10 @@ mxq_status mx_fake_quantize(int fmt, const void* x, int dt, int64_t M, int64_t N
  *          result is then undefined. It is never cleared by the library.
  * K % 32 == 0, N % 16 == 0; all pointers 16-byte aligned. K == 0 writes
  * zeros. One launch of persistent CTAs (at most one per multiprocessor, 192
- * threads, about 200 KB of shared memory each) over 128 x 256 output tiles
- * (128 x 128 when N <= 128). */
+ * threads, about 220 KB of shared memory each): when M > 128 and N > 128,
+ * clusters of two CTAs over 256 x 256 output tiles (the pair form of the
+ * MMA); otherwise single CTAs over 128 x 256 tiles (128 x 128 when
+ * N <= 128). */
 mxq_status mxfp8_gemm(const uint8_t* qa, const uint8_t* sa_swz, const uint8_t* qb,
                       const uint8_t* sb_swz, int64_t M, int64_t N, int64_t K, void* d,
                       int out_dt, int32_t* error_flag, mxq_stream_t stream);
