@@ -10,17 +10,26 @@ needed between steps.
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl mxq|reference]
     python -m torch.distributed.run --nproc-per-node N bench.py --gpus N ...
 
+Timing: the K steps run back to back between two CUDA events (nothing
+recorded between kernels). The roofline's per-kernel time comes from a
+separate loop of back-to-back launches of each kernel alone. Before the
+headline line, one line per remaining workload (planted 256x1024, linear
+weight 4096x4096, 64 stacked experts, NVFP4 8192x8192) gives its median
+kernel time and a bit-exact check against the oracle on sampled rows.
+
 Multi-GPU: every rank quantizes its own batch (rows are independent, so the
 path shards with no exchange); value = bytes of all ranks / max over ranks of
 the device-timed region ("scaling": "weak").
 
-``--impl reference`` times the CPU oracle (test infrastructure) on host cores
-on a bounded sample of the same workload. ``--suite`` prints one extra JSON
-line per workload kernel (documentation, not the default line).
+``--impl reference`` times the CPU oracle (test infrastructure) on the host's
+cores (row chunks on threads, each running the single-threaded oracle) on a
+bounded sample of the same workload. ``--suite`` prints one extra JSON line
+per workload kernel (documentation, not the default line).
 """
 from __future__ import annotations
 
 import argparse
+import ctypes
 import datetime
 import hashlib
 import json
@@ -218,31 +227,88 @@ def reduce_max(value: float, world: int, device) -> float:
 
 # ------------------------------------------------------------ CPU oracle
 
-def time_oracle_round_trip(x: np.ndarray, min_seconds: float):
-    """Oracle MXFP8 quantize + swizzle + dequantize of the rows `x`, repeated
-    until min_seconds have elapsed; returns (seconds per pass, passes,
-    (qweight, scale, dequantized bf16 bits))."""
+def host_threads(cap: int = 64) -> int:
+    """Host cores this process may run on (capped)."""
+    try:
+        n = len(os.sched_getaffinity(0))
+    except AttributeError:
+        n = os.cpu_count() or 1
+    return max(1, min(cap, n))
+
+
+def oracle_round_trip(x: np.ndarray):
+    """Oracle MXFP8 quantize + swizzle + dequantize of the rows x (one
+    single-threaded call of each)."""
+    import oracle
+    q, s = oracle.mxfp8_quantize(x)
+    z = oracle.swizzle_scales(s)
+    y = oracle.mxfp8_dequantize(q, s, out="bf16")
+    return q, s, z, y
+
+
+def pmap(fn, items, threads: int):
+    """[fn(i) for i in items] on `threads` host threads. The oracle's C calls
+    release the interpreter lock (ctypes), so each thread runs the unchanged
+    single-threaded oracle on its own item."""
+    from concurrent.futures import ThreadPoolExecutor
+    items = list(items)
+    if threads == 1:
+        return [fn(i) for i in items]
+    with ThreadPoolExecutor(threads) as ex:
+        return list(ex.map(fn, items))
+
+
+def oracle_rows_parallel(fn, x: np.ndarray, threads: int, chunk: int = 128):
+    """fn over consecutive row chunks of x on `threads` host threads; results
+    in row order."""
+    parts = [np.ascontiguousarray(x[i:i + chunk]) for i in range(0, x.shape[0], chunk)]
+    return pmap(fn, parts, threads)
+
+
+def calibrate_row_seconds(x: np.ndarray, rows: int = 64) -> float:
+    """Single-thread oracle round-trip seconds per row of x."""
     import oracle
     oracle.build()
+    t0 = time.perf_counter()
+    oracle_round_trip(np.ascontiguousarray(x[:rows]))
+    return (time.perf_counter() - t0) / rows
+
+
+def cpu_baseline(x_full: np.ndarray, target_s: float = 12.0):
+    """The oracle round trip on all host cores (row chunks on threads) over
+    the first rows of the workload, as many as fit in about target_s.
+    Returns (cpu_baseline dict, rows, concatenated oracle outputs)."""
+    threads = host_threads()
+    t_row = calibrate_row_seconds(x_full)
+    rows = int(min(x_full.shape[0], max(128, target_s * threads / max(t_row, 1e-9))))
+    rows = rows // 128 * 128 or min(128, x_full.shape[0])
+    x = x_full[:rows]
+    t0 = time.perf_counter()
+    res = oracle_rows_parallel(oracle_round_trip, x, threads)
+    el = time.perf_counter() - t0
+    outs = tuple(np.concatenate([r[i] for r in res]) for i in range(4))
+    nbytes = mxfp8_quant_bytes(rows, N_COLS) + mxfp8_dequant_bytes(rows, N_COLS)
+    return ({"value": nbytes / el / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle",
+             "sample": f"first {rows} of {M_ROWS} rows of the activation workload, quantize "
+                       f"(+swizzle) + dequantize, scalar C oracle on {threads} threads "
+                       f"(128-row chunks), one pass of {el:.1f} s"},
+            rows, outs)
+
+
+def cpu_baseline_single_thread_planted(min_seconds: float = 1.0):
+    """The oracle on one core over the small planted workload (256x1024)."""
+    x = W.planted()
     passes, t0 = 0, time.perf_counter()
     while True:
-        q, s = oracle.mxfp8_quantize(x)
-        oracle.swizzle_scales(s)
-        y = oracle.mxfp8_dequantize(q, s, out="bf16")
+        oracle_round_trip(x)
         passes += 1
         el = time.perf_counter() - t0
         if el >= min_seconds:
-            return el / passes, passes, (q, s, y)
-
-
-def cpu_baseline(x_full: np.ndarray, rows: int = 2048, min_seconds: float = 12.0):
-    """The oracle timed on the first `rows` rows; also returns its outputs."""
-    x = np.ascontiguousarray(x_full[:rows])
-    sec, passes, outs = time_oracle_round_trip(x, min_seconds)
-    nbytes = mxfp8_quant_bytes(rows, N_COLS) + mxfp8_dequant_bytes(rows, N_COLS)
-    return {"value": nbytes / sec / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
-            "sample": f"first {rows} of {M_ROWS} rows of the activation workload, quantize "
-                      f"(+swizzle) + dequantize, {passes} passes, single-threaded scalar C"}, outs
+            break
+    nbytes = mxfp8_quant_bytes(256, 1024) + mxfp8_dequant_bytes(256, 1024)
+    return {"value": nbytes * passes / el / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": f"planted 256x1024, quantize (+swizzle) + dequantize, {passes} passes, "
+                      "one thread"}
 
 
 def run_reference(args):
@@ -251,32 +317,29 @@ def run_reference(args):
         return
     x_all = W.activation(M=M_ROWS, N=N_COLS)
     input_sha = hashlib.sha256(x_all.tobytes()).hexdigest()[:16]
-    t_row, _, _ = time_oracle_round_trip(np.ascontiguousarray(x_all[:64]), 0.5)
-    t_row /= 64
-    budget = 150.0
-    rows = int(max(1, min(M_ROWS, budget / max(1, args.steps + args.warmup) / t_row)))
-    x = np.ascontiguousarray(x_all[:rows])
-    import oracle
+    threads = host_threads()
+    t_row = calibrate_row_seconds(x_all)
+    budget = 120.0
+    rows = int(max(128, min(M_ROWS, budget / max(1, args.steps + args.warmup) * threads / t_row)))
+    rows = min(M_ROWS, rows // 128 * 128 or 128)
+    x = x_all[:rows]
     for _ in range(args.warmup):
-        q, s = oracle.mxfp8_quantize(x)
-        oracle.swizzle_scales(s)
-        oracle.mxfp8_dequantize(q, s, out="bf16")
+        oracle_rows_parallel(oracle_round_trip, x, threads)
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        q, s = oracle.mxfp8_quantize(x)
-        oracle.swizzle_scales(s)
-        oracle.mxfp8_dequantize(q, s, out="bf16")
+        oracle_rows_parallel(oracle_round_trip, x, threads)
     el = time.perf_counter() - t0
     nbytes = (mxfp8_quant_bytes(rows, N_COLS) + mxfp8_dequant_bytes(rows, N_COLS)) * args.steps
     value = nbytes / el / 1e9
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s",
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": el / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": config_block(world, input_sha),
-            "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle",
-                             "sample": f"first {rows} rows per step of the {M_ROWS}x{N_COLS} "
-                                       "activation workload, single-threaded scalar C"},
+            "cpu_baseline": {"value": value, "unit": "GB/s", "cores": threads, "kind": "oracle",
+                             "sample": f"first {rows} of {M_ROWS} rows per step of the "
+                                       f"{M_ROWS}x{N_COLS} activation workload, scalar C oracle "
+                                       f"on {threads} threads (128-row chunks)"},
             "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -297,6 +360,186 @@ def config_block(world, input_sha=None):
 
 # -------------------------------------------------------------------- main
 
+def events_loop(stream, fn, n: int) -> float:
+    """Device milliseconds of n back-to-back calls of fn() on `stream`, with
+    nothing recorded between them (events only before the first and after
+    the last)."""
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(n):
+        fn()
+    b.record(stream)
+    while not b.query():
+        time.sleep(0.0002)
+    torch.cuda.synchronize()
+    return a.elapsed_time(b)
+
+
+def e2e_pipelined(mxq, x_h, outs_h, chunk_rows: int, device):
+    """One end-to-end step through the public Python API: the pinned host
+    input goes to the device in row chunks on one stream, each chunk is
+    quantized (+ swizzled scales) and dequantized on a second stream as soon
+    as it has arrived, and its outputs go back to pinned host memory on a
+    third, so uploads, kernels and downloads of different chunks overlap.
+    chunk_rows is a multiple of 128, so each chunk's swizzled scales are one
+    contiguous slice of the full layout. Returns the device milliseconds of
+    the step (events on the caller's stream around all three streams)."""
+    q_h, s_h, z_h, y_h = outs_h
+    M, N = x_h.shape
+    Sp = (N // 32 + 3) // 4 * 4
+    main = torch.cuda.current_stream(device)
+    up, comp, down = e2e_pipelined.streams
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(main)
+    for st in (up, comp, down):
+        st.wait_event(e0)
+    x_d = e2e_pipelined.x_d
+    keep = []
+    for r0 in range(0, M, chunk_rows):
+        r1 = min(M, r0 + chunk_rows)
+        with torch.cuda.stream(up):
+            x_d[r0:r1].copy_(x_h[r0:r1], non_blocking=True)
+            arrived = torch.cuda.Event()
+            arrived.record(up)
+        with torch.cuda.stream(comp):
+            comp.wait_event(arrived)
+            q, s, z = mxq.mxfp8_quantize(x_d[r0:r1], swizzled=True)
+            y = mxq.mxfp8_dequantize(q, s, torch.bfloat16)
+            done = torch.cuda.Event()
+            done.record(comp)
+        with torch.cuda.stream(down):
+            down.wait_event(done)
+            q_h[r0:r1].copy_(q, non_blocking=True)
+            s_h[r0:r1].copy_(s, non_blocking=True)
+            z_h[r0 * Sp:r0 * Sp + z.numel()].copy_(z, non_blocking=True)
+            y_h[r0:r1].copy_(y, non_blocking=True)
+        keep.append((q, s, z, y))
+    fin = torch.cuda.Event()
+    fin.record(down)
+    main.wait_event(fin)
+    e1.record(main)
+    e1.synchronize()                     # the chunk outputs in `keep` are free after this
+    del keep
+    return e0.elapsed_time(e1)
+
+
+def sample_rows(M: int, n: int, seed: int) -> np.ndarray:
+    """First, last and n seeded random rows of M (sorted, unique)."""
+    rng = np.random.default_rng(seed)
+    rows = set(range(min(M, 64))) | set(range(max(0, M - 64), M))
+    rows |= set(int(r) for r in rng.integers(0, M, n))
+    return np.array(sorted(rows))
+
+
+def config_lines(mxq, device, flush):
+    """One bounded line per remaining workload of the statement of the
+    problem: median device time over repeated launches, algorithmic bytes,
+    GB/s, fractions of the measured and spec HBM peaks, and a bit-exact
+    check of the timed launch's outputs against the oracle on sampled rows
+    (all rows for the small workloads)."""
+    import oracle
+    peak, kind = hbm_peak()
+    threads = host_threads()
+    lines = []
+
+    def bf(a):
+        return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(device)
+
+    def line(cfg, name, nbytes, t_ms, exact, checked, extra=None):
+        med = t_ms
+        d = {"config_line": cfg, "workload": name, "median_us": med * 1e3, "bytes": nbytes,
+             "gbs": nbytes / med / 1e6, "frac_of_" + kind: nbytes / med / 1e6 / peak,
+             "frac_of_spec_8tbs": nbytes / med / 1e6 / SPEC_HBM_GBS,
+             "bit_exact_vs_oracle": bool(exact), "checked": checked}
+        if extra:
+            d.update(extra)
+        lines.append(d)
+        print(json.dumps(d), flush=True)
+
+    # 1: planted 256x1024, quantize (+swizzle) and dequantize, L2 flushed
+    x = W.planted()
+    xd = bf(x)
+    tq = time_kernel(lambda: mxq.mxfp8_quantize(xd, swizzled=True), 50, flush)[0]
+    q, s, z = mxq.mxfp8_quantize(xd, swizzled=True)
+    td = time_kernel(lambda: mxq.mxfp8_dequantize(q, s), 50, flush)[0]
+    y = mxq.mxfp8_dequantize(q, s)
+    qo, so, zo, yo = oracle_round_trip(x)
+    ok = (np.array_equal(q.cpu().numpy(), qo) and np.array_equal(s.cpu().numpy(), so)
+          and np.array_equal(z.cpu().numpy(), zo)
+          and np.array_equal(y.view(torch.int16).cpu().numpy().view(np.uint16), yo))
+    line(1, "MXFP8 quantize (+swizzle) + dequantize, planted bf16 256x1024 (L2 flushed, "
+            "launch-bound)", mxfp8_quant_bytes(256, 1024) + mxfp8_dequant_bytes(256, 1024),
+         tq + td, ok, "all rows, all outputs",
+         {"quantize_us": tq * 1e3, "dequantize_us": td * 1e3,
+          "cpu_baseline_single_thread": cpu_baseline_single_thread_planted()})
+
+    # 2: linear weight 4096x4096, quantize; 8 rotating input/output sets (> 2x L2)
+    x = W.linear_weight()
+    xs = [bf(x) for _ in range(8)]
+    outs = [mxq.mxfp8_quantize(t) for t in xs]
+    L, sp = mxq.lib, ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+    P = [[ctypes.c_void_p(t.data_ptr()) for t in (xs[i], outs[i][0], outs[i][1])] for i in range(8)]
+    k = [0]
+
+    def rot():
+        p = P[k[0] % 8]
+        k[0] += 1
+        L.mxfp8_quantize(p[0], 0, 4096, 4096, 4096, p[1], p[2], None, sp)
+
+    t = time_kernel(rot, 48)[0]
+    qo, so = zip(*oracle_rows_parallel(oracle.mxfp8_quantize, x, threads, 256))
+    ok = (np.array_equal(outs[0][0].cpu().numpy(), np.concatenate(qo))
+          and np.array_equal(outs[0][1].cpu().numpy(), np.concatenate(so)))
+    line(2, "MXFP8 quantize, linear weight bf16 4096x4096 (8 rotating input/output sets)",
+         mxfp8_quant_bytes(4096, 4096, swizzled=False), t, ok, "all rows")
+    del xs, outs, P
+    torch.cuda.empty_cache()
+
+    # 4: 64 experts 2048x7168 stacked, one grouped launch (+ per-expert swizzled scales)
+    x = W.experts()
+    xd = bf(x)
+    del x
+    t = time_kernel(lambda: mxq.mxfp8_quantize_grouped(xd, swizzled=True), 10)[0]
+    q, s, z = mxq.mxfp8_quantize_grouped(xd, swizzled=True)
+    picks = [0, 9, 21, 30, 42, 51, 58, 63]
+    xh = {e: xd[e].view(torch.int16).cpu().numpy().view(np.uint16) for e in picks}
+    res = pmap(lambda e: oracle.mxfp8_quantize(xh[e]), picks, threads)
+    blk = 2048 * 224
+    ok = True
+    for e, (qo, so) in zip(picks, res):
+        ok &= np.array_equal(q[e].cpu().numpy(), qo) and np.array_equal(s[e].cpu().numpy(), so)
+        ok &= np.array_equal(z[e * blk:(e + 1) * blk].cpu().numpy(), oracle.swizzle_scales(so))
+    line(4, "grouped MXFP8 quantize (+ per-expert swizzled scales), 64 stacked experts bf16 "
+            "2048x7168, one launch", mxfp8_quant_bytes(64 * 2048, 7168), t, ok,
+         f"experts {picks}, all outputs")
+    del xd, q, s, z
+    torch.cuda.empty_cache()
+
+    # 5: NVFP4 two passes, 8192x8192
+    x = W.nvfp4_tensor()
+    xd = bf(x)
+    ws = torch.empty(mxq.nvfp4_workspace_bytes(), dtype=torch.uint8, device=device)
+    t = time_kernel(lambda: mxq.nvfp4_quantize(xd, workspace=ws), 30)[0]
+    p, b, g = mxq.nvfp4_quantize(xd, workspace=ws)
+    tg = time_kernel(lambda: mxq.nvfp4_quantize(xd, global_scale=g), 30)[0]
+    go = oracle.nvfp4_global_amax(x) / np.float32(2688.0)
+    rows = sample_rows(8192, 512, 5)
+    res = oracle_rows_parallel(lambda xr: oracle.nvfp4_quantize(xr, float(go))[:2],
+                               x[rows], threads, 64)
+    po, bo = np.concatenate([r[0] for r in res]), np.concatenate([r[1] for r in res])
+    ok = (np.float32(g.item()) == np.float32(go)
+          and np.array_equal(p.cpu().numpy()[rows], po) and np.array_equal(b.cpu().numpy()[rows], bo))
+    line(5, "NVFP4 two-level quantize (amax pass + block pass), bf16 8192x8192",
+         nvfp4_quant_bytes(8192, 8192), t, ok, f"global scale and {rows.size} sampled rows",
+         {"single_read_bytes": nvfp4_quant_bytes(8192, 8192, two_pass=False),
+          "gbs_single_read_count": nvfp4_quant_bytes(8192, 8192, two_pass=False) / t / 1e6,
+          "block_pass_given_scale_us": tg * 1e3,
+          "block_pass_gbs": nvfp4_quant_bytes(8192, 8192, two_pass=False) / tg / 1e6})
+    del xd, p, b
+    torch.cuda.empty_cache()
+    return lines
+
+
 def run(args):
     world, rank, local = dist_setup(args)
     torch.cuda.set_device(local)
@@ -307,7 +550,6 @@ def run(args):
                                 device_id=device)
     import nvfp4_block_scaled_sm_b200 as mxq
     L = mxq.lib
-    import ctypes
 
     xb = W.activation(seed=2 + 1000 * rank, M=M_ROWS, N=N_COLS)
     input_sha = hashlib.sha256(xb.tobytes()).hexdigest()[:16] if rank == 0 else None
@@ -322,93 +564,70 @@ def run(args):
     sp = ctypes.c_void_p(stream.cuda_stream)
     P = [ctypes.c_void_p(t.data_ptr()) for t in (x, q, s, swz, y)]
 
-    def step():
+    def quant():
         st = L.mxfp8_quantize(P[0], 0, M, N, N, P[1], P[2], P[3], sp)
         if st:
             raise mxq.MxqError("mxfp8_quantize", st, L.mxq_status_string(st).decode())
+
+    def dequant():
         st = L.mxfp8_dequantize(P[1], P[2], M, N, P[4], 0, sp)
         if st:
             raise mxq.MxqError("mxfp8_dequantize", st, L.mxq_status_string(st).decode())
+
+    def step():
+        quant()
+        dequant()
 
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize(device)
 
+    # the timed region: K steps back to back, events only around all of them
     K = args.steps
-    # Per-kernel durations come from events around the two kernels of every
-    # SAMPLE_EVERY-th step only: an event recorded between two kernels ends
-    # their programmatic overlap, so events on every step would slow the step.
-    # A short run samples more often (every step at K < 16) so that the
-    # average still rests on about eight launches or more.
-    every = min(SAMPLE_EVERY, max(1, K // 8))
-    sampled = [k for k in range(K) if k % every == every - 1] or [K - 1]
-    ev = {k: [torch.cuda.Event(enable_timing=True) for _ in range(3)] for k in sampled}
-    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize(device)
     with ClockSampler(device) as clk:
-        t_start.record(stream)
-        for k in range(K):
-            e = ev.get(k)
-            if e:
-                e[0].record(stream)
-            L.mxfp8_quantize(P[0], 0, M, N, N, P[1], P[2], P[3], sp)
-            if e:
-                e[1].record(stream)
-            L.mxfp8_dequantize(P[1], P[2], M, N, P[4], 0, sp)
-            if e:
-                e[2].record(stream)
-        t_end.record(stream)
-        # wait by polling so that the sampler thread gets the interpreter while
-        # the GPU works through the queued steps
-        while not t_end.query():
-            time.sleep(0.0002)
-        torch.cuda.synchronize(device)
+        elapsed_ms = events_loop(stream, step, K)
     if world > 1:
         torch.distributed.barrier()
-    elapsed_ms = t_start.elapsed_time(t_end)
-    q_ms = [ev[k][0].elapsed_time(ev[k][1]) for k in sampled]
-    d_ms = [ev[k][1].elapsed_time(ev[k][2]) for k in sampled]
     max_ms = reduce_max(elapsed_ms, world, device)
 
-    # outputs of the timed region's last step, kept for the CPU-baseline leg's check
-    n_check = 2048
-    q_last = q[:n_check].cpu().numpy()
-    s_last = s[:n_check].cpu().numpy()
-    y_last = y[:n_check].view(torch.int16).cpu().numpy().view(np.uint16)
+    # outputs of the timed region's last step, kept for the oracle check
+    q_out, s_out = q.cpu().numpy(), s.cpu().numpy()
+    z_out = swz.cpu().numpy()
+    y_out = y.view(torch.int16).cpu().numpy().view(np.uint16)
 
-    # end-to-end through the public API: pinned host input -> device, quantize,
-    # dequantize, all outputs -> pinned host, every step
-    e2e_steps = max(1, min(K, 10))
+    # per-kernel device time for the roofline: R launches of one kernel back
+    # to back between two events (every launch rewrites the same outputs)
+    R = max(20, min(200, K))
+    with ClockSampler(device) as clk_k:
+        q_ms = events_loop(stream, quant, R) / R
+        d_ms = events_loop(stream, dequant, R) / R
+    q_ms = reduce_max(q_ms, world, device)
+    d_ms = reduce_max(d_ms, world, device)
+
+    # end to end through the public API: pinned host input -> device, quantize
+    # (+ swizzled scales), dequantize, every output -> pinned host, each step,
+    # with uploads, kernels and downloads of row chunks overlapped on 3 streams
+    e2e_steps = max(3, min(K, 10))
+    chunk_rows = 2048
     x_h = torch.from_numpy(xb.view(np.int16)).view(torch.bfloat16).pin_memory()
-    q_h = torch.empty(q.shape, dtype=q.dtype).pin_memory()
-    s_h = torch.empty(s.shape, dtype=s.dtype).pin_memory()
-    z_h = torch.empty(swz.shape, dtype=swz.dtype).pin_memory()
-    y_h = torch.empty(y.shape, dtype=y.dtype).pin_memory()
-    x_d = torch.empty_like(x)
-
-    def e2e_step():
-        x_d.copy_(x_h, non_blocking=True)
-        qq, ss, zz = mxq.mxfp8_quantize(x_d, swizzled=True)
-        yy = mxq.mxfp8_dequantize(qq, ss, torch.bfloat16)
-        q_h.copy_(qq, non_blocking=True)
-        s_h.copy_(ss, non_blocking=True)
-        z_h.copy_(zz, non_blocking=True)
-        y_h.copy_(yy, non_blocking=True)
-        torch.cuda.current_stream(device).synchronize()
-
-    e2e_step()
+    outs_h = (torch.empty(q.shape, dtype=q.dtype).pin_memory(),
+              torch.empty(s.shape, dtype=s.dtype).pin_memory(),
+              torch.empty(swz.shape, dtype=swz.dtype).pin_memory(),
+              torch.empty(y.shape, dtype=y.dtype).pin_memory())
+    e2e_pipelined.streams = tuple(torch.cuda.Stream(device) for _ in range(3))
+    e2e_pipelined.x_d = torch.empty_like(x)
+    e2e_pipelined(mxq, x_h, outs_h, chunk_rows, device)
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize(device)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(e2e_steps):
-        e2e_step()
-    e1.record(stream)
-    torch.cuda.synchronize(device)
-    e2e_ms = reduce_max(e0.elapsed_time(e1) / e2e_steps, world, device)
+    e2e_ms = [e2e_pipelined(mxq, x_h, outs_h, chunk_rows, device) for _ in range(e2e_steps)]
+    e2e_ms = reduce_max(statistics.fmean(e2e_ms), world, device)
+    e2e_same = (np.array_equal(outs_h[0].numpy(), q_out) and np.array_equal(outs_h[1].numpy(), s_out)
+                and np.array_equal(outs_h[2].numpy(), z_out)
+                and np.array_equal(outs_h[3].view(torch.int16).numpy().view(np.uint16), y_out))
 
     if world > 1:
         torch.distributed.barrier()
@@ -416,14 +635,18 @@ def run(args):
     if rank != 0:
         return
 
+    extra = []
+    flush = torch.empty(64 * 2**20, dtype=torch.float32, device=device)  # 256 MB > L2
+    if not args.headline_only:
+        extra = config_lines(mxq, device, flush)
+
     qb, db = mxfp8_quant_bytes(M, N), mxfp8_dequant_bytes(M, N)
     step_bytes = qb + db
     value = step_bytes * K * world / (max_ms / 1e3) / 1e9
     peak, peak_kind = hbm_peak()
-    q_avg, d_avg = statistics.fmean(q_ms), statistics.fmean(d_ms)
     kernels = {
-        "mx_quant_kernel": {"avg_us": q_avg * 1e3, "bytes": qb, "gbs": qb / (q_avg / 1e3) / 1e9},
-        "mx_dequant_kernel": {"avg_us": d_avg * 1e3, "bytes": db, "gbs": db / (d_avg / 1e3) / 1e9},
+        "mx_quant_kernel": {"avg_us": q_ms * 1e3, "bytes": qb, "gbs": qb / (q_ms / 1e3) / 1e9},
+        "mx_dequant_kernel": {"avg_us": d_ms * 1e3, "bytes": db, "gbs": db / (d_ms / 1e3) / 1e9},
     }
     for k in kernels.values():
         k["frac_of_measured"] = k["gbs"] / peak
@@ -439,24 +662,39 @@ def run(args):
         "roofline": {"bound": "hbm", "kernel": dom, "achieved": kernels[dom]["gbs"], "peak": peak,
                      "peak_kind": peak_kind, "unit": "GB/s",
                      "frac": kernels[dom]["gbs"] / peak,
+                     "frac_basis": f"{peak_kind} copy bandwidth ({peak:.1f} GB/s); the statement "
+                                   "of the problem's 80 % target is against the 8 TB/s spec: "
+                                   "frac_of_spec_8tbs",
                      "frac_of_spec_8tbs": kernels[dom]["gbs"] / SPEC_HBM_GBS,
+                     "spec_80pct_target_met": kernels[dom]["gbs"] >= 0.8 * SPEC_HBM_GBS,
                      "algorithmic_bytes_per_launch": kernels[dom]["bytes"],
-                     "traffic": recorded_traffic(dom)},
+                     "traffic": recorded_traffic(dom),
+                     "timing": f"{R} back-to-back launches of each kernel between two events"},
         "breakdown": kernels,
         "e2e": {"value": step_bytes * world / (e2e_ms / 1e3) / 1e9, "unit": "GB/s",
                 "ms_per_step": e2e_ms, "steps": e2e_steps,
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "pipeline": f"{M // chunk_rows} row chunks; upload, kernels and download on "
+                            "three streams", "outputs_equal_device_run": bool(e2e_same)},
         "gpu_launches": 2 * K,
-        "kernel_time_sampling": f"events around both kernels on every {every}th step "
-                                f"({len(sampled)} of {K} steps)",
         "clocks": clk.summary(),
+        "clocks_kernel_loops": clk_k.summary(),
     }
     if not args.no_cpu_baseline:
-        line["cpu_baseline"], (qo, so, yo) = cpu_baseline(xb, n_check)
+        line["cpu_baseline"], rows, (qo, so, zo, yo) = cpu_baseline(xb)
+        Sp = (S + 3) // 4 * 4
         line["verified_bit_exact_first_rows"] = {
-            "rows": n_check,
-            "equal_to_oracle": bool(np.array_equal(q_last, qo) and np.array_equal(s_last, so)
-                                    and np.array_equal(y_last, yo))}
+            "rows": rows,
+            "equal_to_oracle": bool(np.array_equal(q_out[:rows], qo)
+                                    and np.array_equal(s_out[:rows], so)
+                                    and np.array_equal(z_out[:rows * Sp], zo)
+                                    and np.array_equal(y_out[:rows], yo))}
+    if extra:
+        line["configs"] = {str(d["config_line"]): {"gbs": round(d["gbs"], 1),
+                                                    "median_us": round(d["median_us"], 2),
+                                                    "frac_of_" + peak_kind: round(d["frac_of_" + peak_kind], 3),
+                                                    "bit_exact": d["bit_exact_vs_oracle"]}
+                           for d in extra}
     print(json.dumps(line), flush=True)
     if args.suite:
         run_suite(device)
@@ -542,6 +780,28 @@ def run_suite(device, only=None):
 
         emit("mxfp8_quantize linear_weight 4096x4096 (8 rotating input/output sets)",
              mxfp8_quant_bytes(4096, 4096, swizzled=False), time_kernel(rotating, 48))
+        # eight such weights: one call each, against one grouped launch over
+        # the stacked eight (rotating between two stacks, 2 x 268 MB > L2)
+        stacks = [torch.stack(xs), torch.stack(xs).clone()]
+        del xs, qs, ss
+        k[0] = 0
+
+        def eight_calls():
+            st = stacks[k[0] % 2]
+            k[0] += 1
+            for i in range(8):
+                mxq.mxfp8_quantize(st[i])
+
+        def one_grouped():
+            st = stacks[k[0] % 2]
+            k[0] += 1
+            mxq.mxfp8_quantize_grouped(st)
+
+        eight = 8 * mxfp8_quant_bytes(4096, 4096, swizzled=False)
+        emit("8 x mxfp8_quantize linear_weight 4096x4096, one call each", eight,
+             time_kernel(eight_calls, 20))
+        emit("mxfp8_quantize_grouped of the 8 stacked linear weights 8x4096x4096, one launch",
+             eight, time_kernel(one_grouped, 20))
 
     def activation():
         x = bf(W.activation())
@@ -668,6 +928,8 @@ def main():
     ap.add_argument("--suite-only", default=None,
                     help="time only the workload kernels whose workload name contains this")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--headline-only", action="store_true",
+                    help="skip the lines of the other workloads")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")

@@ -78,7 +78,7 @@ typedef enum { MXQ_BF16 = 0, MXQ_FP32 = 1 } mxq_dtype;
 /* MX element formats (mx_fake_quantize). */
 typedef enum { MXQ_FMT_MXFP8 = 0, MXQ_FMT_MXFP4 = 1 } mxq_mx_format;
 
-#define MXQ_ABI_VERSION 1
+#define MXQ_ABI_VERSION 2
 #define MXQ_MXFP8_GROUP 32
 #define MXQ_NVFP4_BLOCK 16
 #define MXQ_GROUPED_MAX_EXPERTS 1024
@@ -131,19 +131,61 @@ mxq_status mxfp8_quantize(const void* x, int dt, int64_t M, int64_t N, int64_t l
 mxq_status mxfp8_dequantize(const uint8_t* qweight, const uint8_t* scale, int64_t M,
                             int64_t N, void* y, int out_dt, mxq_stream_t stream);
 
-/* Grouped MXFP8 quantize of E expert tensors in one launch ("PR #1935
- * 完整报告 ...", 实现拆解 item 4).
+/* Grouped MXFP8 quantize of a stack of E expert weights held in one tensor,
+ * in one launch ("PR #1935 完整报告 ...", 实现拆解 item 4: grouped
+ * quantization of stacked expert weights, mxfp8_group_quantize; "V4 mxfp4
+ * #1372", description: MoE expert weights).
+ *  x            [M_total, N] bf16 or fp32 (dt), contiguous rows; expert e
+ *               owns rows [row_offsets[e], row_offsets[e+1]).
+ *  row_offsets  DEVICE int64 [E + 1], 8-byte aligned, non-decreasing, with
+ *               row_offsets[0] == 0 and row_offsets[E] == M_total (those two
+ *               entries are taken as 0 and M_total, not read). Experts may be
+ *               empty. 1 <= E <= MXQ_GROUPED_MAX_EXPERTS.
+ *  qweight [M_total, N], scale [M_total, N/32]: compact, as for M_total rows.
+ * Groups never cross rows, so every output byte equals what mxfp8_quantize
+ * gives each expert on its own and what it gives the flattened [M_total, N]
+ * tensor: the offsets do not change the compact outputs, and this call does
+ * not read them (mxfp8_quantize_grouped_swizzled does). */
+mxq_status mxfp8_quantize_grouped(const void* x, int dt, int32_t E, const int64_t* row_offsets,
+                                  int64_t M_total, int64_t N, uint8_t* qweight, uint8_t* scale,
+                                  mxq_stream_t stream);
+
+/* mxfp8_quantize_grouped that also writes each expert's scales in its own
+ * 128x4-tile swizzled layout (the layout described at mxfp8_quantize), as a
+ * grouped block-scaled GEMM over the experts reads them: expert e's block is
+ * mxq_swizzled_scale_bytes(M_e, N/32) bytes (its rows padded to a multiple
+ * of 128, padding bytes 0x00) and starts where expert e-1's ends.
+ *  scale_swz  device buffer of swz_bytes bytes; it must hold the sum over the
+ *             experts of mxq_swizzled_scale_bytes(M_e, N/32), which is at
+ *             most mxq_grouped_swizzled_scale_bytes_max(E, M_total, N/32).
+ * The kernel reads row_offsets on the device. Offsets that break the rules
+ * above are clamped into a non-decreasing sequence from 0 to M_total, and no
+ * byte at or past scale_swz + swz_bytes is written, whatever the offsets. */
+mxq_status mxfp8_quantize_grouped_swizzled(const void* x, int dt, int32_t E,
+                                           const int64_t* row_offsets, int64_t M_total, int64_t N,
+                                           uint8_t* qweight, uint8_t* scale, uint8_t* scale_swz,
+                                           int64_t swz_bytes, mxq_stream_t stream);
+
+/* Upper bound of the per-expert swizzled scale bytes of E experts with
+ * M_total rows in all (each expert adds at most 127 padding rows):
+ * floor((M_total + 127 E) / 128) * 128 * ceil(S/4) * 4; -1 for negative
+ * sizes. */
+int64_t mxq_grouped_swizzled_scale_bytes_max(int32_t E, int64_t M_total, int64_t S);
+
+/* Grouped MXFP8 quantize of E expert tensors that live in separate
+ * allocations, in one launch.
  *  xs    HOST array of E device pointers; expert e is a contiguous
  *        [rows[e], N] tensor of dtype dt (16-byte aligned).
  *  rows  HOST array of E row counts (>= 0).
  *  qweight [sum rows, N] and scale [sum rows, N/32]: expert e's rows follow
  *        expert e-1's, as if the experts were stacked and quantized by
  *        mxfp8_quantize (identical bytes).
- * 1 <= E <= MXQ_GROUPED_MAX_EXPERTS. The host arrays are read during the call
- * only. */
-mxq_status mxfp8_quantize_grouped(int32_t E, const void* const* xs, const int64_t* rows,
-                                  int64_t N, int dt, uint8_t* qweight, uint8_t* scale,
-                                  mxq_stream_t stream);
+ * 1 <= E <= MXQ_GROUPED_MAX_EXPERTS (the pointers and per-expert tile counts
+ * travel in the kernel's parameters). The host arrays are read during the
+ * call only. */
+mxq_status mxfp8_quantize_grouped_ptrs(int32_t E, const void* const* xs, const int64_t* rows,
+                                       int64_t N, int dt, uint8_t* qweight, uint8_t* scale,
+                                       mxq_stream_t stream);
 
 /* MXFP8 columnwise quantize: groups of 32 consecutive ROWS of one column (the
  * layout a backward GEMM reads), i.e. the rowwise quantize of the transposed
@@ -191,12 +233,26 @@ mxq_status mxfp4_quantize(const void* x, int dt, int64_t M, int64_t N, int64_t l
 mxq_status mxfp4_dequantize(const uint8_t* packed, const uint8_t* scale, int64_t M, int64_t N,
                             void* y, int out_dt, mxq_stream_t stream);
 
-/* Grouped MXFP4 quantize of E expert tensors in one launch: arguments and
- * layout as for mxfp8_quantize_grouped, outputs packed [sum rows, N/2] and
- * scale [sum rows, N/32], identical to mxfp4_quantize of the stacked rows. */
-mxq_status mxfp4_quantize_grouped(int32_t E, const void* const* xs, const int64_t* rows,
-                                  int64_t N, int dt, uint8_t* packed, uint8_t* scale,
+/* Grouped MXFP4 quantize of a stacked tensor: arguments and rules as for
+ * mxfp8_quantize_grouped, outputs packed [M_total, N/2] and scale
+ * [M_total, N/32], identical to mxfp4_quantize of the stacked rows. */
+mxq_status mxfp4_quantize_grouped(const void* x, int dt, int32_t E, const int64_t* row_offsets,
+                                  int64_t M_total, int64_t N, uint8_t* packed, uint8_t* scale,
                                   mxq_stream_t stream);
+
+/* mxfp4_quantize_grouped plus per-expert swizzled scales, as for
+ * mxfp8_quantize_grouped_swizzled. */
+mxq_status mxfp4_quantize_grouped_swizzled(const void* x, int dt, int32_t E,
+                                           const int64_t* row_offsets, int64_t M_total, int64_t N,
+                                           uint8_t* packed, uint8_t* scale, uint8_t* scale_swz,
+                                           int64_t swz_bytes, mxq_stream_t stream);
+
+/* Grouped MXFP4 quantize of E experts in separate allocations: arguments as
+ * for mxfp8_quantize_grouped_ptrs, outputs packed [sum rows, N/2] and scale
+ * [sum rows, N/32]. */
+mxq_status mxfp4_quantize_grouped_ptrs(int32_t E, const void* const* xs, const int64_t* rows,
+                                       int64_t N, int dt, uint8_t* packed, uint8_t* scale,
+                                       mxq_stream_t stream);
 
 /* ------------------------------------------------------- fake quantize */
 
@@ -286,8 +342,12 @@ mxq_status nvfp4_quantize(const void* x, int dt, int64_t M, int64_t N, int64_t l
  * array inside the library, which every GPU that loads the library holds
  * until the process exits; the call allocates nothing.
  *  - The first call on a device looks up that array's device address with the
- *    caller's current device (one cudaGetSymbolAddress); make that first call
- *    before any stream capture. stream must belong to the current device.
+ *    caller's current device (one cudaGetSymbolAddress) and keeps it, keyed
+ *    by the id of the current CUDA context; make that first call before any
+ *    stream capture. A call that finds another context current (after a
+ *    cudaDeviceReset, say) looks the address up again, so make the first
+ *    call after such a change before any capture too. stream must belong to
+ *    the current device.
  *  - Every call on a device shares the one array, so calls whose work
  *    overlaps on the GPU (for example on two streams) race and give wrong
  *    results; serialize them. Nothing in the array needs to start at zero:
@@ -341,9 +401,14 @@ mxq_status nvfp4_amax_sliced(const void* x, int dt, int64_t M, int64_t N, int64_
                              int32_t n_slices, const int64_t* slice_rows, float* amax,
                              void* workspace, size_t ws_bytes, mxq_stream_t stream);
 
-/* NVFP4 dequantize: eff = decode_e4m3(s_b) * g and y = decode_e2m1(q) * eff,
- * both fp32 products, written as fp32 or bf16 (RNE). global_scale is a device
- * pointer. */
+/* NVFP4 dequantize ("Add FP8, NVFP4, and QARL training and export", review
+ * "What looked solid": the effective scale is the block scale times the
+ * global scale): eff = decode_e4m3(s_b) * g and y = decode_e2m1(q) * eff,
+ * both fp32 products, written as fp32 or bf16 (RNE); NaN products (only from
+ * a non-finite g) are written as the canonical NaN.
+ *  packed [M, N/2], block_scale [M, N/16] as nvfp4_quantize writes them;
+ *  global_scale device fp32 scalar; y [M, N] of out_dt, 16-byte aligned.
+ * Errors: N % 16 != 0, NULL pointers (M > 0), misalignment. */
 mxq_status nvfp4_dequantize(const uint8_t* packed, const uint8_t* block_scale,
                             const float* global_scale, int64_t M, int64_t N, void* y,
                             int out_dt, mxq_stream_t stream);

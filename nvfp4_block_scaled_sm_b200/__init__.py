@@ -27,7 +27,7 @@ __all__ = [
     "mxfp8_gemm",
     "nvfp4_amax", "nvfp4_quantize", "nvfp4_dequantize",
     "nvfp4_amax_sliced", "nvfp4_quantize_sliced", "nvfp4_quantize_experts",
-    "swizzled_scale_bytes", "nvfp4_workspace_bytes",
+    "swizzled_scale_bytes", "nvfp4_workspace_bytes", "set_output_allocator",
     "as_float8_e4m3", "as_float8_e8m0", "as_float4_e2m1x2",
 ]
 
@@ -62,11 +62,17 @@ def _load() -> ctypes.CDLL:
     L.mxq_nvfp4_workspace_bytes.argtypes, L.mxq_nvfp4_workspace_bytes.restype = [i64, i64], sz
     L.mxfp8_quantize.argtypes = [vp, i32, i64, i64, i64, vp, vp, vp, vp]
     L.mxfp8_dequantize.argtypes = [vp, vp, i64, i64, vp, i32, vp]
-    L.mxfp8_quantize_grouped.argtypes = [i32, vp, vp, i64, i32, vp, vp, vp]
+    L.mxfp8_quantize_grouped.argtypes = [vp, i32, i32, vp, i64, i64, vp, vp, vp]
+    L.mxfp8_quantize_grouped_swizzled.argtypes = [vp, i32, i32, vp, i64, i64, vp, vp, vp, i64, vp]
+    L.mxfp8_quantize_grouped_ptrs.argtypes = [i32, vp, vp, i64, i32, vp, vp, vp]
+    L.mxq_grouped_swizzled_scale_bytes_max.argtypes = [i32, i64, i64]
+    L.mxq_grouped_swizzled_scale_bytes_max.restype = i64
     L.mxfp8_quantize_columnwise.argtypes = [vp, i32, i64, i64, i64, vp, vp, vp, vp, vp]
     L.mxfp4_quantize.argtypes = [vp, i32, i64, i64, i64, vp, vp, vp, vp]
     L.mxfp4_dequantize.argtypes = [vp, vp, i64, i64, vp, i32, vp]
-    L.mxfp4_quantize_grouped.argtypes = [i32, vp, vp, i64, i32, vp, vp, vp]
+    L.mxfp4_quantize_grouped.argtypes = [vp, i32, i32, vp, i64, i64, vp, vp, vp]
+    L.mxfp4_quantize_grouped_swizzled.argtypes = [vp, i32, i32, vp, i64, i64, vp, vp, vp, i64, vp]
+    L.mxfp4_quantize_grouped_ptrs.argtypes = [i32, vp, vp, i64, i32, vp, vp, vp]
     L.mx_fake_quantize.argtypes = [i32, vp, i32, i64, i64, i64, vp, i32, vp]
     L.mxfp8_gemm.argtypes = [vp, vp, vp, vp, i64, i64, i64, vp, i32, vp, vp]
     L.nvfp4_amax.argtypes = [vp, i32, i64, i64, i64, vp, vp, sz, vp]
@@ -78,8 +84,10 @@ def _load() -> ctypes.CDLL:
                                         sz, vp]
     L.nvfp4_amax_sliced.argtypes = [vp, i32, i64, i64, i64, i32, vp, vp, vp, sz, vp]
     for f in ("mxfp8_quantize", "mxfp8_dequantize", "mxfp8_quantize_grouped",
+              "mxfp8_quantize_grouped_swizzled", "mxfp8_quantize_grouped_ptrs",
               "mxfp8_quantize_columnwise", "mxfp4_quantize", "mxfp4_dequantize",
-              "mxfp4_quantize_grouped", "mx_fake_quantize", "mxfp8_gemm", "nvfp4_amax",
+              "mxfp4_quantize_grouped", "mxfp4_quantize_grouped_swizzled",
+              "mxfp4_quantize_grouped_ptrs", "mx_fake_quantize", "mxfp8_gemm", "nvfp4_amax",
               "nvfp4_quantize_sliced", "nvfp4_amax_sliced",
               "nvfp4_quantize", "nvfp4_dequantize"):
         getattr(L, f).restype = i32
@@ -142,6 +150,35 @@ def _ptr(t: torch.Tensor | None):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
+_output_allocator = None
+
+
+def set_output_allocator(fn):
+    """Route every output and workspace tensor this module allocates through
+    ``fn(shape, dtype, device) -> torch.Tensor`` (for example a memory pool,
+    or a checker that places each buffer between guard bytes); ``None``
+    restores ``torch.empty``. The tensor returned must be contiguous, have
+    the requested shape and dtype and start on a 256-byte boundary. Returns
+    the previous allocator."""
+    global _output_allocator
+    prev, _output_allocator = _output_allocator, fn
+    return prev
+
+
+def _empty(shape, dtype: torch.dtype, device) -> torch.Tensor:
+    shape = (int(shape),) if isinstance(shape, int) else tuple(int(d) for d in shape)
+    if _output_allocator is None:
+        return torch.empty(shape, dtype=dtype, device=device)
+    t = _output_allocator(shape, dtype, device)
+    if tuple(t.shape) != shape or t.dtype != dtype or not t.is_contiguous():
+        raise RuntimeError("the output allocator returned a tensor of the wrong layout")
+    return t
+
+
+def _zeros(shape, dtype: torch.dtype, device) -> torch.Tensor:
+    return _empty(shape, dtype, device).zero_()
+
+
 def swizzled_scale_bytes(M: int, S: int) -> int:
     return int(lib.mxq_swizzled_scale_bytes(M, S))
 
@@ -156,12 +193,11 @@ def _mx_quantize(fn: str, x: torch.Tensor, swizzled: bool, per_byte: int):
     _require_cuda(x)
     dt = _dtype_code(x.dtype)
     M, N, ld = _rows_view(x)
-    q = torch.empty((*x.shape[:-1], N // per_byte), dtype=torch.uint8, device=x.device)
-    s = torch.empty((*x.shape[:-1], N // 32), dtype=torch.uint8, device=x.device)
+    q = _empty((*x.shape[:-1], N // per_byte), torch.uint8, x.device)
+    s = _empty((*x.shape[:-1], N // 32), torch.uint8, x.device)
     swz = None
     if swizzled:
-        swz = torch.empty(max(swizzled_scale_bytes(M, N // 32), 0), dtype=torch.uint8,
-                          device=x.device)
+        swz = _empty((max(swizzled_scale_bytes(M, N // 32), 0),), torch.uint8, x.device)
     _check(fn, getattr(lib, fn)(_ptr(x), dt, M, N, ld, _ptr(q), _ptr(s), _ptr(swz), _stream(x)))
     return (q, s, swz) if swizzled else (q, s)
 
@@ -177,15 +213,66 @@ def _mx_dequantize(fn: str, q: torch.Tensor, scale: torch.Tensor, dtype: torch.d
     M = q.numel() * per_byte // N if N else 0
     if scale.numel() != M * (N // 32):
         raise ValueError("scale does not match the codes")
-    y = torch.empty((*q.shape[:-1], N), dtype=dtype, device=q.device)
+    y = _empty((*q.shape[:-1], N), dtype, q.device)
     _check(fn, getattr(lib, fn)(_ptr(q), _ptr(scale), M, N, _ptr(y), _dtype_code(dtype),
                                 _stream(q)))
     return y
 
 
-def _mx_quantize_grouped(fn: str, xs, per_byte: int):
-    stacked = isinstance(xs, torch.Tensor)
-    parts = list(xs.unbind(0)) if stacked else list(xs)
+def _offsets_on(dev, row_offsets, E: int, M: int):
+    """(device int64 offsets [E + 1], host row counts or None) from row
+    offsets given as a sequence, a CPU tensor or a CUDA tensor."""
+    if isinstance(row_offsets, torch.Tensor) and row_offsets.is_cuda:
+        if row_offsets.dtype != torch.int64 or row_offsets.numel() != E + 1:
+            raise TypeError("row_offsets must be int64 with E + 1 entries")
+        return row_offsets.contiguous(), None
+    host = [int(v) for v in (row_offsets.tolist() if isinstance(row_offsets, torch.Tensor)
+                             else row_offsets)]
+    if len(host) != E + 1 or host[0] != 0 or host[-1] != M or \
+            any(b < a for a, b in zip(host[:-1], host[1:])):
+        raise ValueError(f"row_offsets must rise from 0 to the {M} rows in {E + 1} entries")
+    off = torch.tensor(host, dtype=torch.int64).to(dev, non_blocking=False)
+    return off, [b - a for a, b in zip(host[:-1], host[1:])]
+
+
+def _mx_quantize_grouped(fmt: str, xs, per_byte: int, row_offsets=None, swizzled=False):
+    if isinstance(xs, torch.Tensor) and (xs.dim() == 3 or row_offsets is not None):
+        # one stacked tensor: [E, M, N], or [M_total, N] with row offsets
+        _require_cuda(xs)
+        if not xs.is_contiguous():
+            raise ValueError("the stacked tensor must be contiguous")
+        dt = _dtype_code(xs.dtype)
+        N = xs.shape[-1]
+        M = xs.numel() // N if N else 0
+        if row_offsets is None:
+            E, R = xs.shape[0], xs.shape[1]
+            row_offsets = [e * R for e in range(E + 1)]
+        else:
+            if xs.dim() != 2:
+                raise ValueError("row_offsets go with a 2-D [M_total, N] tensor")
+            E = (row_offsets.numel() if isinstance(row_offsets, torch.Tensor)
+                 else len(row_offsets)) - 1
+        off, counts = _offsets_on(xs.device, row_offsets, E, M)
+        q = _empty((*xs.shape[:-1], N // per_byte), torch.uint8, xs.device)
+        s = _empty((*xs.shape[:-1], N // 32), torch.uint8, xs.device)
+        if not swizzled:
+            _check(f"{fmt}_quantize_grouped",
+                   getattr(lib, f"{fmt}_quantize_grouped")(_ptr(xs), dt, E, _ptr(off), M, N,
+                                                           _ptr(q), _ptr(s), _stream(xs)))
+            return q, s
+        if counts is not None:
+            nswz = sum(swizzled_scale_bytes(m, N // 32) for m in counts)
+        else:
+            nswz = int(lib.mxq_grouped_swizzled_scale_bytes_max(E, M, N // 32))
+        swz = _empty((nswz,), torch.uint8, xs.device)
+        _check(f"{fmt}_quantize_grouped_swizzled",
+               getattr(lib, f"{fmt}_quantize_grouped_swizzled")(
+                   _ptr(xs), dt, E, _ptr(off), M, N, _ptr(q), _ptr(s), _ptr(swz), nswz,
+                   _stream(xs)))
+        return q, s, swz
+    if swizzled:
+        raise ValueError("per-expert swizzled scales need one stacked tensor")
+    parts = list(xs.unbind(0)) if isinstance(xs, torch.Tensor) else list(xs)
     if not parts:
         raise ValueError("no experts")
     _require_cuda(*parts)
@@ -201,15 +288,14 @@ def _mx_quantize_grouped(fn: str, xs, per_byte: int):
     E = len(parts)
     total = sum(rows)
     dev = parts[0].device
-    q = torch.empty((total, N // per_byte), dtype=torch.uint8, device=dev)
-    s = torch.empty((total, N // 32), dtype=torch.uint8, device=dev)
+    q = _empty((total, N // per_byte), torch.uint8, dev)
+    s = _empty((total, N // 32), torch.uint8, dev)
     ptrs = (ctypes.c_void_p * E)(*[p.data_ptr() for p in parts])
     rws = (ctypes.c_int64 * E)(*rows)
+    fn = f"{fmt}_quantize_grouped_ptrs"
     _check(fn, getattr(lib, fn)(E, ctypes.cast(ptrs, ctypes.c_void_p),
                                 ctypes.cast(rws, ctypes.c_void_p), N, dt, _ptr(q), _ptr(s),
                                 _stream(parts[0])))
-    if stacked:
-        return q.view(*xs.shape[:-1], N // per_byte), s.view(*xs.shape[:-1], N // 32)
     return q, s
 
 
@@ -230,13 +316,20 @@ def mxfp8_dequantize(qweight: torch.Tensor, scale: torch.Tensor,
     return _mx_dequantize("mxfp8_dequantize", qweight, scale, dtype, 1)
 
 
-def mxfp8_quantize_grouped(xs: torch.Tensor | Sequence[torch.Tensor]):
-    """Grouped MXFP8 of expert tensors sharing N, in one launch.
+def mxfp8_quantize_grouped(xs: torch.Tensor | Sequence[torch.Tensor], *, row_offsets=None,
+                           swizzled: bool = False):
+    """Grouped MXFP8 of expert weights sharing N, in one launch.
 
-    ``xs`` is a stacked [E, M, N] tensor (results [E, M, N] and [E, M, N/32])
-    or a sequence of contiguous [M_e, N] tensors (results concatenated along
-    rows: [sum M_e, N] and [sum M_e, N/32])."""
-    return _mx_quantize_grouped("mxfp8_quantize_grouped", xs, 1)
+    ``xs`` is one stacked tensor, [E, M, N] (results [E, M, N] and
+    [E, M, N/32]) or [M_total, N] with ``row_offsets`` (E + 1 rising row
+    offsets from 0 to M_total, as a list or an int64 tensor, on the host or on
+    the device); or a sequence of contiguous [M_e, N] tensors in separate
+    allocations (results concatenated along rows: [sum M_e, N] and
+    [sum M_e, N/32]). With ``swizzled=True`` (stacked tensors only) a third,
+    flat uint8 tensor holds each expert's scales in its own 128x4-tile
+    layout, expert after expert; when the offsets live on the device it is
+    sized by the upper bound of ``mxq_grouped_swizzled_scale_bytes_max``."""
+    return _mx_quantize_grouped("mxfp8", xs, 1, row_offsets, swizzled)
 
 
 def mxfp8_quantize_columnwise(x: torch.Tensor, *, rowwise: bool = False):
@@ -251,12 +344,12 @@ def mxfp8_quantize_columnwise(x: torch.Tensor, *, rowwise: bool = False):
     dt = _dtype_code(x.dtype)
     M, N, ld = _rows_view(x)
     dev = x.device
-    q_t = torch.empty((N, M), dtype=torch.uint8, device=dev)
-    s_t = torch.empty((N, (M + 31) // 32), dtype=torch.uint8, device=dev)
+    q_t = _empty((N, M), torch.uint8, dev)
+    s_t = _empty((N, (M + 31) // 32), torch.uint8, dev)
     q = s = None
     if rowwise:
-        q = torch.empty((M, N), dtype=torch.uint8, device=dev)
-        s = torch.empty((M, N // 32), dtype=torch.uint8, device=dev)
+        q = _empty((M, N), torch.uint8, dev)
+        s = _empty((M, N // 32), torch.uint8, dev)
     _check("mxfp8_quantize_columnwise",
            lib.mxfp8_quantize_columnwise(_ptr(x), dt, M, N, ld, _ptr(q_t), _ptr(s_t), _ptr(q),
                                          _ptr(s), _stream(x)))
@@ -283,10 +376,11 @@ def mxfp4_dequantize(packed: torch.Tensor, scale: torch.Tensor,
     return _mx_dequantize("mxfp4_dequantize", packed, scale, dtype, 2)
 
 
-def mxfp4_quantize_grouped(xs: torch.Tensor | Sequence[torch.Tensor]):
-    """Grouped MXFP4 of expert tensors sharing N, in one launch (layout as
-    :func:`mxfp8_quantize_grouped`, codes packed [.., N // 2])."""
-    return _mx_quantize_grouped("mxfp4_quantize_grouped", xs, 2)
+def mxfp4_quantize_grouped(xs: torch.Tensor | Sequence[torch.Tensor], *, row_offsets=None,
+                           swizzled: bool = False):
+    """Grouped MXFP4 of expert weights sharing N, in one launch (arguments
+    and layouts as :func:`mxfp8_quantize_grouped`, codes packed [.., N // 2])."""
+    return _mx_quantize_grouped("mxfp4", xs, 2, row_offsets, swizzled)
 
 
 def mx_fake_quantize(x: torch.Tensor, fmt: str = "mxfp4",
@@ -301,7 +395,7 @@ def mx_fake_quantize(x: torch.Tensor, fmt: str = "mxfp4",
     dt = _dtype_code(x.dtype)
     dtype = x.dtype if dtype is None else dtype
     M, N, ld = _rows_view(x)
-    y = torch.empty(x.shape, dtype=dtype, device=x.device)
+    y = _empty(x.shape, dtype, x.device)
     _check("mx_fake_quantize", lib.mx_fake_quantize(formats[fmt], _ptr(x), dt, M, N, ld, _ptr(y),
                                                     _dtype_code(dtype), _stream(x)))
     return y
@@ -331,7 +425,7 @@ def mxfp8_gemm(qa: torch.Tensor, sa_swizzled: torch.Tensor, qb: torch.Tensor,
         raise ValueError("swizzled scales are smaller than the operands need")
     if error_flag is not None and (error_flag.dtype != torch.int32 or not error_flag.is_cuda):
         raise TypeError("error_flag must be an int32 CUDA tensor")
-    d = torch.empty((M, N), dtype=dtype, device=qa.device)
+    d = _empty((M, N), dtype, qa.device)
     _check("mxfp8_gemm", lib.mxfp8_gemm(_ptr(qa), _ptr(sa_swizzled), _ptr(qb), _ptr(sb_swizzled),
                                         M, N, K, _ptr(d), _dtype_code(dtype), _ptr(error_flag),
                                         _stream(qa)))
@@ -345,9 +439,9 @@ def nvfp4_amax(x: torch.Tensor, workspace: torch.Tensor | None = None) -> torch.
     _require_cuda(x)
     dt = _dtype_code(x.dtype)
     M, N, ld = _rows_view(x)
-    out = torch.zeros((), dtype=torch.float32, device=x.device)
-    ws = workspace if workspace is not None else torch.empty(
-        nvfp4_workspace_bytes(M, N), dtype=torch.uint8, device=x.device)
+    out = _zeros((), torch.float32, x.device)
+    ws = workspace if workspace is not None else _empty(
+        nvfp4_workspace_bytes(M, N), torch.uint8, x.device)
     _check("nvfp4_amax", lib.nvfp4_amax(_ptr(x), dt, M, N, ld, _ptr(out), _ptr(ws),
                                         ws.numel() * ws.element_size(), _stream(x)))
     return out
@@ -366,8 +460,8 @@ def nvfp4_quantize(x: torch.Tensor, global_scale: torch.Tensor | None = None,
     dt = _dtype_code(x.dtype)
     M, N, ld = _rows_view(x)
     dev = x.device
-    packed = torch.empty((*x.shape[:-1], N // 2), dtype=torch.uint8, device=dev)
-    bs = torch.empty((*x.shape[:-1], N // 16), dtype=torch.uint8, device=dev)
+    packed = _empty((*x.shape[:-1], N // 2), torch.uint8, dev)
+    bs = _empty((*x.shape[:-1], N // 16), torch.uint8, dev)
     flags = 0
     if global_scale is not None:
         if global_scale.dtype != torch.float32 or global_scale.numel() != 1:
@@ -375,13 +469,13 @@ def nvfp4_quantize(x: torch.Tensor, global_scale: torch.Tensor | None = None,
         g = global_scale.to(dev)
         flags = NVFP4_GLOBAL_GIVEN
     else:
-        g = torch.empty((), dtype=torch.float32, device=dev)
+        g = _empty((), torch.float32, dev)
     if amax is not None and (amax.dtype != torch.float32 or amax.numel() != 1):
         raise TypeError("amax must be a single fp32 value")
     ws = None
     if global_scale is None and amax is None:
-        ws = workspace if workspace is not None else torch.empty(
-            nvfp4_workspace_bytes(M, N), dtype=torch.uint8, device=dev)
+        ws = workspace if workspace is not None else _empty(
+            nvfp4_workspace_bytes(M, N), torch.uint8, dev)
     _check("nvfp4_quantize",
            lib.nvfp4_quantize(_ptr(x), dt, M, N, ld, _ptr(packed), _ptr(bs), _ptr(g), _ptr(amax),
                               flags, _ptr(ws), 0 if ws is None else ws.numel() * ws.element_size(),
@@ -399,7 +493,7 @@ def _slice_array(slice_rows, M):
 def _sliced_workspace(n, dev, workspace):
     if workspace is not None:
         return workspace
-    return torch.empty(int(lib.mxq_nvfp4_sliced_workspace_bytes(n)), dtype=torch.uint8, device=dev)
+    return _empty(int(lib.mxq_nvfp4_sliced_workspace_bytes(n)), torch.uint8, dev)
 
 
 def nvfp4_amax_sliced(x: torch.Tensor, slice_rows: Sequence[int],
@@ -410,7 +504,7 @@ def nvfp4_amax_sliced(x: torch.Tensor, slice_rows: Sequence[int],
     dt = _dtype_code(x.dtype)
     M, N, ld = _rows_view(x)
     rows, S = _slice_array(slice_rows, M)
-    out = torch.zeros(S, dtype=torch.float32, device=x.device)
+    out = _zeros(S, torch.float32, x.device)
     ws = _sliced_workspace(S, x.device, workspace)
     _check("nvfp4_amax_sliced",
            lib.nvfp4_amax_sliced(_ptr(x), dt, M, N, ld, S, ctypes.cast(rows, ctypes.c_void_p),
@@ -435,8 +529,8 @@ def nvfp4_quantize_sliced(x: torch.Tensor, slice_rows: Sequence[int],
     M, N, ld = _rows_view(x)
     rows, S = _slice_array(slice_rows, M)
     dev = x.device
-    packed = torch.empty((*x.shape[:-1], N // 2), dtype=torch.uint8, device=dev)
-    bs = torch.empty((*x.shape[:-1], N // 16), dtype=torch.uint8, device=dev)
+    packed = _empty((*x.shape[:-1], N // 2), torch.uint8, dev)
+    bs = _empty((*x.shape[:-1], N // 16), torch.uint8, dev)
     flags = 0
     if global_scales is not None:
         if global_scales.dtype != torch.float32 or global_scales.numel() != S:
@@ -444,7 +538,7 @@ def nvfp4_quantize_sliced(x: torch.Tensor, slice_rows: Sequence[int],
         g = global_scales.to(dev).contiguous()
         flags = NVFP4_GLOBAL_GIVEN
     else:
-        g = torch.zeros(S, dtype=torch.float32, device=dev)
+        g = _zeros(S, torch.float32, dev)
     if amax is not None:
         if amax.dtype != torch.float32 or amax.numel() != S:
             raise TypeError("amax must be fp32 with one value per slice")
@@ -489,7 +583,7 @@ def nvfp4_dequantize(packed: torch.Tensor, block_scale: torch.Tensor, global_sca
     M = packed.numel() * 2 // N if N else 0
     if block_scale.numel() != M * (N // 16):
         raise ValueError("block_scale does not match packed")
-    y = torch.empty((*packed.shape[:-1], N), dtype=dtype, device=packed.device)
+    y = _empty((*packed.shape[:-1], N), dtype, packed.device)
     _check("nvfp4_dequantize",
            lib.nvfp4_dequantize(_ptr(packed), _ptr(block_scale), _ptr(global_scale), M, N, _ptr(y),
                                 _dtype_code(dtype), _stream(packed)))

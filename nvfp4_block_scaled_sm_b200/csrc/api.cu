@@ -52,4 +52,10 @@ int64_t mxq_swizzled_scale_bytes(int64_t M, int64_t S) {
   return ((M + 127) / 128 * 128) * ((S + 3) / 4 * 4);
 }
 
+int64_t mxq_grouped_swizzled_scale_bytes_max(int32_t E, int64_t M_total, int64_t S) {
+  if (E < 0 || M_total < 0 || S < 0) return -1;
+  // each expert pads its rows to a multiple of 128, adding at most 127 rows
+  return ((M_total + 127 * int64_t(E)) / 128 * 128) * ((S + 3) / 4 * 4);
+}
+
 }  // extern "C"

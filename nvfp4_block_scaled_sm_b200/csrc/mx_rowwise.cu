@@ -101,10 +101,72 @@ struct QuantArgs {
   uint64_t pad_a;        // swizzle padding entries right of the real scale columns
   uint64_t pad_b;        // swizzle padding entries below the real rows
   int32_t E;             // experts
+  const int64_t* offs;   // device row offsets [E + 1] of a stacked tensor (SWZ == kSwzExperts)
+  uint64_t swz_cap;      // bytes of the swizzled output (SWZ == kSwzExperts)
   const void* x[MAXE];
   uint64_t gbase[MAXE + 1];  // first output group of expert e; gbase[E] = all groups
   uint32_t tbase[MAXE + 1];  // first CTA of expert e; tbase[E] = grid size
 };
+
+// Swizzled-scale modes of mx_quant_kernel: none; one 128x4-tile layout for
+// the whole [M, S] scale; one layout per expert of a stacked tensor, expert
+// e's block starting where expert e-1's 128-row-padded block ends.
+constexpr int kSwzNone = 0;
+constexpr int kSwzTensor = 1;
+constexpr int kSwzExperts = 2;
+
+// Row offsets of a stacked tensor's experts, read into shared memory by one
+// warp: off[e] = the device offsets clamped into a non-decreasing sequence
+// from off[0] = 0 to off[E] = M (so no write can leave the layout, whatever
+// the offsets hold), and pb[e] = first row of expert e in the per-expert
+// padded layout, pb[e + 1] = pb[e] + ceil((off[e + 1] - off[e]) / 128) * 128.
+__device__ __noinline__ void load_expert_rows(const int64_t* __restrict__ g_off, int E,
+                                              int64_t M, int64_t* off, int64_t* pb) {
+  if (threadIdx.x < 32) {
+    const int lane = threadIdx.x;
+    int64_t carry_off = 0, carry_pb = 0;
+    for (int base = 0; base <= E; base += 32) {
+      const int e = base + lane;
+      int64_t v = 0;
+      if (e > 0 && e < E) v = g_off[e];
+      if (e >= E) v = M;
+      v = v < 0 ? 0 : (v > M ? M : v);
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int64_t t = __shfl_up_sync(kFull, v, o);
+        if (lane >= o) v = t > v ? t : v;
+      }
+      v = carry_off > v ? carry_off : v;
+      int64_t prev = __shfl_up_sync(kFull, v, 1);
+      if (lane == 0) prev = carry_off;
+      int64_t d = (e == 0 || e > E) ? 0 : ((v - prev + 127) & ~int64_t(127));
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int64_t t = __shfl_up_sync(kFull, d, o);
+        if (lane >= o) d += t;
+      }
+      d += carry_pb;
+      if (e <= E) {
+        off[e] = v;
+        pb[e] = d;
+      }
+      carry_off = __shfl_sync(kFull, v, 31);
+      carry_pb = __shfl_sync(kFull, d, 31);
+    }
+  }
+  __syncthreads();
+}
+
+// The expert holding row r (0 <= r < off[E]): the largest e < E with
+// off[e] <= r, which skips empty experts.
+__device__ __forceinline__ int expert_of_row(const int64_t* off, int E, int64_t r) {
+  int lo = 0, hi = E;  // invariant: off[lo] <= r < off[hi]
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (off[mid] <= r) lo = mid; else hi = mid;
+  }
+  return lo;
+}
 
 // Zero bytes of the swizzled layout outside the real [M, S] scales.
 template <int MAXE>
@@ -128,7 +190,30 @@ __device__ __forceinline__ void fill_swizzle_padding(const QuantArgs<MAXE>& a) {
   }
 }
 
-template <typename InT, bool V8, bool STRIDED, bool SWZ, int MAXE, int FMT>
+// Per-expert swizzled layout (kSwzExperts): zero padding of the experts whose
+// last group lies in this CTA's groups [tg0, tg0 + nt): the rows from the
+// expert's end up to its next multiple of 128, all Sp columns.
+template <int MAXE>
+__device__ __forceinline__ void fill_expert_row_padding(const QuantArgs<MAXE>& a, const int64_t* off,
+                                                        const int64_t* pb, uint64_t tg0,
+                                                        uint32_t nt) {
+  const uint64_t S = a.S;
+  const int64_t r0 = int64_t(tg0 / S), r1 = int64_t((tg0 + nt - 1) / S);
+  const uint32_t Sp = a.Sp4 * 4;
+  for (int e = expert_of_row(off, a.E, r0); e < a.E && off[e] <= r1; e++) {
+    const int64_t m = off[e + 1] - off[e];
+    if (m == 0) continue;
+    const uint64_t last = uint64_t(off[e + 1]) * S - 1;  // the expert's last group
+    if (last < tg0 || last >= tg0 + nt) continue;
+    const uint64_t rows = uint64_t(pb[e + 1] - pb[e] - m);
+    for (uint64_t p = threadIdx.x; p < rows * Sp; p += kThreads) {
+      const uint64_t dst = swz_offset(uint64_t(pb[e] + m) + p / Sp, uint32_t(p % Sp), a.Sp4);
+      if (dst < a.swz_cap) st_u8(a.swz + dst, 0);
+    }
+  }
+}
+
+template <typename InT, bool V8, bool STRIDED, int SWZ, int MAXE, int FMT>
 __global__ void __launch_bounds__(kThreads)
 mx_quant_kernel(const __grid_constant__ QuantArgs<MAXE> a) {
   pdl_enter();
@@ -156,9 +241,10 @@ mx_quant_kernel(const __grid_constant__ QuantArgs<MAXE> a) {
   uint8_t* st = a.scale + a.gbase[e] + tg0;
 
   // row / column of the lane's group (strided input, swizzled scales)
+  constexpr bool kRC = STRIDED || SWZ != kSwzNone;
   uint64_t r = 0;
   uint32_t c = 0;
-  if constexpr (STRIDED || SWZ) {
+  if constexpr (kRC) {
     const uint64_t g = tg0 + lg0;
     r = a.rows.div(g);
     c = uint32_t(g - r * a.S);
@@ -169,7 +255,7 @@ mx_quant_kernel(const __grid_constant__ QuantArgs<MAXE> a) {
   for (int u = 0; u < kSteps; u++) {
     rr[u] = r;
     cc[u] = c;
-    if constexpr (STRIDED || SWZ) {
+    if constexpr (kRC) {
       c += kGroupsPerStep;
       while (c >= a.S) {
         c -= a.S;
@@ -191,6 +277,12 @@ mx_quant_kernel(const __grid_constant__ QuantArgs<MAXE> a) {
     if (full || lg < nt) v[u].template load<V8>(p); else v[u].zero();
   }
 
+  // experts' row ranges and padded bases (while the loads are in flight)
+  extern __shared__ int64_t s_rows[];
+  int64_t* off = s_rows;
+  int64_t* pb = s_rows + (a.E + 1);
+  if constexpr (SWZ == kSwzExperts) load_expert_rows(a.offs, a.E, int64_t(a.M), off, pb);
+
 #pragma unroll
   for (int u = 0; u < kSteps; u++) {
     const uint32_t lg = lg0 + u * kGroupsPerStep;
@@ -207,11 +299,24 @@ mx_quant_kernel(const __grid_constant__ QuantArgs<MAXE> a) {
       else st_v2(qt + lg * CB, o2);
       if (half == 0) {
         st_u8(st + lg, b);
-        if constexpr (SWZ) st_u8(a.swz + swz_offset(rr[u], cc[u], a.Sp4), b);
+        if constexpr (SWZ == kSwzTensor) st_u8(a.swz + swz_offset(rr[u], cc[u], a.Sp4), b);
+        if constexpr (SWZ == kSwzExperts) {
+          const int ex = expert_of_row(off, a.E, int64_t(rr[u]));
+          const uint64_t pr = uint64_t(pb[ex] + (int64_t(rr[u]) - off[ex]));  // padded row
+          const uint64_t dst = swz_offset(pr, cc[u], a.Sp4);
+          if (dst < a.swz_cap) st_u8(a.swz + dst, b);
+          if (cc[u] == a.S - 1) {  // the row's padding columns
+            for (uint32_t cp = a.S; cp < a.Sp4 * 4; cp++) {
+              const uint64_t dp = swz_offset(pr, cp, a.Sp4);
+              if (dp < a.swz_cap) st_u8(a.swz + dp, 0);
+            }
+          }
+        }
       }
     }
   }
-  if constexpr (SWZ) fill_swizzle_padding(a);
+  if constexpr (SWZ == kSwzTensor) fill_swizzle_padding(a);
+  if constexpr (SWZ == kSwzExperts) fill_expert_row_padding(a, off, pb, tg0, nt);
 }
 
 // ------------------------------------------------------- decode and store
@@ -441,20 +546,23 @@ mx_fake_quant_kernel(const __grid_constant__ FakeArgs a) {
 
 inline bool aligned32(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 31u) == 0; }
 
-template <typename InT, bool V8, bool STRIDED, bool SWZ, int MAXE, int FMT>
+template <typename InT, bool V8, bool STRIDED, int SWZ, int MAXE, int FMT>
 mxq_status launch_quant(const QuantArgs<MAXE>& a, uint32_t grid, cudaStream_t stream) {
-  return launched(launch_pdl(mx_quant_kernel<InT, V8, STRIDED, SWZ, MAXE, FMT>, grid, stream, a));
+  // the per-expert swizzle keeps the experts' row offsets in shared memory
+  const size_t smem = SWZ == kSwzExperts ? 2 * sizeof(int64_t) * size_t(a.E + 1) : 0;
+  return launched(launch_pdl_ex(mx_quant_kernel<InT, V8, STRIDED, SWZ, MAXE, FMT>, grid, kThreads,
+                                smem, stream, a));
 }
 
 template <typename InT, bool V8, int FMT>
 mxq_status dispatch_single(const QuantArgs<1>& a, bool strided, bool swz, uint32_t grid,
                            cudaStream_t s) {
   if (strided) {
-    return swz ? launch_quant<InT, V8, true, true, 1, FMT>(a, grid, s)
-               : launch_quant<InT, V8, true, false, 1, FMT>(a, grid, s);
+    return swz ? launch_quant<InT, V8, true, kSwzTensor, 1, FMT>(a, grid, s)
+               : launch_quant<InT, V8, true, kSwzNone, 1, FMT>(a, grid, s);
   }
-  return swz ? launch_quant<InT, V8, false, true, 1, FMT>(a, grid, s)
-             : launch_quant<InT, V8, false, false, 1, FMT>(a, grid, s);
+  return swz ? launch_quant<InT, V8, false, kSwzTensor, 1, FMT>(a, grid, s)
+             : launch_quant<InT, V8, false, kSwzNone, 1, FMT>(a, grid, s);
 }
 
 template <int FMT>
@@ -552,11 +660,11 @@ mxq_status grouped_impl(int32_t E, const void* const* xs, const int64_t* rows, i
   a.S = uint32_t(S);
   const uint32_t grid = uint32_t(tiles);
   if (dt == MXQ_BF16) {
-    return v8 ? launch_quant<uint16_t, true, false, false, MAXE, FMT>(a, grid, stream)
-              : launch_quant<uint16_t, false, false, false, MAXE, FMT>(a, grid, stream);
+    return v8 ? launch_quant<uint16_t, true, false, kSwzNone, MAXE, FMT>(a, grid, stream)
+              : launch_quant<uint16_t, false, false, kSwzNone, MAXE, FMT>(a, grid, stream);
   }
-  return v8 ? launch_quant<float, true, false, false, MAXE, FMT>(a, grid, stream)
-            : launch_quant<float, false, false, false, MAXE, FMT>(a, grid, stream);
+  return v8 ? launch_quant<float, true, false, kSwzNone, MAXE, FMT>(a, grid, stream)
+            : launch_quant<float, false, false, kSwzNone, MAXE, FMT>(a, grid, stream);
 }
 
 template <int FMT>
@@ -581,6 +689,61 @@ mxq_status grouped_entry(int32_t E, const void* const* xs, const int64_t* rows, 
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (E <= 64) return grouped_impl<64, FMT>(E, xs, rows, N, dt, q, scale, s);
   return grouped_impl<MXQ_GROUPED_MAX_EXPERTS, FMT>(E, xs, rows, N, dt, q, scale, s);
+}
+
+// Grouped quantize of a stacked tensor: the compact outputs are those of the
+// flattened [M, N] call (groups never cross rows, so expert boundaries change
+// no byte of them); the device row offsets place each expert's swizzled scale
+// block.
+template <int FMT>
+mxq_status grouped_stacked_entry(const void* x, int dt, int32_t E, const int64_t* row_offsets,
+                                 int64_t M, int64_t N, uint8_t* q, uint8_t* scale,
+                                 uint8_t* scale_swz, int64_t swz_bytes, mxq_stream_t stream) {
+  if (!valid_dtype(dt)) return MXQ_ERR_DTYPE;
+  if (E < 1 || E > MXQ_GROUPED_MAX_EXPERTS || M < 0 || N < 0 || N % 32 != 0) return MXQ_ERR_SHAPE;
+  if (!row_offsets) return MXQ_ERR_NULL;
+  if (reinterpret_cast<uintptr_t>(row_offsets) & 7u) return MXQ_ERR_ALIGN;
+  if (scale_swz && swz_bytes < 0) return MXQ_ERR_SHAPE;
+  if (M == 0 || N == 0) return MXQ_OK;
+  if (!x || !q || !scale) return MXQ_ERR_NULL;
+  const uint64_t S = uint64_t(N) / 32;
+  const uint64_t groups = uint64_t(M) * S;
+  const uint64_t tiles = (groups + kGroupsPerTile - 1) / kGroupsPerTile;
+  if (S > 0xffffffffull || tiles > 0x7fffffffull) return MXQ_ERR_SHAPE;
+  const uint64_t row_bytes = uint64_t(N) * elem_size(dt);
+  if (!aligned16(x) || row_bytes % 16 != 0 || !aligned16(q)) return MXQ_ERR_ALIGN;
+  QuantArgs<1> a{};
+  a.q = q;
+  a.scale = scale;
+  a.swz = scale_swz;
+  a.ld = N;
+  a.rows = FastDiv::make(uint32_t(S));
+  a.S = uint32_t(S);
+  a.Sp4 = uint32_t((S + 3) / 4);
+  a.M = uint64_t(M);
+  a.E = E;
+  a.offs = row_offsets;
+  a.swz_cap = scale_swz ? uint64_t(swz_bytes) : 0;
+  a.x[0] = x;
+  a.gbase[0] = 0;
+  a.gbase[1] = groups;
+  a.tbase[0] = 0;
+  a.tbase[1] = uint32_t(tiles);
+  const bool v8 = aligned32(x) && row_bytes % 32 == 0;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const uint32_t grid = uint32_t(tiles);
+  if (scale_swz == nullptr) {
+    if (dt == MXQ_BF16)
+      return v8 ? launch_quant<uint16_t, true, false, kSwzNone, 1, FMT>(a, grid, s)
+                : launch_quant<uint16_t, false, false, kSwzNone, 1, FMT>(a, grid, s);
+    return v8 ? launch_quant<float, true, false, kSwzNone, 1, FMT>(a, grid, s)
+              : launch_quant<float, false, false, kSwzNone, 1, FMT>(a, grid, s);
+  }
+  if (dt == MXQ_BF16)
+    return v8 ? launch_quant<uint16_t, true, false, kSwzExperts, 1, FMT>(a, grid, s)
+              : launch_quant<uint16_t, false, false, kSwzExperts, 1, FMT>(a, grid, s);
+  return v8 ? launch_quant<float, true, false, kSwzExperts, 1, FMT>(a, grid, s)
+            : launch_quant<float, false, false, kSwzExperts, 1, FMT>(a, grid, s);
 }
 
 template <typename InT, typename OutT, int FMT>
@@ -620,9 +783,25 @@ mxq_status mxfp8_dequantize(const uint8_t* qweight, const uint8_t* scale, int64_
   return mxq::dequantize_impl<mxq::kE4M3>(qweight, scale, M, N, y, out_dt, stream);
 }
 
-mxq_status mxfp8_quantize_grouped(int32_t E, const void* const* xs, const int64_t* rows,
-                                  int64_t N, int dt, uint8_t* qweight, uint8_t* scale,
+mxq_status mxfp8_quantize_grouped(const void* x, int dt, int32_t E, const int64_t* row_offsets,
+                                  int64_t M_total, int64_t N, uint8_t* qweight, uint8_t* scale,
                                   mxq_stream_t stream) {
+  return mxq::grouped_stacked_entry<mxq::kE4M3>(x, dt, E, row_offsets, M_total, N, qweight, scale,
+                                                nullptr, 0, stream);
+}
+
+mxq_status mxfp8_quantize_grouped_swizzled(const void* x, int dt, int32_t E,
+                                           const int64_t* row_offsets, int64_t M_total, int64_t N,
+                                           uint8_t* qweight, uint8_t* scale, uint8_t* scale_swz,
+                                           int64_t swz_bytes, mxq_stream_t stream) {
+  if (!scale_swz) return MXQ_ERR_NULL;
+  return mxq::grouped_stacked_entry<mxq::kE4M3>(x, dt, E, row_offsets, M_total, N, qweight, scale,
+                                                scale_swz, swz_bytes, stream);
+}
+
+mxq_status mxfp8_quantize_grouped_ptrs(int32_t E, const void* const* xs, const int64_t* rows,
+                                       int64_t N, int dt, uint8_t* qweight, uint8_t* scale,
+                                       mxq_stream_t stream) {
   return mxq::grouped_entry<mxq::kE4M3>(E, xs, rows, N, dt, qweight, scale, stream);
 }
 
@@ -637,9 +816,25 @@ mxq_status mxfp4_dequantize(const uint8_t* packed, const uint8_t* scale, int64_t
   return mxq::dequantize_impl<mxq::kE2M1>(packed, scale, M, N, y, out_dt, stream);
 }
 
-mxq_status mxfp4_quantize_grouped(int32_t E, const void* const* xs, const int64_t* rows,
-                                  int64_t N, int dt, uint8_t* packed, uint8_t* scale,
+mxq_status mxfp4_quantize_grouped(const void* x, int dt, int32_t E, const int64_t* row_offsets,
+                                  int64_t M_total, int64_t N, uint8_t* packed, uint8_t* scale,
                                   mxq_stream_t stream) {
+  return mxq::grouped_stacked_entry<mxq::kE2M1>(x, dt, E, row_offsets, M_total, N, packed, scale,
+                                                nullptr, 0, stream);
+}
+
+mxq_status mxfp4_quantize_grouped_swizzled(const void* x, int dt, int32_t E,
+                                           const int64_t* row_offsets, int64_t M_total, int64_t N,
+                                           uint8_t* packed, uint8_t* scale, uint8_t* scale_swz,
+                                           int64_t swz_bytes, mxq_stream_t stream) {
+  if (!scale_swz) return MXQ_ERR_NULL;
+  return mxq::grouped_stacked_entry<mxq::kE2M1>(x, dt, E, row_offsets, M_total, N, packed, scale,
+                                                scale_swz, swz_bytes, stream);
+}
+
+mxq_status mxfp4_quantize_grouped_ptrs(int32_t E, const void* const* xs, const int64_t* rows,
+                                       int64_t N, int dt, uint8_t* packed, uint8_t* scale,
+                                       mxq_stream_t stream) {
   return mxq::grouped_entry<mxq::kE2M1>(E, xs, rows, N, dt, packed, scale, stream);
 }
 

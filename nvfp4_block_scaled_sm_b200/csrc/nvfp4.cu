@@ -47,6 +47,8 @@
 // Work split of the block pass: a lane owns one block (16 elements, one
 // 256-bit load of bf16), writes 8 packed bytes and one scale byte, so a warp
 // reads 1 KiB and writes 256 + 32 contiguous bytes per step.
+#include <cuda.h>
+
 #include "common.cuh"
 
 namespace mxq {
@@ -896,12 +898,51 @@ constexpr int kNoallocPartials = kMaxPartials;  // 2048 floats = 8 KiB per devic
 static __device__ __align__(256) float g_noalloc_partials[kNoallocPartials];
 
 constexpr int kMaxDevices = 256;
-std::mutex g_noalloc_mu;
-float* g_noalloc_ptr[kMaxDevices] = {};  // device address of the array, per device
 
-// Device address of g_noalloc_partials on the current device. The first call
-// on a device looks it up (cudaGetSymbolAddress, with that device current);
-// later calls reuse it.
+// The array's device address is cached per device together with the id of
+// the CUDA context it was looked up in. A context that is destroyed and
+// created again (cudaDeviceReset, or a driver-API context of the caller's)
+// reloads the library's module, and the array may then sit elsewhere: a
+// changed context id makes the next call look the address up again.
+struct NoallocSlot {
+  unsigned long long ctx_id;  // 0: nothing cached
+  float* ptr;
+};
+std::mutex g_noalloc_mu;
+NoallocSlot g_noalloc_slot[kMaxDevices] = {};
+
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+
+// Id of the calling thread's current CUDA context (driver entry points
+// fetched through the runtime, so the library needs no link against the
+// driver library); false when there is none yet or the driver lacks the call.
+bool current_context_id(unsigned long long* id) {
+  static std::once_flag once;
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &f, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess && q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<CtxGetCurrentFn>(f);
+    f = nullptr;
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetId", &f, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess && q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<CtxGetIdFn>(f);
+    cudaGetLastError();
+  });
+  if (!get_current || !get_id) return false;
+  CUcontext ctx = nullptr;
+  if (get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return false;
+  return get_id(ctx, id) == CUDA_SUCCESS && *id != 0;
+}
+
+// Device address of g_noalloc_partials in the current device's context. The
+// first call on a device (and the first after that device's context changed)
+// looks it up with cudaGetSymbolAddress, with that device current; later
+// calls reuse it. Without a context id to key on, every call looks it up.
 mxq_status noalloc_scratch(float** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -911,16 +952,22 @@ mxq_status noalloc_scratch(float** out) {
   }
   if (dev < 0 || dev >= kMaxDevices) return MXQ_ERR_ARG;
   std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  if (g_noalloc_ptr[dev] == nullptr) {
-    void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_noalloc_partials);
-    if (e != cudaSuccess) {
-      record_cuda_error(e);
-      return MXQ_ERR_CUDA;
-    }
-    g_noalloc_ptr[dev] = static_cast<float*>(p);
+  NoallocSlot& slot = g_noalloc_slot[dev];
+  unsigned long long id = 0;
+  if (slot.ptr != nullptr && current_context_id(&id) && id == slot.ctx_id) {
+    *out = slot.ptr;
+    return MXQ_OK;
   }
-  *out = g_noalloc_ptr[dev];
+  void* p = nullptr;
+  e = cudaGetSymbolAddress(&p, g_noalloc_partials);
+  if (e != cudaSuccess) {
+    record_cuda_error(e);
+    return MXQ_ERR_CUDA;
+  }
+  // the lookup made the device's context current if it was not yet
+  slot.ptr = current_context_id(&id) ? static_cast<float*>(p) : nullptr;
+  slot.ctx_id = slot.ptr ? id : 0;
+  *out = static_cast<float*>(p);
   return MXQ_OK;
 }
 

@@ -240,15 +240,26 @@ def swizzle_scales(s: np.ndarray) -> np.ndarray:
     return out
 
 
-def mxfp8_quantize_grouped(xs):
-    """Grouped MXFP8 of a list of expert inputs [M_e, N] (shared N): each
-    expert quantized on its own, results concatenated along rows."""
+def _grouped(quantize, xs, swizzled):
     qs, ss = [], []
     for x in xs:
-        q, s = mxfp8_quantize(x)
+        q, s = quantize(x)
         qs.append(q)
         ss.append(s)
-    return np.concatenate(qs, 0), np.concatenate(ss, 0)
+    out = (np.concatenate(qs, 0), np.concatenate(ss, 0))
+    if swizzled:
+        out += (np.concatenate([swizzle_scales(s) for s in ss]),)
+    return out
+
+
+def mxfp8_quantize_grouped(xs, swizzled: bool = False):
+    """Grouped MXFP8 of a list of expert inputs [M_e, N] (shared N): each
+    expert quantized on its own, results concatenated along rows. With
+    ``swizzled``, also each expert's scales in its own 128x4-tile layout
+    (``swizzle_scales`` of that expert's compact scales), the experts' blocks
+    concatenated in expert order, as a grouped block-scaled GEMM reads one
+    scale matrix per expert."""
+    return _grouped(mxfp8_quantize, xs, swizzled)
 
 
 # -------------------------------------------------------------------- MXFP4
@@ -265,6 +276,11 @@ def mxfp4_quantize(x: np.ndarray):
     s = np.empty((M, N // 32), np.uint8)
     _check(lib().orc_mxfp4_quantize(_ptr(a), dt, M, N, N, _ptr(packed), _ptr(s)), "mxfp4_quantize")
     return packed, s
+
+
+def mxfp4_quantize_grouped(xs, swizzled: bool = False):
+    """Grouped MXFP4: as :func:`mxfp8_quantize_grouped` with MXFP4 codes."""
+    return _grouped(mxfp4_quantize, xs, swizzled)
 
 
 def mxfp4_dequantize(packed: np.ndarray, s: np.ndarray, out: str = "bf16") -> np.ndarray:

@@ -18,3 +18,23 @@ def orc():
     import oracle
     oracle.build()
     return oracle
+
+
+@pytest.fixture(autouse=True)
+def guard_bands(request):
+    """For every GPU test: the binding allocates each output and workspace
+    between canary bands (tests/gpu_util.GuardedAllocator), and the bands are
+    checked when the test ends, so a write past either end of any output
+    fails the test."""
+    if request.node.get_closest_marker("gpu") is None:
+        yield None
+        return
+    import nvfp4_block_scaled_sm_b200 as mxq
+    from gpu_util import GuardedAllocator
+    alloc = GuardedAllocator()
+    prev = mxq.set_output_allocator(alloc)
+    try:
+        yield alloc
+    finally:
+        mxq.set_output_allocator(prev)
+    alloc.check()

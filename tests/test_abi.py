@@ -45,7 +45,7 @@ def test_library_exports_every_declared_symbol():
 
 
 def test_version_and_strings():
-    assert mxq.lib.mxq_abi_version() == 1
+    assert mxq.lib.mxq_abi_version() == 2
     for s in range(8):
         assert mxq.lib.mxq_status_string(s)
     assert mxq.lib.mxq_status_string(99) == b"unknown status"
@@ -103,9 +103,9 @@ def test_mxfp4_validation():
     assert L.mxfp4_dequantize(A, A, 4, 64, A + 2, 0, None) == ALIGN
     rows = (ctypes.c_int64 * 2)(4, 0)
     ptrs = (ctypes.c_void_p * 2)(A, None)
-    assert L.mxfp4_quantize_grouped(0, ptrs, rows, 64, 0, A, A, None) == SHAPE
-    assert L.mxfp4_quantize_grouped(2, ptrs, rows, 40, 0, A, A, None) == SHAPE
-    assert L.mxfp4_quantize_grouped(2, ptrs, rows, 64, 0, None, A, None) == NULL
+    assert L.mxfp4_quantize_grouped_ptrs(0, ptrs, rows, 64, 0, A, A, None) == SHAPE
+    assert L.mxfp4_quantize_grouped_ptrs(2, ptrs, rows, 40, 0, A, A, None) == SHAPE
+    assert L.mxfp4_quantize_grouped_ptrs(2, ptrs, rows, 64, 0, None, A, None) == NULL
 
 
 def test_fake_quantize_validation():
@@ -124,26 +124,26 @@ def test_fake_quantize_validation():
     assert L.mx_fake_quantize(0, None, 1, 0, 64, 64, None, 1, None) == OK
 
 
-def test_grouped_validation():
+def test_grouped_ptrs_validation():
     L = mxq.lib
     ptrs = (ctypes.c_void_p * 3)(A, A, A)
     rows = (ctypes.c_int64 * 3)(4, 0, 2)
     P, R = ctypes.cast(ptrs, ctypes.c_void_p), ctypes.cast(rows, ctypes.c_void_p)
-    assert L.mxfp8_quantize_grouped(0, P, R, 64, 0, A, A, None) == SHAPE
-    assert L.mxfp8_quantize_grouped(1025, P, R, 64, 0, A, A, None) == SHAPE
-    assert L.mxfp8_quantize_grouped(3, P, R, 48, 0, A, A, None) == SHAPE
-    assert L.mxfp8_quantize_grouped(3, P, R, 64, 5, A, A, None) == DTYPE
-    assert L.mxfp8_quantize_grouped(3, None, R, 64, 0, A, A, None) == NULL
-    assert L.mxfp8_quantize_grouped(3, P, R, 64, 0, None, A, None) == NULL
-    assert L.mxfp8_quantize_grouped(3, P, R, 64, 0, A + 1, A, None) == ALIGN
+    assert L.mxfp8_quantize_grouped_ptrs(0, P, R, 64, 0, A, A, None) == SHAPE
+    assert L.mxfp8_quantize_grouped_ptrs(1025, P, R, 64, 0, A, A, None) == SHAPE
+    assert L.mxfp8_quantize_grouped_ptrs(3, P, R, 48, 0, A, A, None) == SHAPE
+    assert L.mxfp8_quantize_grouped_ptrs(3, P, R, 64, 5, A, A, None) == DTYPE
+    assert L.mxfp8_quantize_grouped_ptrs(3, None, R, 64, 0, A, A, None) == NULL
+    assert L.mxfp8_quantize_grouped_ptrs(3, P, R, 64, 0, None, A, None) == NULL
+    assert L.mxfp8_quantize_grouped_ptrs(3, P, R, 64, 0, A + 1, A, None) == ALIGN
     bad_rows = (ctypes.c_int64 * 3)(4, -1, 2)
-    assert L.mxfp8_quantize_grouped(3, P, ctypes.cast(bad_rows, ctypes.c_void_p), 64, 0, A, A,
+    assert L.mxfp8_quantize_grouped_ptrs(3, P, ctypes.cast(bad_rows, ctypes.c_void_p), 64, 0, A, A,
                                     None) == SHAPE
     mis = (ctypes.c_void_p * 3)(A, A, A + 8)
-    assert L.mxfp8_quantize_grouped(3, ctypes.cast(mis, ctypes.c_void_p), R, 64, 0, A, A,
+    assert L.mxfp8_quantize_grouped_ptrs(3, ctypes.cast(mis, ctypes.c_void_p), R, 64, 0, A, A,
                                     None) == ALIGN
     zero_rows = (ctypes.c_int64 * 3)(0, 0, 0)
-    assert L.mxfp8_quantize_grouped(3, P, ctypes.cast(zero_rows, ctypes.c_void_p), 64, 0, None,
+    assert L.mxfp8_quantize_grouped_ptrs(3, P, ctypes.cast(zero_rows, ctypes.c_void_p), 64, 0, None,
                                     None, None) == OK
 
 
@@ -151,8 +151,47 @@ def test_grouped_null_pointer_only_matters_for_nonempty_expert():
     L = mxq.lib
     rows = (ctypes.c_int64 * 2)(4, 0)
     ptrs = (ctypes.c_void_p * 2)(None, A)
-    assert L.mxfp8_quantize_grouped(2, ctypes.cast(ptrs, ctypes.c_void_p),
-                                    ctypes.cast(rows, ctypes.c_void_p), 64, 0, A, A, None) == NULL
+    assert L.mxfp8_quantize_grouped_ptrs(2, ctypes.cast(ptrs, ctypes.c_void_p),
+                                         ctypes.cast(rows, ctypes.c_void_p), 64, 0, A, A,
+                                         None) == NULL
+
+
+def test_grouped_stacked_validation():
+    L = mxq.lib
+    O = A + 0x100      # fake device row offsets (never read on the host)
+    for G in (L.mxfp8_quantize_grouped, L.mxfp4_quantize_grouped):
+        assert G(A, 0, 0, O, 64, 64, A, A, None) == SHAPE
+        assert G(A, 0, 1025, O, 64, 64, A, A, None) == SHAPE
+        assert G(A, 0, 4, O, -1, 64, A, A, None) == SHAPE
+        assert G(A, 0, 4, O, 64, 48, A, A, None) == SHAPE
+        assert G(A, 6, 4, O, 64, 64, A, A, None) == DTYPE
+        assert G(A, 0, 4, None, 64, 64, A, A, None) == NULL
+        assert G(A, 0, 4, O + 4, 64, 64, A, A, None) == ALIGN
+        assert G(None, 0, 4, O, 64, 64, A, A, None) == NULL
+        assert G(A, 0, 4, O, 64, 64, None, A, None) == NULL
+        assert G(A, 0, 4, O, 64, 64, A, None, None) == NULL
+        assert G(A + 2, 0, 4, O, 64, 64, A, A, None) == ALIGN
+        assert G(A, 0, 4, O, 64, 64, A + 8, A, None) == ALIGN
+        assert G(None, 0, 4, O, 0, 64, None, None, None) == OK
+    for G in (L.mxfp8_quantize_grouped_swizzled, L.mxfp4_quantize_grouped_swizzled):
+        assert G(A, 0, 4, O, 64, 64, A, A, None, 4096, None) == NULL
+        assert G(A, 0, 4, O, 64, 64, A, A, A, -1, None) == SHAPE
+        assert G(A, 0, 4, None, 64, 64, A, A, A, 4096, None) == NULL
+        assert G(None, 0, 4, O, 0, 64, None, None, A, 0, None) == OK
+
+
+def test_grouped_swizzled_bound():
+    B = mxq.lib.mxq_grouped_swizzled_scale_bytes_max
+    assert B(1, 100, 7) == 128 * 8
+    assert B(64, 64 * 2048, 224) == (64 * 2048 + 127 * 64) // 128 * 128 * 224
+    assert B(3, 1, 4) == 256 * 4           # (1 + 381) // 128 = 2 tiles of rows
+    assert B(-1, 4, 4) == -1 and B(1, -4, 4) == -1
+    # the bound covers every split of M_total rows into E experts
+    import itertools
+    for E in (1, 2, 3):
+        for rows in itertools.product(range(0, 300, 37), repeat=E):
+            need = sum(mxq.swizzled_scale_bytes(r, 5) for r in rows)
+            assert need <= B(E, sum(rows), 5)
 
 
 def test_nvfp4_validation():

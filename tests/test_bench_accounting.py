@@ -39,3 +39,27 @@ def test_headline_step_bytes():
     quantize with swizzled scales and 355,991,552 B for the dequantize."""
     assert bench.mxfp8_quant_bytes(16384, 7168) == 359_661_568
     assert bench.mxfp8_dequant_bytes(16384, 7168) == 355_991_552
+
+
+def test_cpu_baseline_chunks_equal_one_call():
+    """The benchmark's multi-core oracle leg (row chunks on threads, each a
+    single-threaded oracle call) gives the bytes of one call over all rows."""
+    import numpy as np
+
+    import oracle
+    import workloads as W
+    x = W.activation(seed=3, M=300, N=256)
+    parts = bench.oracle_rows_parallel(bench.oracle_round_trip, x, 4)
+    q, s, z, y = (np.concatenate([p[i] for p in parts]) for i in range(4))
+    qo, so = oracle.mxfp8_quantize(x)
+    assert np.array_equal(q, qo) and np.array_equal(s, so)
+    assert np.array_equal(y, oracle.mxfp8_dequantize(qo, so, out="bf16"))
+    # 128-row chunks: each chunk's swizzled block is a slice of the whole layout
+    assert np.array_equal(z[:256 * 8], oracle.swizzle_scales(so)[:256 * 8])
+
+
+def test_sample_rows():
+    import numpy as np
+    r = bench.sample_rows(8192, 100, 5)
+    assert r[0] == 0 and r[-1] == 8191 and np.all(np.diff(r) > 0)
+    assert set(range(64)) <= set(r.tolist()) and set(range(8128, 8192)) <= set(r.tolist())

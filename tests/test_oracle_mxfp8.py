@@ -172,6 +172,29 @@ def test_grouped_equals_per_expert_and_flattened(orc):
         assert np.array_equal(sr[off:off + part.shape[0]], s1)
 
 
+def test_grouped_swizzled_blocks(orc):
+    """Per-expert swizzled scales: for experts of 128-row multiples the blocks
+    meet without padding, so they equal the torch permute formulation of the
+    stacked scales; for ragged experts each block is the permute formulation
+    of that expert's scales, padded on its own to 128 rows, in expert order."""
+    xs = W.experts(seed=11, E=3, M=256, N=160)
+    q, s, z = orc.mxfp8_quantize_grouped(list(xs), swizzled=True)
+    assert np.array_equal(z, refs.swizzle_torch(s))
+    rows = [5, 0, 130, 128, 1]
+    ragged = [W.linear_weight(seed=20 + i, M=max(r, 1), N=96)[:r] for i, r in enumerate(rows)]
+    q, s, z = orc.mxfp8_quantize_grouped(ragged, swizzled=True)
+    pos = 0
+    for i, r in enumerate(rows):
+        off = sum(rows[:i])
+        block = refs.swizzle_torch(s[off:off + r]) if r else np.zeros(0, np.uint8)
+        assert np.array_equal(z[pos:pos + block.size], block), f"expert {i}"
+        pos += block.size
+    assert pos == z.size == sum((r + 127) // 128 * 128 for r in rows) * 4
+    p4, s4, z4 = orc.mxfp4_quantize_grouped(ragged, swizzled=True)
+    assert np.array_equal(s4, np.concatenate([orc.mxfp4_quantize(x)[1] for x in ragged]))
+    assert z4.size == z.size
+
+
 def test_strided_equals_contiguous(orc):
     base = W.activation(seed=10, M=48, N=320)
     q1, s1 = orc.mxfp8_quantize(np.ascontiguousarray(base[:, :256]))
