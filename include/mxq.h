@@ -155,12 +155,15 @@ mxq_status mxfp8_quantize_grouped(const void* x, int dt, int32_t E, const int64_
  * grouped block-scaled GEMM over the experts reads them: expert e's block is
  * mxq_swizzled_scale_bytes(M_e, N/32) bytes (its rows padded to a multiple
  * of 128, padding bytes 0x00) and starts where expert e-1's ends.
- *  scale_swz  device buffer of swz_bytes bytes; it must hold the sum over the
- *             experts of mxq_swizzled_scale_bytes(M_e, N/32), which is at
- *             most mxq_grouped_swizzled_scale_bytes_max(E, M_total, N/32).
- * The kernel reads row_offsets on the device. Offsets that break the rules
- * above are clamped into a non-decreasing sequence from 0 to M_total, and no
- * byte at or past scale_swz + swz_bytes is written, whatever the offsets. */
+ *  scale_swz  device buffer of swz_bytes bytes, 16-byte aligned; it must hold
+ *             the sum over the experts of mxq_swizzled_scale_bytes(M_e, N/32),
+ *             which is at most mxq_grouped_swizzled_scale_bytes_max(E,
+ *             M_total, N/32).
+ * Two launches: the quantize of mxfp8_quantize_grouped, then a gather of each
+ * expert's compact scales into its swizzled block, which reads row_offsets on
+ * the device. Offsets that break the rules above are clamped into a
+ * non-decreasing sequence from 0 to M_total, and no byte at or past
+ * scale_swz + swz_bytes is written, whatever the offsets. */
 mxq_status mxfp8_quantize_grouped_swizzled(const void* x, int dt, int32_t E,
                                            const int64_t* row_offsets, int64_t M_total, int64_t N,
                                            uint8_t* qweight, uint8_t* scale, uint8_t* scale_swz,

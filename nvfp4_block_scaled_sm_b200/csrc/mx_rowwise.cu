@@ -101,36 +101,36 @@ struct QuantArgs {
   uint64_t pad_a;        // swizzle padding entries right of the real scale columns
   uint64_t pad_b;        // swizzle padding entries below the real rows
   int32_t E;             // experts
-  const int64_t* offs;   // device row offsets [E + 1] of a stacked tensor (SWZ == kSwzExperts)
-  uint64_t swz_cap;      // bytes of the swizzled output (SWZ == kSwzExperts)
   const void* x[MAXE];
   uint64_t gbase[MAXE + 1];  // first output group of expert e; gbase[E] = all groups
   uint32_t tbase[MAXE + 1];  // first CTA of expert e; tbase[E] = grid size
 };
 
-// Swizzled-scale modes of mx_quant_kernel: none; one 128x4-tile layout for
-// the whole [M, S] scale; one layout per expert of a stacked tensor, expert
-// e's block starting where expert e-1's 128-row-padded block ends.
+// Swizzled-scale modes of mx_quant_kernel: none, or one 128x4-tile layout for
+// the whole [M, S] scale.
 constexpr int kSwzNone = 0;
 constexpr int kSwzTensor = 1;
-constexpr int kSwzExperts = 2;
 
-// Row offsets of a stacked tensor's experts, read into shared memory by one
-// warp: off[e] = the device offsets clamped into a non-decreasing sequence
-// from off[0] = 0 to off[E] = M (so no write can leave the layout, whatever
-// the offsets hold), and pb[e] = first row of expert e in the per-expert
-// padded layout, pb[e + 1] = pb[e] + ceil((off[e + 1] - off[e]) / 128) * 128.
-__device__ __noinline__ void load_expert_rows(const int64_t* __restrict__ g_off, int E,
+// Row offsets of a stacked tensor's experts in shared memory: off[e] = the
+// device offsets clamped into a non-decreasing sequence from off[0] = 0 to
+// off[E] = M (so no write can leave the layout, whatever the offsets hold),
+// and pb[e] = first row of expert e in the per-expert padded layout,
+// pb[e + 1] = pb[e] + ceil((off[e + 1] - off[e]) / 128) * 128. All threads
+// load the offsets (one global round trip), then one warp scans them in
+// shared memory, 32 entries at a time.
+__device__ __forceinline__ void load_expert_rows(const int64_t* __restrict__ g_off, int E,
                                               int64_t M, int64_t* off, int64_t* pb) {
+  for (int e = threadIdx.x; e <= E; e += kThreads) {
+    int64_t v = e == 0 ? 0 : (e == E ? M : g_off[e]);
+    off[e] = v < 0 ? 0 : (v > M ? M : v);
+  }
+  __syncthreads();
   if (threadIdx.x < 32) {
     const int lane = threadIdx.x;
     int64_t carry_off = 0, carry_pb = 0;
     for (int base = 0; base <= E; base += 32) {
       const int e = base + lane;
-      int64_t v = 0;
-      if (e > 0 && e < E) v = g_off[e];
-      if (e >= E) v = M;
-      v = v < 0 ? 0 : (v > M ? M : v);
+      int64_t v = e <= E ? off[e] : M;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
         const int64_t t = __shfl_up_sync(kFull, v, o);
@@ -157,15 +157,70 @@ __device__ __noinline__ void load_expert_rows(const int64_t* __restrict__ g_off,
   __syncthreads();
 }
 
-// The expert holding row r (0 <= r < off[E]): the largest e < E with
-// off[e] <= r, which skips empty experts.
-__device__ __forceinline__ int expert_of_row(const int64_t* off, int E, int64_t r) {
-  int lo = 0, hi = E;  // invariant: off[lo] <= r < off[hi]
-  while (hi - lo > 1) {
-    const int mid = (lo + hi) >> 1;
-    if (off[mid] <= r) lo = mid; else hi = mid;
+// Per-expert swizzled scales of a stacked tensor, gathered from its compact
+// scales [M, S] (written by the quantize launch just before, in stream
+// order): output block i (128 padded rows x Sp = 4 ceil(S/4) columns, at
+// byte 128 i Sp) belongs to the expert e with pb[e] <= 128 i < pb[e + 1] and
+// holds that expert's rows off[e] + 128 i - pb[e] .. +127; rows past the
+// expert's end and columns past S are 0x00. Persistent CTAs build the row
+// table once, then write whole blocks in output order, one 4-byte word (four
+// scale columns of one row) per thread and step. No byte at or past `cap` is
+// written, whatever the offsets hold.
+__global__ void __launch_bounds__(kThreads)
+mx_swizzle_experts_kernel(const uint8_t* __restrict__ scale, uint8_t* __restrict__ swz,
+                          const int64_t* __restrict__ offs, int32_t E, int64_t M, uint32_t S,
+                          uint32_t Sp4, uint64_t cap, bool words_aligned) {
+  pdl_enter();
+  extern __shared__ int64_t s_rows[];
+  int64_t* off = s_rows;
+  int64_t* pb = s_rows + (E + 1);
+  load_expert_rows(offs, E, M, off, pb);
+  const uint64_t blocks = uint64_t(pb[E]) >> 7;
+  const uint32_t words = 128 * Sp4;  // 4-byte words per output block
+  for (uint64_t i = blockIdx.x; i < blocks; i += gridDim.x) {
+    const int64_t prow = int64_t(i) << 7;
+    int lo = 0, hi = E;  // invariant: pb[lo] <= prow < pb[hi]
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (pb[mid] <= prow) lo = mid; else hi = mid;
+    }
+    const int64_t r0 = off[lo] + (prow - pb[lo]);  // first source row of the block
+    const int64_t rend = off[lo + 1];
+    constexpr int kU = 8;  // words per thread and round, all loaded before any is stored
+    for (uint32_t w0 = threadIdx.x; w0 < words; w0 += kThreads * kU) {
+      uint32_t v[kU];
+#pragma unroll
+      for (int u = 0; u < kU; u++) {
+        const uint32_t w = w0 + u * kThreads;
+        const uint32_t j = w >> 7, wi = w & 127;    // tile of 4 columns, word in the tile
+        const int64_t row = r0 + int64_t((wi & 3) * 32 + (wi >> 2));
+        v[u] = 0;
+        if (w < words && row < rend) {
+          const uint8_t* src = scale + uint64_t(row) * S + 4 * j;
+          if (words_aligned) {
+            v[u] = *reinterpret_cast<const uint32_t*>(src);
+          } else {
+#pragma unroll
+            for (uint32_t k = 0; k < 4; k++)
+              if (4 * j + k < S) v[u] |= uint32_t(src[k]) << (8 * k);
+          }
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kU; u++) {
+        const uint32_t w = w0 + u * kThreads;
+        if (w >= words) continue;
+        const uint64_t o = (i * words + w) * 4;
+        if (o + 4 <= cap) {
+          st_u32(swz + o, v[u]);
+        } else {
+#pragma unroll
+          for (uint32_t k = 0; k < 4; k++)
+            if (o + k < cap) st_u8(swz + o + k, (v[u] >> (8 * k)) & 0xffu);
+        }
+      }
+    }
   }
-  return lo;
 }
 
 // Zero bytes of the swizzled layout outside the real [M, S] scales.
@@ -187,29 +242,6 @@ __device__ __forceinline__ void fill_swizzle_padding(const QuantArgs<MAXE>& a) {
       c = uint32_t(t % Sp);
     }
     st_u8(a.swz + swz_offset(r, c, a.Sp4), 0);
-  }
-}
-
-// Per-expert swizzled layout (kSwzExperts): zero padding of the experts whose
-// last group lies in this CTA's groups [tg0, tg0 + nt): the rows from the
-// expert's end up to its next multiple of 128, all Sp columns.
-template <int MAXE>
-__device__ __forceinline__ void fill_expert_row_padding(const QuantArgs<MAXE>& a, const int64_t* off,
-                                                        const int64_t* pb, uint64_t tg0,
-                                                        uint32_t nt) {
-  const uint64_t S = a.S;
-  const int64_t r0 = int64_t(tg0 / S), r1 = int64_t((tg0 + nt - 1) / S);
-  const uint32_t Sp = a.Sp4 * 4;
-  for (int e = expert_of_row(off, a.E, r0); e < a.E && off[e] <= r1; e++) {
-    const int64_t m = off[e + 1] - off[e];
-    if (m == 0) continue;
-    const uint64_t last = uint64_t(off[e + 1]) * S - 1;  // the expert's last group
-    if (last < tg0 || last >= tg0 + nt) continue;
-    const uint64_t rows = uint64_t(pb[e + 1] - pb[e] - m);
-    for (uint64_t p = threadIdx.x; p < rows * Sp; p += kThreads) {
-      const uint64_t dst = swz_offset(uint64_t(pb[e] + m) + p / Sp, uint32_t(p % Sp), a.Sp4);
-      if (dst < a.swz_cap) st_u8(a.swz + dst, 0);
-    }
   }
 }
 
@@ -277,12 +309,6 @@ mx_quant_kernel(const __grid_constant__ QuantArgs<MAXE> a) {
     if (full || lg < nt) v[u].template load<V8>(p); else v[u].zero();
   }
 
-  // experts' row ranges and padded bases (while the loads are in flight)
-  extern __shared__ int64_t s_rows[];
-  int64_t* off = s_rows;
-  int64_t* pb = s_rows + (a.E + 1);
-  if constexpr (SWZ == kSwzExperts) load_expert_rows(a.offs, a.E, int64_t(a.M), off, pb);
-
 #pragma unroll
   for (int u = 0; u < kSteps; u++) {
     const uint32_t lg = lg0 + u * kGroupsPerStep;
@@ -300,23 +326,10 @@ mx_quant_kernel(const __grid_constant__ QuantArgs<MAXE> a) {
       if (half == 0) {
         st_u8(st + lg, b);
         if constexpr (SWZ == kSwzTensor) st_u8(a.swz + swz_offset(rr[u], cc[u], a.Sp4), b);
-        if constexpr (SWZ == kSwzExperts) {
-          const int ex = expert_of_row(off, a.E, int64_t(rr[u]));
-          const uint64_t pr = uint64_t(pb[ex] + (int64_t(rr[u]) - off[ex]));  // padded row
-          const uint64_t dst = swz_offset(pr, cc[u], a.Sp4);
-          if (dst < a.swz_cap) st_u8(a.swz + dst, b);
-          if (cc[u] == a.S - 1) {  // the row's padding columns
-            for (uint32_t cp = a.S; cp < a.Sp4 * 4; cp++) {
-              const uint64_t dp = swz_offset(pr, cp, a.Sp4);
-              if (dp < a.swz_cap) st_u8(a.swz + dp, 0);
-            }
-          }
-        }
       }
     }
   }
   if constexpr (SWZ == kSwzTensor) fill_swizzle_padding(a);
-  if constexpr (SWZ == kSwzExperts) fill_expert_row_padding(a, off, pb, tg0, nt);
 }
 
 // ------------------------------------------------------- decode and store
@@ -548,10 +561,7 @@ inline bool aligned32(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 
 template <typename InT, bool V8, bool STRIDED, int SWZ, int MAXE, int FMT>
 mxq_status launch_quant(const QuantArgs<MAXE>& a, uint32_t grid, cudaStream_t stream) {
-  // the per-expert swizzle keeps the experts' row offsets in shared memory
-  const size_t smem = SWZ == kSwzExperts ? 2 * sizeof(int64_t) * size_t(a.E + 1) : 0;
-  return launched(launch_pdl_ex(mx_quant_kernel<InT, V8, STRIDED, SWZ, MAXE, FMT>, grid, kThreads,
-                                smem, stream, a));
+  return launched(launch_pdl(mx_quant_kernel<InT, V8, STRIDED, SWZ, MAXE, FMT>, grid, stream, a));
 }
 
 template <typename InT, bool V8, int FMT>
@@ -693,8 +703,9 @@ mxq_status grouped_entry(int32_t E, const void* const* xs, const int64_t* rows, 
 
 // Grouped quantize of a stacked tensor: the compact outputs are those of the
 // flattened [M, N] call (groups never cross rows, so expert boundaries change
-// no byte of them); the device row offsets place each expert's swizzled scale
-// block.
+// no byte of them), in one launch; with scale_swz a second launch gathers
+// each expert's scales into its own swizzled block, placed by the device row
+// offsets.
 template <int FMT>
 mxq_status grouped_stacked_entry(const void* x, int dt, int32_t E, const int64_t* row_offsets,
                                  int64_t M, int64_t N, uint8_t* q, uint8_t* scale,
@@ -704,6 +715,7 @@ mxq_status grouped_stacked_entry(const void* x, int dt, int32_t E, const int64_t
   if (!row_offsets) return MXQ_ERR_NULL;
   if (reinterpret_cast<uintptr_t>(row_offsets) & 7u) return MXQ_ERR_ALIGN;
   if (scale_swz && swz_bytes < 0) return MXQ_ERR_SHAPE;
+  if (scale_swz && !aligned16(scale_swz)) return MXQ_ERR_ALIGN;
   if (M == 0 || N == 0) return MXQ_OK;
   if (!x || !q || !scale) return MXQ_ERR_NULL;
   const uint64_t S = uint64_t(N) / 32;
@@ -715,15 +727,11 @@ mxq_status grouped_stacked_entry(const void* x, int dt, int32_t E, const int64_t
   QuantArgs<1> a{};
   a.q = q;
   a.scale = scale;
-  a.swz = scale_swz;
   a.ld = N;
   a.rows = FastDiv::make(uint32_t(S));
   a.S = uint32_t(S);
-  a.Sp4 = uint32_t((S + 3) / 4);
   a.M = uint64_t(M);
-  a.E = E;
-  a.offs = row_offsets;
-  a.swz_cap = scale_swz ? uint64_t(swz_bytes) : 0;
+  a.E = 1;
   a.x[0] = x;
   a.gbase[0] = 0;
   a.gbase[1] = groups;
@@ -732,18 +740,25 @@ mxq_status grouped_stacked_entry(const void* x, int dt, int32_t E, const int64_t
   const bool v8 = aligned32(x) && row_bytes % 32 == 0;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const uint32_t grid = uint32_t(tiles);
-  if (scale_swz == nullptr) {
-    if (dt == MXQ_BF16)
-      return v8 ? launch_quant<uint16_t, true, false, kSwzNone, 1, FMT>(a, grid, s)
-                : launch_quant<uint16_t, false, false, kSwzNone, 1, FMT>(a, grid, s);
-    return v8 ? launch_quant<float, true, false, kSwzNone, 1, FMT>(a, grid, s)
-              : launch_quant<float, false, false, kSwzNone, 1, FMT>(a, grid, s);
-  }
+  mxq_status st;
   if (dt == MXQ_BF16)
-    return v8 ? launch_quant<uint16_t, true, false, kSwzExperts, 1, FMT>(a, grid, s)
-              : launch_quant<uint16_t, false, false, kSwzExperts, 1, FMT>(a, grid, s);
-  return v8 ? launch_quant<float, true, false, kSwzExperts, 1, FMT>(a, grid, s)
-            : launch_quant<float, false, false, kSwzExperts, 1, FMT>(a, grid, s);
+    st = v8 ? launch_quant<uint16_t, true, false, kSwzNone, 1, FMT>(a, grid, s)
+            : launch_quant<uint16_t, false, false, kSwzNone, 1, FMT>(a, grid, s);
+  else
+    st = v8 ? launch_quant<float, true, false, kSwzNone, 1, FMT>(a, grid, s)
+            : launch_quant<float, false, false, kSwzNone, 1, FMT>(a, grid, s);
+  if (st != MXQ_OK || scale_swz == nullptr) return st;
+  // the gather: as many persistent CTAs as there can be output blocks, up to
+  // four per multiprocessor
+  const uint32_t Sp4 = uint32_t((S + 3) / 4);
+  const uint64_t max_blocks = (uint64_t(M) + 127 * uint64_t(E)) / 128;
+  const uint64_t cap_ctas = uint64_t(sm_count()) * 4;
+  const uint32_t sgrid = uint32_t(std::max<uint64_t>(1, std::min(max_blocks, cap_ctas)));
+  const size_t smem = 2 * sizeof(int64_t) * size_t(E + 1);
+  const bool words_aligned = S % 4 == 0 && (reinterpret_cast<uintptr_t>(scale) & 3u) == 0;
+  return launched(launch_pdl_ex(mx_swizzle_experts_kernel, sgrid, kThreads, smem, s,
+                                static_cast<const uint8_t*>(scale), scale_swz, row_offsets, E,
+                                int64_t(M), uint32_t(S), Sp4, uint64_t(swz_bytes), words_aligned));
 }
 
 template <typename InT, typename OutT, int FMT>

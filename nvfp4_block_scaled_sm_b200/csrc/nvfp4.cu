@@ -32,8 +32,9 @@
 // approximate reciprocal would not be normal), is put on a shared list and
 // recomputed by the definition, with IEEE divisions, after the tile's main
 // loop; the out-of-line exact path then costs the main loop one predicated
-// shared atomic. Blocks with eff == 0 (the zero-block guard) get sign-kept
-// zero codes inline. Products below the normal range are far below the first
+// shared atomic. Blocks with eff == 0 (the zero-block guard: all-zero blocks,
+// or a zero global scale) fail the same range test and get their sign-kept
+// zero codes on the exact path too. Products below the normal range are far below the first
 // midpoint and overflowing products far above the last, so neither can change
 // a code.
 //
@@ -287,14 +288,12 @@ __device__ __forceinline__ void quant_tile(const QuantArgs& a, uint64_t tb0, uin
       sb = cvt_e4m3x2(s, 0.0f) & 0xffu;  // NaN -> 0x7F
       eff = __fmul_rn(decode_e4m3(sb), g);
     }
-    uint2 codes;
-    if (eff == 0.0f) {
-      codes = zero_codes(v[u]);
-    } else {
-      bool sure_codes;
-      codes = e2m1_codes(v[u], eff, sure_codes);
-      sure = sure && sure_codes;
-    }
+    // eff == 0 (the zero-block guard) fails the reciprocal's range test
+    // inside e2m1_codes, so such blocks are left to the exact path, which
+    // writes their sign-kept zeros; the main loop carries no code for them
+    bool sure_codes;
+    const uint2 codes = e2m1_codes(v[u], eff, sure_codes);
+    sure = sure && sure_codes;
     st_v2(pk + lb * 8, codes);
     st_u8(sc + lb, sb);
     if (__builtin_expect(!sure, 0)) fix_list[atomicAdd(fix_count, 1u)] = uint16_t(lb);

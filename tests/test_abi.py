@@ -177,6 +177,7 @@ def test_grouped_stacked_validation():
         assert G(A, 0, 4, O, 64, 64, A, A, None, 4096, None) == NULL
         assert G(A, 0, 4, O, 64, 64, A, A, A, -1, None) == SHAPE
         assert G(A, 0, 4, None, 64, 64, A, A, A, 4096, None) == NULL
+        assert G(A, 0, 4, O, 64, 64, A, A, A + 8, 4096, None) == ALIGN
         assert G(None, 0, 4, O, 0, 64, None, None, A, 0, None) == OK
 
 
