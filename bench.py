@@ -442,6 +442,10 @@ def config_lines(mxq, device, flush):
     threads = host_threads()
     lines = []
 
+    def check(st):
+        if st:
+            raise mxq.MxqError("bench", st, mxq.lib.mxq_status_string(st).decode())
+
     def bf(a):
         return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(device)
 
@@ -473,55 +477,91 @@ def config_lines(mxq, device, flush):
          {"quantize_us": tq * 1e3, "dequantize_us": td * 1e3,
           "cpu_baseline_single_thread": cpu_baseline_single_thread_planted()})
 
-    # 2: linear weight 4096x4096, quantize; 8 rotating input/output sets (> 2x L2)
+    # 2: linear weight 4096x4096, quantize; 8 rotating input/output sets (> 2x L2),
+    # back-to-back launches
+    L, sp = mxq.lib, ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+    stream = torch.cuda.current_stream(device)
+    V = lambda t: ctypes.c_void_p(t.data_ptr())
     x = W.linear_weight()
     xs = [bf(x) for _ in range(8)]
     outs = [mxq.mxfp8_quantize(t) for t in xs]
-    L, sp = mxq.lib, ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
-    P = [[ctypes.c_void_p(t.data_ptr()) for t in (xs[i], outs[i][0], outs[i][1])] for i in range(8)]
+    P = [[V(t) for t in (xs[i], outs[i][0], outs[i][1])] for i in range(8)]
     k = [0]
 
     def rot():
         p = P[k[0] % 8]
         k[0] += 1
-        L.mxfp8_quantize(p[0], 0, 4096, 4096, 4096, p[1], p[2], None, sp)
+        check(L.mxfp8_quantize(p[0], 0, 4096, 4096, 4096, p[1], p[2], None, sp))
 
-    t = time_kernel(rot, 48)[0]
+    for _ in range(8):
+        rot()
+    t = events_loop(stream, rot, 96) / 96
     qo, so = zip(*oracle_rows_parallel(oracle.mxfp8_quantize, x, threads, 256))
     ok = (np.array_equal(outs[0][0].cpu().numpy(), np.concatenate(qo))
           and np.array_equal(outs[0][1].cpu().numpy(), np.concatenate(so)))
-    line(2, "MXFP8 quantize, linear weight bf16 4096x4096 (8 rotating input/output sets)",
-         mxfp8_quant_bytes(4096, 4096, swizzled=False), t, ok, "all rows")
+    line(2, "MXFP8 quantize, linear weight bf16 4096x4096 (8 rotating input/output sets, "
+            "back-to-back launches)", mxfp8_quant_bytes(4096, 4096, swizzled=False), t, ok,
+         "all rows")
     del xs, outs, P
     torch.cuda.empty_cache()
 
-    # 4: 64 experts 2048x7168 stacked, one grouped launch (+ per-expert swizzled scales)
+    # 4: 64 experts 2048x7168 stacked, one grouped launch (compact outputs), and
+    # with the per-expert swizzled scales (a second, gather launch)
+    E, R, Nn = 64, 2048, 7168
     x = W.experts()
     xd = bf(x)
     del x
-    t = time_kernel(lambda: mxq.mxfp8_quantize_grouped(xd, swizzled=True), 10)[0]
-    q, s, z = mxq.mxfp8_quantize_grouped(xd, swizzled=True)
+    off = (torch.arange(E + 1, dtype=torch.int64) * R).to(device)
+    q = torch.empty((E * R, Nn), dtype=torch.uint8, device=device)
+    s = torch.empty((E * R, Nn // 32), dtype=torch.uint8, device=device)
+    z = torch.empty(E * R * (Nn // 32), dtype=torch.uint8, device=device)
+    grouped = lambda: check(L.mxfp8_quantize_grouped(V(xd), 0, E, V(off), E * R, Nn, V(q), V(s), sp))
+    grouped_swz = lambda: check(L.mxfp8_quantize_grouped_swizzled(
+        V(xd), 0, E, V(off), E * R, Nn, V(q), V(s), V(z), z.numel(), sp))
+    for _ in range(3):
+        grouped_swz()
+    t_swz = events_loop(stream, grouped_swz, 10) / 10
+    for _ in range(3):
+        grouped()
+    t = events_loop(stream, grouped, 10) / 10
+    grouped_swz()
     picks = [0, 9, 21, 30, 42, 51, 58, 63]
     xh = {e: xd[e].view(torch.int16).cpu().numpy().view(np.uint16) for e in picks}
     res = pmap(lambda e: oracle.mxfp8_quantize(xh[e]), picks, threads)
-    blk = 2048 * 224
+    blk = R * (Nn // 32)
     ok = True
+    qv, sv = q.view(E, R, Nn), s.view(E, R, Nn // 32)
     for e, (qo, so) in zip(picks, res):
-        ok &= np.array_equal(q[e].cpu().numpy(), qo) and np.array_equal(s[e].cpu().numpy(), so)
+        ok &= np.array_equal(qv[e].cpu().numpy(), qo) and np.array_equal(sv[e].cpu().numpy(), so)
         ok &= np.array_equal(z[e * blk:(e + 1) * blk].cpu().numpy(), oracle.swizzle_scales(so))
-    line(4, "grouped MXFP8 quantize (+ per-expert swizzled scales), 64 stacked experts bf16 "
-            "2048x7168, one launch", mxfp8_quant_bytes(64 * 2048, 7168), t, ok,
-         f"experts {picks}, all outputs")
-    del xd, q, s, z
+    line(4, "grouped MXFP8 quantize, 64 stacked experts bf16 2048x7168, one launch "
+            "(back-to-back launches)", mxfp8_quant_bytes(E * R, Nn, swizzled=False), t, ok,
+         f"experts {picks}: codes, scales and per-expert swizzled scales",
+         {"with_per_expert_swizzled_scales_us": t_swz * 1e3,
+          "with_per_expert_swizzled_scales_gbs": mxfp8_quant_bytes(E * R, Nn) / t_swz / 1e6})
+    del xd, q, s, z, qv, sv
     torch.cuda.empty_cache()
 
-    # 5: NVFP4 two passes, 8192x8192
+    # 5: NVFP4 two passes, 8192x8192 (and the block pass alone, given the scale)
     x = W.nvfp4_tensor()
     xd = bf(x)
     ws = torch.empty(mxq.nvfp4_workspace_bytes(), dtype=torch.uint8, device=device)
-    t = time_kernel(lambda: mxq.nvfp4_quantize(xd, workspace=ws), 30)[0]
-    p, b, g = mxq.nvfp4_quantize(xd, workspace=ws)
-    tg = time_kernel(lambda: mxq.nvfp4_quantize(xd, global_scale=g), 30)[0]
+    p = torch.empty((8192, 4096), dtype=torch.uint8, device=device)
+    b = torch.empty((8192, 512), dtype=torch.uint8, device=device)
+    g = torch.empty((), dtype=torch.float32, device=device)
+    gg = torch.empty((), dtype=torch.float32, device=device)
+    two = lambda: check(L.nvfp4_quantize(V(xd), 0, 8192, 8192, 8192, V(p), V(b), V(g), None, 0,
+                                         V(ws), ws.numel(), sp))
+    given = lambda: check(L.nvfp4_quantize(V(xd), 0, 8192, 8192, 8192, V(p), V(b), V(gg), None, 1,
+                                           None, 0, sp))
+    for _ in range(3):
+        two()
+    t = events_loop(stream, two, 30) / 30
+    gg.copy_(g)
+    for _ in range(3):
+        given()
+    tg = events_loop(stream, given, 30) / 30
+    two()
     go = oracle.nvfp4_global_amax(x) / np.float32(2688.0)
     rows = sample_rows(8192, 512, 5)
     res = oracle_rows_parallel(lambda xr: oracle.nvfp4_quantize(xr, float(go))[:2],
@@ -529,12 +569,13 @@ def config_lines(mxq, device, flush):
     po, bo = np.concatenate([r[0] for r in res]), np.concatenate([r[1] for r in res])
     ok = (np.float32(g.item()) == np.float32(go)
           and np.array_equal(p.cpu().numpy()[rows], po) and np.array_equal(b.cpu().numpy()[rows], bo))
-    line(5, "NVFP4 two-level quantize (amax pass + block pass), bf16 8192x8192",
-         nvfp4_quant_bytes(8192, 8192), t, ok, f"global scale and {rows.size} sampled rows",
-         {"single_read_bytes": nvfp4_quant_bytes(8192, 8192, two_pass=False),
-          "gbs_single_read_count": nvfp4_quant_bytes(8192, 8192, two_pass=False) / t / 1e6,
-          "block_pass_given_scale_us": tg * 1e3,
-          "block_pass_gbs": nvfp4_quant_bytes(8192, 8192, two_pass=False) / tg / 1e6})
+    single = nvfp4_quant_bytes(8192, 8192, two_pass=False)
+    line(5, "NVFP4 two-level quantize (amax pass + block pass), bf16 8192x8192 (back-to-back "
+            "launches)", nvfp4_quant_bytes(8192, 8192), t, ok,
+         f"global scale and {rows.size} sampled rows",
+         {"single_read_bytes": single, "gbs_single_read_count": single / t / 1e6,
+          "block_pass_given_scale_us": tg * 1e3, "block_pass_gbs": single / tg / 1e6,
+          "block_pass_frac_of_" + kind: single / tg / 1e6 / peak})
     del xd, p, b
     torch.cuda.empty_cache()
     return lines
@@ -649,7 +690,7 @@ def run(args):
         "mx_dequant_kernel": {"avg_us": d_ms * 1e3, "bytes": db, "gbs": db / (d_ms / 1e3) / 1e9},
     }
     for k in kernels.values():
-        k["frac_of_measured"] = k["gbs"] / peak
+        k["frac_of_" + peak_kind] = k["gbs"] / peak
         k["frac_of_spec_8tbs"] = k["gbs"] / SPEC_HBM_GBS
     dom = max(kernels, key=lambda k: kernels[k]["avg_us"])
     h2d = x.numel() * 2
@@ -707,31 +748,47 @@ def _flush_l2(buf):
 
 
 def time_kernel(fn, iters, flush_buf=None, poll=False):
-    """Median device time (ms) of fn() over iters launches, L2 flushed between
-    launches when flush_buf is given (the flush is outside the timed span).
-    poll: wait for the last event by polling, so that a clock-sampling thread
-    runs while the GPU works."""
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in range(iters)]
+    """Device time (ms) per call of fn(). Without flush_buf: five loops of
+    `iters` back-to-back calls, events only around each loop; returns the
+    median, lowest and highest per-call average of the loops. With flush_buf
+    (small workloads): L2 flushed before each call by a write larger than L2,
+    events around each call alone; returns median, p10 and p90. poll: wait
+    for the last event by polling, so that a clock-sampling thread runs while
+    the GPU works."""
     for _ in range(3):
         fn()
-    for a, b in evs:
-        if flush_buf is not None:
+    torch.cuda.synchronize()
+    if flush_buf is None:
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(5)]
+        for a, b in evs:
+            a.record()
+            for _ in range(iters):
+                fn()
+            b.record()
+    else:
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(iters)]
+        for a, b in evs:
             _flush_l2(flush_buf)
-        a.record()
-        fn()
-        b.record()
+            a.record()
+            fn()
+            b.record()
     if poll:
         while not evs[-1][1].query():
             time.sleep(0.0002)
     torch.cuda.synchronize()
+    if flush_buf is None:
+        t = sorted(a.elapsed_time(b) / iters for a, b in evs)
+        return t[2], t[0], t[-1]
     t = sorted(a.elapsed_time(b) for a, b in evs)
     return t[len(t) // 2], t[len(t) // 10], t[(len(t) * 9) // 10]
 
 
 def run_suite(device, only=None):
-    """One JSON line per workload kernel: median device time over repeated
-    launches (L2 flushed between launches for the 50 MB workload, the others
+    """One JSON line per workload kernel: device time per launch of repeated
+    back-to-back launches (L2 flushed before each launch for the 50 MB workload
+    and smaller, which are timed one launch at a time; the others
     exceed L2), algorithmic bytes, GB/s and fraction of the HBM peak."""
     import ctypes
 
@@ -780,28 +837,33 @@ def run_suite(device, only=None):
 
         emit("mxfp8_quantize linear_weight 4096x4096 (8 rotating input/output sets)",
              mxfp8_quant_bytes(4096, 4096, swizzled=False), time_kernel(rotating, 48))
-        # eight such weights: one call each, against one grouped launch over
-        # the stacked eight (rotating between two stacks, 2 x 268 MB > L2)
+        # eight such weights: one C-ABI call each, against one grouped launch
+        # over the stacked eight (rotating between two stacks, 2 x 268 MB > L2)
         stacks = [torch.stack(xs), torch.stack(xs).clone()]
-        del xs, qs, ss
+        del xs, qs, ss, P
+        q8 = torch.empty((8 * 4096, 4096), dtype=torch.uint8, device=device)
+        s8 = torch.empty((8 * 4096, 128), dtype=torch.uint8, device=device)
+        off8 = (torch.arange(9, dtype=torch.int64) * 4096).to(device)
+        V = lambda t: ctypes.c_void_p(t.data_ptr())
         k[0] = 0
 
         def eight_calls():
             st = stacks[k[0] % 2]
             k[0] += 1
             for i in range(8):
-                mxq.mxfp8_quantize(st[i])
+                L.mxfp8_quantize(V(st[i]), 0, 4096, 4096, 4096, V(q8[4096 * i:]), V(s8[4096 * i:]),
+                                 None, sp)
 
         def one_grouped():
             st = stacks[k[0] % 2]
             k[0] += 1
-            mxq.mxfp8_quantize_grouped(st)
+            L.mxfp8_quantize_grouped(V(st), 0, 8, V(off8), 8 * 4096, 4096, V(q8), V(s8), sp)
 
         eight = 8 * mxfp8_quant_bytes(4096, 4096, swizzled=False)
         emit("8 x mxfp8_quantize linear_weight 4096x4096, one call each", eight,
-             time_kernel(eight_calls, 20))
+             time_kernel(eight_calls, 10))
         emit("mxfp8_quantize_grouped of the 8 stacked linear weights 8x4096x4096, one launch",
-             eight, time_kernel(one_grouped, 20))
+             eight, time_kernel(one_grouped, 10))
 
     def activation():
         x = bf(W.activation())
