@@ -154,3 +154,33 @@ def test_full_size_sampled():
     exact, absum = oracle_product(xa[rows], xb[cols])
     got = d.float().cpu().numpy()[np.ix_(rows, cols)]
     check_tol(got, exact, absum, 7168, True, "full size, sampled")
+
+
+@pytest.mark.parametrize("fmt_rows", [[128, 200, 64, 0, 1], [256, 300]])
+def test_per_expert_swizzled_scales_feed_the_gemm(fmt_rows):
+    """The grouped quantize's per-expert swizzled scales, read by the tensor
+    cores: expert e's block of the swizzled output is handed to the GEMM as
+    that expert's scale layout, and each expert's product must equal the
+    oracle's exactly (power-of-two grid inputs). This pins the per-expert
+    layout with a hardware consumer, not only with the oracle's composition."""
+    rows = fmt_rows
+    K = 256
+    parts = [W.gemm_pow2_operand(3000 + i, max(r, 1), K)[:r] for i, r in enumerate(rows)]
+    x = np.concatenate(parts, 0)
+    offs = np.concatenate([[0], np.cumsum(rows)]).tolist()
+    q, s, z = mxq.mxfp8_quantize_grouped(dev(x), row_offsets=offs, swizzled=True)
+    xb = W.gemm_pow2_operand(4000, 144, K)
+    qb, _, zb = mxq.mxfp8_quantize(dev(xb), swizzled=True)
+    qbo, sbo = oracle.mxfp8_quantize(xb)
+    pos = 0
+    for e, r in enumerate(rows):
+        nb = mxq.swizzled_scale_bytes(r, K // 32)
+        if r:
+            d = mxq.mxfp8_gemm(q[offs[e]:offs[e + 1]].contiguous(), z[pos:pos + nb], qb, zb,
+                               torch.float32)
+            qa_o, sa_o = oracle.mxfp8_quantize(parts[e])
+            exact = oracle.mxfp8_gemm(qa_o, sa_o, qbo, sbo)
+            got = host(d).view(np.float32).astype(np.float64)
+            assert np.array_equal(got, exact), f"expert {e}: {int((got != exact).sum())} entries differ"
+        pos += nb
+    assert pos == z.numel()
