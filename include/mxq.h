@@ -169,6 +169,18 @@ mxq_status mxfp8_quantize_grouped_swizzled(const void* x, int dt, int32_t E,
                                            uint8_t* qweight, uint8_t* scale, uint8_t* scale_swz,
                                            int64_t swz_bytes, mxq_stream_t stream);
 
+/* Writes a compact [M, S] scale array in the 128x4-tile layout described at
+ * mxfp8_quantize (rows padded to a multiple of 128 and columns to a multiple
+ * of 4 with 0x00): the E8M0 scales of mxfp8_quantize / mxfp4_quantize
+ * (S = N/32), or the E4M3 block scales of nvfp4_quantize (S = N/16), which
+ * block-scaled tensor-core MMAs read in the same tiling. (The pages have no
+ * such step; it lays out what the quantizers wrote.)
+ *  scale      device [M, S] bytes, row-major, compact.
+ *  scale_swz  device, 16-byte aligned, mxq_swizzled_scale_bytes(M, S) bytes.
+ * M == 0 or S == 0 writes nothing. One launch. */
+mxq_status mxq_swizzle_scales(const uint8_t* scale, int64_t M, int64_t S, uint8_t* scale_swz,
+                              mxq_stream_t stream);
+
 /* Upper bound of the per-expert swizzled scale bytes of E experts with
  * M_total rows in all (each expert adds at most 127 padding rows):
  * floor((M_total + 127 E) / 128) * 128 * ceil(S/4) * 4; -1 for negative

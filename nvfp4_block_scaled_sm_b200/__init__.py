@@ -27,7 +27,7 @@ __all__ = [
     "mxfp8_gemm",
     "nvfp4_amax", "nvfp4_quantize", "nvfp4_dequantize",
     "nvfp4_amax_sliced", "nvfp4_quantize_sliced", "nvfp4_quantize_experts",
-    "swizzled_scale_bytes", "nvfp4_workspace_bytes", "set_output_allocator",
+    "swizzled_scale_bytes", "nvfp4_workspace_bytes", "set_output_allocator", "swizzle_scales",
     "as_float8_e4m3", "as_float8_e8m0", "as_float4_e2m1x2",
 ]
 
@@ -65,6 +65,7 @@ def _load() -> ctypes.CDLL:
     L.mxfp8_quantize_grouped.argtypes = [vp, i32, i32, vp, i64, i64, vp, vp, vp]
     L.mxfp8_quantize_grouped_swizzled.argtypes = [vp, i32, i32, vp, i64, i64, vp, vp, vp, i64, vp]
     L.mxfp8_quantize_grouped_ptrs.argtypes = [i32, vp, vp, i64, i32, vp, vp, vp]
+    L.mxq_swizzle_scales.argtypes = [vp, i64, i64, vp, vp]
     L.mxq_grouped_swizzled_scale_bytes_max.argtypes = [i32, i64, i64]
     L.mxq_grouped_swizzled_scale_bytes_max.restype = i64
     L.mxfp8_quantize_columnwise.argtypes = [vp, i32, i64, i64, i64, vp, vp, vp, vp, vp]
@@ -87,7 +88,7 @@ def _load() -> ctypes.CDLL:
               "mxfp8_quantize_grouped_swizzled", "mxfp8_quantize_grouped_ptrs",
               "mxfp8_quantize_columnwise", "mxfp4_quantize", "mxfp4_dequantize",
               "mxfp4_quantize_grouped", "mxfp4_quantize_grouped_swizzled",
-              "mxfp4_quantize_grouped_ptrs", "mx_fake_quantize", "mxfp8_gemm", "nvfp4_amax",
+              "mxfp4_quantize_grouped_ptrs", "mx_fake_quantize", "mxq_swizzle_scales", "mxfp8_gemm", "nvfp4_amax",
               "nvfp4_quantize_sliced", "nvfp4_amax_sliced",
               "nvfp4_quantize", "nvfp4_dequantize"):
         getattr(L, f).restype = i32
@@ -185,6 +186,22 @@ def swizzled_scale_bytes(M: int, S: int) -> int:
 
 def nvfp4_workspace_bytes(M: int = 0, N: int = 0) -> int:
     return int(lib.mxq_nvfp4_workspace_bytes(M, N))
+
+
+def swizzle_scales(scale: torch.Tensor) -> torch.Tensor:
+    """A compact [..., S] uint8 scale tensor (E8M0 scales of the MX
+    quantizers, or NVFP4's E4M3 block scales) in the 128x4-tile layout read by
+    block-scaled tensor-core MMA, as a flat uint8 tensor of
+    ``swizzled_scale_bytes(M, S)`` bytes (M = the product of the leading
+    dimensions)."""
+    _require_cuda(scale)
+    if scale.dtype != torch.uint8 or not scale.is_contiguous() or scale.dim() == 0:
+        raise TypeError("scale must be a contiguous uint8 tensor")
+    S = scale.shape[-1]
+    M = scale.numel() // S if S else 0
+    out = _empty((max(swizzled_scale_bytes(M, S), 0),), torch.uint8, scale.device)
+    _check("mxq_swizzle_scales", lib.mxq_swizzle_scales(_ptr(scale), M, S, _ptr(out), _stream(scale)))
+    return out
 
 
 # ------------------------------------------------------------------ MXFP8

@@ -814,6 +814,26 @@ mxq_status mxfp8_quantize_grouped_swizzled(const void* x, int dt, int32_t E,
                                                 scale_swz, swz_bytes, stream);
 }
 
+mxq_status mxq_swizzle_scales(const uint8_t* scale, int64_t M, int64_t S, uint8_t* scale_swz,
+                              mxq_stream_t stream) {
+  using namespace mxq;
+  if (M < 0 || S < 0 || S > 0xffffffffll) return MXQ_ERR_SHAPE;
+  if (M == 0 || S == 0) return MXQ_OK;
+  if (!scale || !scale_swz) return MXQ_ERR_NULL;
+  if (!aligned16(scale_swz)) return MXQ_ERR_ALIGN;
+  // the one-expert case of the per-expert gather: its row table is {0, M},
+  // so the offsets pointer is never read
+  const uint32_t Sp4 = uint32_t((S + 3) / 4);
+  const uint64_t blocks = (uint64_t(M) + 127) / 128;
+  const uint32_t grid = uint32_t(std::max<uint64_t>(1, std::min(blocks, uint64_t(sm_count()) * 4)));
+  const uint64_t bytes = blocks * 128 * uint64_t(Sp4) * 4;
+  const bool words_aligned = S % 4 == 0 && (reinterpret_cast<uintptr_t>(scale) & 3u) == 0;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  return launched(launch_pdl_ex(mx_swizzle_experts_kernel, grid, kThreads, 2 * sizeof(int64_t) * 2, s,
+                                scale, scale_swz, static_cast<const int64_t*>(nullptr), int32_t(1),
+                                M, uint32_t(S), Sp4, bytes, words_aligned));
+}
+
 mxq_status mxfp8_quantize_grouped_ptrs(int32_t E, const void* const* xs, const int64_t* rows,
                                        int64_t N, int dt, uint8_t* qweight, uint8_t* scale,
                                        mxq_stream_t stream) {

@@ -181,6 +181,17 @@ def test_grouped_stacked_validation():
         assert G(None, 0, 4, O, 0, 64, None, None, A, 0, None) == OK
 
 
+def test_swizzle_scales_validation():
+    Z = mxq.lib.mxq_swizzle_scales
+    assert Z(A, -1, 4, A, None) == SHAPE
+    assert Z(A, 4, -1, A, None) == SHAPE
+    assert Z(None, 4, 4, A, None) == NULL
+    assert Z(A, 4, 4, None, None) == NULL
+    assert Z(A, 4, 4, A + 4, None) == ALIGN
+    assert Z(None, 0, 4, None, None) == OK
+    assert Z(None, 4, 0, None, None) == OK
+
+
 def test_grouped_swizzled_bound():
     B = mxq.lib.mxq_grouped_swizzled_scale_bytes_max
     assert B(1, 100, 7) == 128 * 8

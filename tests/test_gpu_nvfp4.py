@@ -95,3 +95,57 @@ def test_zero_and_special_values():
 def test_errors():
     with pytest.raises(mxq.MxqError):
         mxq.nvfp4_quantize(torch.zeros(4, 24, dtype=torch.bfloat16, device="cuda"))
+
+
+@pytest.mark.parametrize("M,S", [(1, 1), (130, 7), (300, 33), (256, 224), (4096, 512)])
+def test_swizzle_scales_standalone(M, S):
+    """mxq_swizzle_scales on arbitrary bytes equals the oracle's layout."""
+    s = np.random.default_rng(M * 7 + S).integers(0, 256, (M, S), dtype=np.uint8)
+    z = mxq.swizzle_scales(dev(s))
+    assert_same(host(z), oracle.swizzle_scales(s), f"swizzled [{M}, {S}]")
+
+
+def test_nvfp4_block_scales_swizzled():
+    x = W.nvfp4_tensor(seed=44, M=333, N=1024)
+    _, b, _ = mxq.nvfp4_quantize(dev(x))
+    _, bo, _ = oracle.nvfp4_quantize(x)
+    assert_same(host(mxq.swizzle_scales(b)), oracle.swizzle_scales(bo), "NVFP4 swizzled block scales")
+
+
+def _nvfp4_values(packed, bs):
+    """float64 [M, N] of decode_e2m1(code) * decode_e4m3(block scale), from
+    the oracle's outputs (the global scale left out)."""
+    e2 = np.array([oracle.e2m1_decode(c) for c in range(16)], np.float64)
+    e4 = oracle.e4m3_decode_table()
+    codes = np.stack([packed & 0xF, packed >> 4], axis=-1).reshape(packed.shape[0], -1)
+    return e2[codes] * np.repeat(e4[bs], 16, axis=1)
+
+
+def test_nvfp4_swizzled_block_scales_feed_a_library_gemm():
+    """NVIDIA's library block-scaled GEMM (through torch scaled_mm, NVFP4
+    operands with E4M3 block scales per 16 in the 128x4-tile layout) reads
+    this library's packed codes and swizzled block scales and reproduces the
+    oracle's product within fp32 accumulation error: a consumer pin of the
+    NVFP4 scale layout. Each E2M1 x E4M3 product pair is exact in fp32."""
+    F = torch.nn.functional
+    M, N, K = 256, 384, 512
+    xa, xb = W.nvfp4_tensor(seed=45, M=M, N=K), W.nvfp4_tensor(seed=46, M=N, N=K)
+    pa, ba, _ = mxq.nvfp4_quantize(dev(xa))
+    pb, bb, _ = mxq.nvfp4_quantize(dev(xb))
+    try:
+        d = F.scaled_mm(pa.view(torch.float4_e2m1fn_x2), pb.view(torch.float4_e2m1fn_x2).t(),
+                        mxq.swizzle_scales(ba).view(torch.float8_e4m3fn), F.ScalingType.BlockWise1x16,
+                        mxq.swizzle_scales(bb).view(torch.float8_e4m3fn), F.ScalingType.BlockWise1x16,
+                        swizzle_a=F.SwizzleType.SWIZZLE_32_4_4, swizzle_b=F.SwizzleType.SWIZZLE_32_4_4,
+                        output_dtype=torch.float32)
+    except (RuntimeError, NotImplementedError, TypeError, AttributeError) as e:
+        pytest.skip(f"this torch build runs no NVFP4 scaled_mm: {str(e)[:120]}")
+    torch.cuda.synchronize()
+    pao, bao, _ = oracle.nvfp4_quantize(xa)
+    pbo, bbo, _ = oracle.nvfp4_quantize(xb)
+    A, B = _nvfp4_values(pao, bao), _nvfp4_values(pbo, bbo)
+    exact = A @ B.T
+    tol = K * 2.0 ** -22 * (np.abs(A) @ np.abs(B).T) + 1e-30
+    got = d.cpu().numpy().astype(np.float64)
+    bad = np.abs(got - exact) > tol
+    assert not bad.any(), f"{int(bad.sum())} entries outside the bound, first {np.argwhere(bad)[:4].tolist()}"
