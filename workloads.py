@@ -22,6 +22,11 @@ tests can draw smaller instances of the same recipe):
                     U(0.01, 0.05), values N(0, std), seed 3.
 5. ``nvfp4_tensor`` bf16 [8192, 8192] N(0,1) with 0.05 % of entries replaced
                     by +-U(20, 100), seed 4.
+
+``normal_on_device`` is the one generator that draws on the GPU (torch's
+seeded CUDA generator): it makes tensors of billions of elements that the host
+generator would take minutes to produce. The oracle reads rows of such a
+tensor copied back from the device.
 """
 from __future__ import annotations
 
@@ -282,3 +287,18 @@ def nvfp4_block_scale_sweep_fp32(seed: int = 5) -> np.ndarray:
               * np.resize(amax, rows * 16)[:, None])
     blocks[:, 0] = np.resize(amax, rows * 16)
     return blocks.reshape(rows, 256)
+
+
+# ------------------------------------------------------------ large inputs
+
+def normal_on_device(M: int, N: int, seed: int, device="cuda") -> torch.Tensor:
+    """bf16 [M, N] N(0,1) drawn on the device by torch's seeded CUDA
+    generator, in row chunks (each chunk drawn in fp32 and cast to bf16)."""
+    gen = torch.Generator(device=device)
+    gen.manual_seed(seed)
+    x = torch.empty((M, N), dtype=torch.bfloat16, device=device)
+    step = max(1, (1 << 26) // max(N, 1))
+    for r in range(0, M, step):
+        x[r:r + step] = torch.randn((min(step, M - r), N), generator=gen, device=device,
+                                    dtype=torch.float32).to(torch.bfloat16)
+    return x
