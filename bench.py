@@ -117,6 +117,7 @@ def tensor_peak(sustained=False):
 KERNEL_SOURCES = {"mx_quant_kernel": ("common.cuh", "mx_rowwise.cu"),
                   "mx_dequant_kernel": ("common.cuh", "mx_rowwise.cu"),
                   "mx_fake_quant_kernel": ("common.cuh", "mx_rowwise.cu"),
+                  "mx_swizzle_experts_kernel": ("common.cuh", "mx_rowwise.cu"),
                   "mxfp8_colwise_kernel": ("common.cuh", "colwise.cu"),
                   "nvfp4_amax_kernel": ("common.cuh", "nvfp4.cu"),
                   "nvfp4_quant_kernel": ("common.cuh", "nvfp4.cu"),
@@ -640,10 +641,16 @@ def run(args):
     y_out = y.view(torch.int16).cpu().numpy().view(np.uint16)
 
     # per-kernel device time for the roofline: R launches of one kernel back
-    # to back between two events (every launch rewrites the same outputs)
-    R = max(20, min(200, K))
+    # to back between two events (every launch rewrites the same outputs),
+    # after three untimed ones, so that the write-back of the other kernel's
+    # dirty lines left in L2 does not land in the loop
+    R = max(50, min(200, K))
     with ClockSampler(device) as clk_k:
+        for _ in range(3):
+            quant()
         q_ms = events_loop(stream, quant, R) / R
+        for _ in range(3):
+            dequant()
         d_ms = events_loop(stream, dequant, R) / R
     q_ms = reduce_max(q_ms, world, device)
     d_ms = reduce_max(d_ms, world, device)
@@ -710,7 +717,8 @@ def run(args):
                      "spec_80pct_target_met": kernels[dom]["gbs"] >= 0.8 * SPEC_HBM_GBS,
                      "algorithmic_bytes_per_launch": kernels[dom]["bytes"],
                      "traffic": recorded_traffic(dom),
-                     "timing": f"{R} back-to-back launches of each kernel between two events"},
+                     "timing": f"{R} back-to-back launches of each kernel between two events, "
+                               "after 3 untimed ones"},
         "breakdown": kernels,
         "e2e": {"value": step_bytes * world / (e2e_ms / 1e3) / 1e9, "unit": "GB/s",
                 "ms_per_step": e2e_ms, "steps": e2e_steps,
