@@ -15,6 +15,7 @@ N/32), the scale being the dequantization multiplier ("_scale_inv").
 from __future__ import annotations
 
 import ctypes
+import functools
 import os
 from typing import Sequence
 
@@ -28,6 +29,7 @@ __all__ = [
     "nvfp4_amax", "nvfp4_quantize", "nvfp4_dequantize",
     "nvfp4_amax_sliced", "nvfp4_quantize_sliced", "nvfp4_quantize_experts",
     "swizzled_scale_bytes", "nvfp4_workspace_bytes", "set_output_allocator", "swizzle_scales",
+    "set_nvtx",
     "as_float8_e4m3", "as_float8_e8m0", "as_float4_e2m1x2",
 ]
 
@@ -619,3 +621,41 @@ def as_float8_e8m0(s: torch.Tensor) -> torch.Tensor:
 
 def as_float4_e2m1x2(p: torch.Tensor) -> torch.Tensor:
     return p.view(torch.float4_e2m1fn_x2)
+
+
+# ------------------------------------------------------------------ NVTX
+
+_nvtx = False
+
+
+def set_nvtx(enabled: bool) -> bool:
+    """Wrap every quantization call of this module in an NVTX range named
+    ``mxq.<function>`` (for a profiler's timeline) when ``enabled``; off by
+    default. Returns the previous setting."""
+    global _nvtx
+    prev, _nvtx = _nvtx, bool(enabled)
+    return prev
+
+
+def _traced(fn):
+    name = "mxq." + fn.__name__
+
+    @functools.wraps(fn)
+    def wrapper(*args, **kwargs):
+        if not _nvtx:
+            return fn(*args, **kwargs)
+        torch.cuda.nvtx.range_push(name)
+        try:
+            return fn(*args, **kwargs)
+        finally:
+            torch.cuda.nvtx.range_pop()
+    return wrapper
+
+
+for _name in ("mxfp8_quantize", "mxfp8_dequantize", "mxfp8_quantize_grouped",
+              "mxfp8_quantize_columnwise", "mxfp4_quantize", "mxfp4_dequantize",
+              "mxfp4_quantize_grouped", "mx_fake_quantize", "mxfp8_gemm", "nvfp4_amax",
+              "nvfp4_quantize", "nvfp4_dequantize", "nvfp4_amax_sliced", "nvfp4_quantize_sliced",
+              "nvfp4_quantize_experts", "swizzle_scales"):
+    globals()[_name] = _traced(globals()[_name])
+del _name

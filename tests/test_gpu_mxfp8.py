@@ -130,3 +130,35 @@ def test_requantize_is_identity():
     q, s = mxq.mxfp8_quantize(x)
     q2, s2 = mxq.mxfp8_quantize(mxq.mxfp8_dequantize(q, s, torch.float32))
     assert torch.equal(q, q2) and torch.equal(s, s2)
+
+
+def test_nvtx_ranges_and_a_failing_allocation():
+    """With NVTX ranges on, results are unchanged; an output allocation that
+    fails (a host-side fault injected through the allocator hook) surfaces as
+    the allocator's exception, and the next call works."""
+    x = W.activation(seed=5, M=64, N=256)
+    q0, s0 = mxq.mxfp8_quantize(dev(x))
+    prev = mxq.set_nvtx(True)
+    try:
+        q1, s1 = mxq.mxfp8_quantize(dev(x))
+    finally:
+        mxq.set_nvtx(prev)
+    assert torch.equal(q0, q1) and torch.equal(s0, s1)
+
+    calls = []
+
+    def failing(shape, dtype, device):
+        calls.append(shape)
+        if len(calls) == 2:
+            raise MemoryError("injected allocation failure")
+        return torch.empty(shape, dtype=dtype, device=device)
+
+    old = mxq.set_output_allocator(failing)
+    try:
+        with pytest.raises(MemoryError, match="injected"):
+            mxq.mxfp8_quantize(dev(x))
+    finally:
+        mxq.set_output_allocator(old)
+    q2, s2 = mxq.mxfp8_quantize(dev(x))
+    torch.cuda.synchronize()
+    assert torch.equal(q0, q2) and torch.equal(s0, s2)

@@ -55,3 +55,10 @@ def test_binding_uses_the_hook():
         assert mxq.set_output_allocator(prev) is alloc
     assert seen == [((2, 3), torch.uint8), ((4,), torch.float32)]
     assert t.shape == (2, 3) and float(z.abs().sum()) == 0.0
+
+
+def test_nvtx_wrapping_keeps_the_api():
+    mxq = pytest.importorskip("nvfp4_block_scaled_sm_b200")
+    assert mxq.mxfp8_quantize.__name__ == "mxfp8_quantize"
+    assert "MXFP8 rowwise quantize" in mxq.mxfp8_quantize.__doc__
+    assert mxq.set_nvtx(False) is False and mxq.set_nvtx(False) is False

@@ -1,0 +1,98 @@
+"""Properties of the oracle on small inputs that hypothesis draws and shrinks:
+arbitrary bf16 bit patterns (NaN, infinities, subnormals included) in
+[m, 32 k] shapes. Each property follows from the definitions alone:
+
+- the E8M0 byte is the clamp formula of the group's non-NaN amax;
+- quantize is idempotent through the fp32 dequantization (finite inputs);
+- a normal, unsaturated E4M3 result dequantizes within 2^-4 of its input;
+- grouped quantize equals quantizing each expert on its own;
+- NVFP4: the block holding the tensor's amax gets scale 448 (0x7E) and its
+  largest element code 6.
+"""
+import numpy as np
+from hypothesis import HealthCheck, given, settings
+from hypothesis import strategies as st
+from hypothesis.extra.numpy import arrays
+
+import oracle
+
+SETTINGS = settings(max_examples=150, deadline=None,
+                    suppress_health_check=[HealthCheck.too_slow, HealthCheck.data_too_large])
+
+
+def bf16_arrays(max_rows=6, max_groups=3, finite=False):
+    def build(shape):
+        elems = st.integers(0, 0xFFFF)
+        if finite:
+            elems = elems.filter(lambda b: (b & 0x7F80) != 0x7F80)
+        return arrays(np.uint16, shape, elements=elems)
+    shapes = st.tuples(st.integers(1, max_rows), st.integers(1, max_groups)).map(
+        lambda t: (t[0], 32 * t[1]))
+    return shapes.flatmap(build)
+
+
+def f64(bits):
+    return (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+@SETTINGS
+@given(bf16_arrays())
+def test_scale_byte_is_the_clamp_of_the_group_amax(x):
+    _, s = oracle.mxfp8_quantize(x)
+    v = np.abs(f64(x)).reshape(x.shape[0], -1, 32)
+    amax = np.where(np.isnan(v), -1.0, v).max(axis=2)
+    amax = np.maximum(amax, 0.0)
+    want = np.empty(amax.shape, np.int64)
+    for i, a in np.ndenumerate(amax):
+        if a == 0:
+            want[i] = 127
+        elif np.isinf(a):
+            want[i] = 254
+        else:
+            want[i] = min(254, max(0, np.frexp(a)[1] - 1 + 127 - 8))
+    assert np.array_equal(s.astype(np.int64), want)
+
+
+@SETTINGS
+@given(bf16_arrays(finite=True))
+def test_quantize_is_idempotent_through_fp32_dequant(x):
+    q, s = oracle.mxfp8_quantize(x)
+    y = oracle.mxfp8_dequantize(q, s, out="f32")
+    q2, s2 = oracle.mxfp8_quantize(y)
+    assert np.array_equal(q2, q) and np.array_equal(s2, s)
+
+
+@SETTINGS
+@given(bf16_arrays(finite=True))
+def test_dequantized_error_of_normal_results(x):
+    q, s = oracle.mxfp8_quantize(x)
+    y = oracle.mxfp8_dequantize(q, s, out="f32").astype(np.float64)
+    xv = f64(x)
+    mag = q & 0x7F
+    normal = (mag >= 0x08) & (mag < 0x7E)          # normal E4M3 codes below the saturation value
+    err = np.abs(y - xv)
+    assert np.all(err[normal] <= 2.0 ** -4 * np.abs(xv[normal]))
+
+
+@SETTINGS
+@given(bf16_arrays(max_rows=9), st.lists(st.integers(0, 9), min_size=1, max_size=4))
+def test_grouped_equals_per_expert(x, cuts):
+    cuts = sorted(min(c, x.shape[0]) for c in cuts)
+    bounds = [0] + cuts + [x.shape[0]]
+    parts = [x[a:b] for a, b in zip(bounds[:-1], bounds[1:])]
+    qg, sg = oracle.mxfp8_quantize_grouped(parts)
+    qf, sf = oracle.mxfp8_quantize(x)
+    assert np.array_equal(qg, qf) and np.array_equal(sg, sf)
+
+
+@SETTINGS
+@given(bf16_arrays(finite=True))
+def test_nvfp4_block_of_the_amax(x):
+    v = np.abs(f64(x))
+    if v.max() == 0:
+        return
+    packed, bs, g = oracle.nvfp4_quantize(x)
+    r, c = np.unravel_index(np.argmax(v), v.shape)
+    assert bs[r, c // 16] == 0x7E
+    code = (packed[r, c // 2] >> (4 * (c % 2))) & 0x7
+    assert code == 0x7                                  # |x| / eff rounds to 6
