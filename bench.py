@@ -24,7 +24,7 @@ the device-timed region ("scaling": "weak").
 ``--impl reference`` times the CPU oracle (test infrastructure) on the host's
 cores (row chunks on threads, each running the single-threaded oracle) on a
 bounded sample of the same workload. ``--suite`` prints one extra JSON line
-per workload kernel (documentation, not the default line).
+per workload kernel (documentation beside the headline line).
 """
 from __future__ import annotations
 
