@@ -157,6 +157,11 @@ __device__ __forceinline__ void load_expert_rows(const int64_t* __restrict__ g_o
   __syncthreads();
 }
 
+// Swizzled scales are limited to S <= 2^27 columns (2^25 four-column tiles):
+// the gather counts the 4-byte words of a 128-row output block in 32 bits, and
+// the padding writer the padded width 4 ceil(S/4).
+constexpr uint32_t kMaxSwizzleTileCols = 1u << 25;
+
 // Per-expert swizzled scales of a stacked tensor, gathered from its compact
 // scales [M, S] (written by the quantize launch just before, in stream
 // order): output block i (128 padded rows x Sp = 4 ceil(S/4) columns, at
@@ -586,6 +591,7 @@ mxq_status quantize_impl(const void* x, int dt, int64_t M, int64_t N, int64_t ld
   const uint64_t groups = uint64_t(M) * S;
   const uint64_t tiles = (groups + kGroupsPerTile - 1) / kGroupsPerTile;
   if (S > 0xffffffffull || tiles > 0x7fffffffull) return MXQ_ERR_SHAPE;
+  if (scale_swz != nullptr && (S + 3) / 4 > kMaxSwizzleTileCols) return MXQ_ERR_SHAPE;
   const uint64_t row_bytes = uint64_t(ld_x) * elem_size(dt);
   if (!aligned16(x) || row_bytes % 16 != 0 || !aligned16(q)) return MXQ_ERR_ALIGN;
 
@@ -722,6 +728,7 @@ mxq_status grouped_stacked_entry(const void* x, int dt, int32_t E, const int64_t
   const uint64_t groups = uint64_t(M) * S;
   const uint64_t tiles = (groups + kGroupsPerTile - 1) / kGroupsPerTile;
   if (S > 0xffffffffull || tiles > 0x7fffffffull) return MXQ_ERR_SHAPE;
+  if (scale_swz != nullptr && (S + 3) / 4 > kMaxSwizzleTileCols) return MXQ_ERR_SHAPE;
   const uint64_t row_bytes = uint64_t(N) * elem_size(dt);
   if (!aligned16(x) || row_bytes % 16 != 0 || !aligned16(q)) return MXQ_ERR_ALIGN;
   QuantArgs<1> a{};
@@ -817,7 +824,7 @@ mxq_status mxfp8_quantize_grouped_swizzled(const void* x, int dt, int32_t E,
 mxq_status mxq_swizzle_scales(const uint8_t* scale, int64_t M, int64_t S, uint8_t* scale_swz,
                               mxq_stream_t stream) {
   using namespace mxq;
-  if (M < 0 || S < 0 || S > 0xffffffffll) return MXQ_ERR_SHAPE;
+  if (M < 0 || S < 0 || (S + 3) / 4 > kMaxSwizzleTileCols) return MXQ_ERR_SHAPE;
   if (M == 0 || S == 0) return MXQ_OK;
   if (!scale || !scale_swz) return MXQ_ERR_NULL;
   if (!aligned16(scale_swz)) return MXQ_ERR_ALIGN;
