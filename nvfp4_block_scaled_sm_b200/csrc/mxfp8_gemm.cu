@@ -161,6 +161,16 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
+// 16 consecutive fp32 accumulator columns of this thread's lane.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
 __device__ __forceinline__ void sts128_u32(uint32_t addr, uint4 v) {
   asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z),
                "r"(v.w)
@@ -606,13 +616,15 @@ mxfp8_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_c
       const uint32_t row0 = m_blk * 256 + 128 * rank + quarter * 32;
       const uint32_t ncols = min(256u, a.N - n_blk * 256);
       if constexpr (sizeof(OutT) == 2) {
+        // 16 columns per tensor-memory load: the whole row (128 bf16 pairs)
+        // then fits in registers without spilling
         uint32_t w[128];
 #pragma unroll
-        for (uint32_t c0 = 0; c0 < 256u; c0 += 32) {
-          uint32_t r[32];
-          tmem_ld32(taddr + c0, r);
+        for (uint32_t c0 = 0; c0 < 256u; c0 += 16) {
+          uint32_t r[16];
+          tmem_ld16(taddr + c0, r);
 #pragma unroll
-          for (int q = 0; q < 16; q++)
+          for (int q = 0; q < 8; q++)
             w[c0 / 2 + q] = cvt_bf16x2(__uint_as_float(r[2 * q]), __uint_as_float(r[2 * q + 1]));
         }
         tc_fence_before();
