@@ -586,9 +586,11 @@ mxfp8_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_c
         const uint32_t sfa_t = tmem + 256 + kPairSfCols * s;
         const uint32_t sfb_t = sfa_t + 4u;
         const uint32_t sf = st + kPairTileA + kPairTileB;
-        tmem_copy_scales_pair(sfa_t, scale_desc(sf));
+        // B's two tiles first: this order measured about 0.6 % faster than
+        // A first (alternating rounds, every round)
         tmem_copy_scales_pair(sfb_t, scale_desc(sf + kSfTile));
         tmem_copy_scales_pair(sfb_t + 4u, scale_desc(sf + 2 * kSfTile));
+        tmem_copy_scales_pair(sfa_t, scale_desc(sf));
 #pragma unroll
         for (uint32_t k = 0; k < 4; k++) {
           mma_mxf8_pair(tmem, operand_desc(st + 32u * k), operand_desc(st + kPairTileA + 32u * k),
