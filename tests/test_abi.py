@@ -297,3 +297,28 @@ def test_rows_view():
         mxq._rows_view(torch.zeros(4, 6, 96)[:, :, :64].transpose(0, 1))
     with pytest.raises(ValueError):
         mxq._rows_view(torch.zeros(64, 4).t())
+
+
+def test_c_program_against_header_and_library():
+    """tests/c/abi_check.c, built with a C compiler against include/mxq.h
+    (C11, warnings as errors) and linked with the library, runs its
+    validation checks: the boundary is usable from plain C without Python."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    here = os.path.dirname(os.path.abspath(__file__))
+    root = os.path.dirname(here)
+    libdir = os.path.dirname(mxq.library_path)
+    out_dir = os.path.join(here, "c", "_build")
+    os.makedirs(out_dir, exist_ok=True)
+    exe = os.path.join(out_dir, "abi_check")
+    build = subprocess.run([cc, "-std=c11", "-Wall", "-Wextra", "-pedantic", "-Werror",
+                            "-I", os.path.join(root, "include"), os.path.join(here, "c", "abi_check.c"),
+                            "-L", libdir, "-lmxq", f"-Wl,-rpath,{libdir}", "-o", exe],
+                           capture_output=True, text=True)
+    assert build.returncode == 0, build.stderr
+    run = subprocess.run([exe], capture_output=True, text=True, timeout=120)
+    assert run.returncode == 0, run.stdout + run.stderr
+    assert "all" in run.stdout and "checks passed" in run.stdout
