@@ -2,6 +2,8 @@
 roofline figure it prints) equal the sizes of the buffers each kernel reads
 and writes: the input, the codes, the compact scales and, where written, the
 swizzled scales as the library sizes them. No GPU needed."""
+import os
+
 import pytest
 
 import bench
@@ -63,3 +65,40 @@ def test_sample_rows():
     r = bench.sample_rows(8192, 100, 5)
     assert r[0] == 0 and r[-1] == 8191 and np.all(np.diff(r) > 0)
     assert set(range(64)) <= set(r.tolist()) and set(range(8128, 8192)) <= set(r.tolist())
+
+
+def test_reference_arm_prints_the_contract_line():
+    """`bench.py --impl reference` (the oracle on the host cores, no GPU)
+    prints one JSON line with the keys the driver reads."""
+    import json
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    run = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--impl", "reference",
+                          "--steps", "1", "--warmup", "3"], capture_output=True, text=True,
+                         timeout=600, cwd=root)
+    assert run.returncode == 0, run.stderr[-2000:]
+    lines = [l for l in run.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1, run.stdout[-2000:]
+    d = json.loads(lines[0])
+    for k in ("impl", "metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+              "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config",
+              "cpu_baseline", "e2e"):
+        assert k in d, k
+    assert d["impl"] == "reference" and d["unit"] == "GB/s" and d["value"] > 0
+    assert d["steps"] == 1 and d["warmup"] == 3 and d["higher_is_better"] is True
+    assert "workload" in d["config"]
+    cb = d["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == d["value"] and cb["sample"]
+    e = d["e2e"]
+    assert e["value"] == d["value"] and e["h2d_bytes_per_step"] == 0 and e["d2h_bytes_per_step"] == 0
+
+
+def test_bench_rejects_short_warmup():
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    run = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--warmup", "2"],
+                         capture_output=True, text=True, timeout=300, cwd=root)
+    assert run.returncode != 0
+    assert "warmup" in (run.stdout + run.stderr)
