@@ -4,13 +4,16 @@ arbitrary bf16 bit patterns (NaN, infinities, subnormals included) in
 
 - the E8M0 byte is the clamp formula of the group's non-NaN amax;
 - quantize is idempotent through the fp32 dequantization (finite inputs);
-- a normal, unsaturated E4M3 result dequantizes within 2^-4 of its input;
+- an element whose scaled value |x| 2^(127 - byte) lies in E4M3's normal
+  range [2^-6, 448] dequantizes within 2^-4 of itself (below 2^-6 it rounds
+  on the subnormal grid m 2^-9, whose half spacing is a larger fraction of
+  the value: just below 2^-6 it can round up to 2^-6, 6.7 % away);
 - grouped quantize equals quantizing each expert on its own;
 - NVFP4: the block holding the tensor's amax gets scale 448 (0x7E) and its
   largest element code 6.
 """
 import numpy as np
-from hypothesis import HealthCheck, given, settings
+from hypothesis import HealthCheck, example, given, settings
 from hypothesis import strategies as st
 from hypothesis.extra.numpy import arrays
 
@@ -64,12 +67,17 @@ def test_quantize_is_idempotent_through_fp32_dequant(x):
 
 @SETTINGS
 @given(bf16_arrays(finite=True))
-def test_dequantized_error_of_normal_results(x):
+# an element scaled to 0.0146484375, just below 2^-6, beside an amax of 2^111:
+# it rounds up on the subnormal grid to the smallest normal, 6.7 % away
+@example(np.array([[0] * 30 + [0x6FF0, 0x7700]], np.uint16))
+def test_dequantized_error_of_normal_range_inputs(x):
     q, s = oracle.mxfp8_quantize(x)
     y = oracle.mxfp8_dequantize(q, s, out="f32").astype(np.float64)
     xv = f64(x)
-    mag = q & 0x7F
-    normal = (mag >= 0x08) & (mag < 0x7E)          # normal E4M3 codes below the saturation value
+    # the element scaled by its group's power of two (exact in float64)
+    scale = np.repeat(np.ldexp(1.0, s.astype(np.int64) - 127), 32, axis=1)
+    v = np.abs(xv) / scale
+    normal = (v >= 2.0 ** -6) & (v <= 448.0)      # E4M3's normal range, no saturation
     err = np.abs(y - xv)
     assert np.all(err[normal] <= 2.0 ** -4 * np.abs(xv[normal]))
 
