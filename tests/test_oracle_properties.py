@@ -12,6 +12,8 @@ arbitrary bf16 bit patterns (NaN, infinities, subnormals included) in
 - NVFP4: the block holding the tensor's amax gets scale 448 (0x7E) and its
   largest element code 6.
 """
+import os
+
 import numpy as np
 from hypothesis import HealthCheck, example, given, settings
 from hypothesis import strategies as st
@@ -20,8 +22,10 @@ from hypothesis.extra.numpy import arrays
 import oracle
 
 # derandomized: the same 150 examples per property on every run, so the suite
-# is repeatable; `pytest --hypothesis-seed=N` explores other draws
-SETTINGS = settings(max_examples=150, deadline=None, derandomize=True,
+# is repeatable; MXQ_PROPERTY_EXPLORE=1 draws fresh examples (with
+# `--hypothesis-seed=N` to replay a run)
+SETTINGS = settings(max_examples=150, deadline=None,
+                    derandomize=os.environ.get("MXQ_PROPERTY_EXPLORE") != "1",
                     suppress_health_check=[HealthCheck.too_slow, HealthCheck.data_too_large])
 
 
