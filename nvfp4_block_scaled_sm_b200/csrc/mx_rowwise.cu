@@ -421,7 +421,9 @@ __device__ __forceinline__ void store16(OutT* dst, const float (&f)[16], bool an
 // A lane owns 16 codes (one 16-byte load of E4M3 codes, one 8-byte load of
 // packed E2M1) and writes 16 outputs (32 bytes of bf16, 64 of fp32, with
 // 256-bit stores when 32-byte aligned); two lanes a group; 16 groups per warp
-// step.
+// step. Tiles are taken from the last to the first: a dequantize that follows
+// a quantize of the same codes then starts on the rows that quantize wrote
+// last, much of which is still in L2 (measured 1-2 % off the pair's time).
 constexpr int kDqSteps = 2;
 constexpr int kDqGroupsPerWarp = 16 * kDqSteps;
 constexpr int kDqGroupsPerTile = kDqGroupsPerWarp * (kThreads / 32);
@@ -432,7 +434,7 @@ mx_dequant_kernel(const uint8_t* __restrict__ q, const uint8_t* __restrict__ sca
                   OutT* __restrict__ y, uint64_t ng) {
   pdl_enter();
   constexpr uint32_t CB = kCodeBytes<FMT>;
-  const uint64_t g0 = uint64_t(blockIdx.x) * kDqGroupsPerTile;
+  const uint64_t g0 = uint64_t(gridDim.x - 1 - blockIdx.x) * kDqGroupsPerTile;
   const uint64_t left = ng - g0;
   const uint32_t nt = left < kDqGroupsPerTile ? uint32_t(left) : uint32_t(kDqGroupsPerTile);
   const bool full = nt == kDqGroupsPerTile;
