@@ -121,18 +121,25 @@ __device__ __forceinline__ uint32_t instr_desc(uint32_t k) {
   return (k << 4) | (uint32_t(BN >> 3) << 17) | (1u << 23) | (uint32_t(kBM >> 4) << 24) | (k << 29);
 }
 
-__device__ __forceinline__ void mma_mxf8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+// The MMA and the scale copy take their shared-memory descriptors as 32-bit
+// words (low words of A and B, one high word): the issuing lane then only adds
+// offsets to precomputed words.
+__device__ __forceinline__ void mma_mxf8(uint32_t d_tmem, uint32_t a_lo, uint32_t b_lo, uint32_t hi,
                                          uint32_t idesc, uint32_t sfa_tmem, uint32_t sfb_tmem,
                                          uint32_t accumulate) {
   asm volatile(
-      "{ .reg .pred p; setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p; }"
-      ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      "{ .reg .pred p; .reg .b64 da, db; setp.ne.b32 p, %5, 0;\n\t"
+      "mov.b64 da, {%1, %3}; mov.b64 db, {%2, %3};\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], da, db, %4, [%6], [%7], p; }"
+      ::"r"(d_tmem), "r"(a_lo), "r"(b_lo), "r"(hi), "r"(idesc), "r"(accumulate), "r"(sfa_tmem),
+        "r"(sfb_tmem)
       : "memory");
 }
 
-__device__ __forceinline__ void tmem_copy_scales(uint32_t taddr, uint64_t sdesc) {
-  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+__device__ __forceinline__ void tmem_copy_scales(uint32_t taddr, uint32_t lo, uint32_t hi) {
+  asm volatile("{ .reg .b64 d; mov.b64 d, {%1, %2};\n\t"
+               "tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], d; }" ::"r"(taddr), "r"(lo), "r"(hi)
+               : "memory");
 }
 
 __device__ __forceinline__ void mma_commit(uint32_t bar) {
@@ -271,7 +278,13 @@ mxfp8_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_consta
     }
   } else if (warp == 1 && lane == 0) {
     // ------------------------------------------------------- MMA issuer
-    uint32_t it = 0;
+    // descriptors as 32-bit words plus offsets, as in the pair kernel
+    const uint64_t op0 = operand_desc(base);
+    const uint64_t sc0 = scale_desc(base + C::kTileA + C::kTileB);
+    const uint32_t op_lo = uint32_t(op0), op_hi = uint32_t(op0 >> 32);
+    const uint32_t sc_lo = uint32_t(sc0), sc_hi = uint32_t(sc0 >> 32);
+    constexpr uint32_t kStageW = kStageBytes >> 4, kTileAW = C::kTileA >> 4, kSfW = kSfTile >> 4;
+    uint32_t s = 0, phase = 0;
     for (uint32_t i = 0; i < n_my; i++) {
       // the epilogue must have read the previous tile's accumulator
       if (i > 0 && !mbar_wait(acc_empty, (i - 1) & 1u, kWaitNs)) {
@@ -280,29 +293,30 @@ mxfp8_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_consta
       }
       tc_fence_after();
       bool ok = true;
-      for (uint32_t kb = 0; kb < a.nk; kb++, it++) {
-        const int s = it % kStages;
-        const uint32_t phase = (it / kStages) & 1u;
+      for (uint32_t kb = 0; kb < a.nk; kb++) {
         if (!mbar_wait(full_bar(s), phase, kWaitNs)) {
           record_error(a.err, kErrFullWait);
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint32_t st = base + s * kStageBytes;
+        const uint32_t so = s * kStageW;
         const uint32_t sfa_t = tmem + BN + C::kSfColsPerStage * s;
         const uint32_t sfb_t = sfa_t + 4u;
-        const uint32_t sf = st + C::kTileA + C::kTileB;
-        tmem_copy_scales(sfa_t, scale_desc(sf));
+        tmem_copy_scales(sfa_t, sc_lo + so, sc_hi);
 #pragma unroll
         for (uint32_t j = 0; j < C::kSfbTiles; j++)
-          tmem_copy_scales(sfb_t + 4u * j, scale_desc(sf + kSfTile * (1 + j)));
+          tmem_copy_scales(sfb_t + 4u * j, sc_lo + so + kSfW * (1 + j), sc_hi);
 #pragma unroll
         for (uint32_t k = 0; k < 4; k++) {
-          mma_mxf8(tmem, operand_desc(st + 32u * k), operand_desc(st + C::kTileA + 32u * k),
-                   instr_desc<BN>(k), sfa_t | (k << 30), sfb_t | (k << 30), (kb | k) != 0u);
+          mma_mxf8(tmem, op_lo + so + 2 * k, op_lo + so + kTileAW + 2 * k, op_hi, instr_desc<BN>(k),
+                   sfa_t | (k << 30), sfb_t | (k << 30), (kb | k) != 0u);
         }
         mma_commit(empty_bar(s));
+        if (++s == kStages) {
+          s = 0;
+          phase ^= 1u;
+        }
       }
       if (!ok) break;
       mma_commit(acc_full);
@@ -461,18 +475,23 @@ __device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap
       : "memory");
 }
 
-__device__ __forceinline__ void mma_mxf8_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
-                                              uint32_t idesc, uint32_t sfa_tmem, uint32_t sfb_tmem,
-                                              uint32_t accumulate) {
+// The pair forms of mma_mxf8 and tmem_copy_scales.
+__device__ __forceinline__ void mma_mxf8_pair(uint32_t d_tmem, uint32_t a_lo, uint32_t b_lo,
+                                              uint32_t hi, uint32_t idesc, uint32_t sfa_tmem,
+                                              uint32_t sfb_tmem, uint32_t accumulate) {
   asm volatile(
-      "{ .reg .pred p; setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::2.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p; }"
-      ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      "{ .reg .pred p; .reg .b64 da, db; setp.ne.b32 p, %5, 0;\n\t"
+      "mov.b64 da, {%1, %3}; mov.b64 db, {%2, %3};\n\t"
+      "tcgen05.mma.cta_group::2.kind::mxf8f6f4.block_scale [%0], da, db, %4, [%6], [%7], p; }"
+      ::"r"(d_tmem), "r"(a_lo), "r"(b_lo), "r"(hi), "r"(idesc), "r"(accumulate), "r"(sfa_tmem),
+        "r"(sfb_tmem)
       : "memory");
 }
 
-__device__ __forceinline__ void tmem_copy_scales_pair(uint32_t taddr, uint64_t sdesc) {
-  asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+__device__ __forceinline__ void tmem_copy_scales_pair(uint32_t taddr, uint32_t lo, uint32_t hi) {
+  asm volatile("{ .reg .b64 d; mov.b64 d, {%1, %2};\n\t"
+               "tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], d; }" ::"r"(taddr), "r"(lo), "r"(hi)
+               : "memory");
 }
 
 // Arrives on the barrier at this shared offset in both CTAs of the pair once
@@ -565,7 +584,18 @@ mxfp8_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_c
     }
   } else if (warp == 1 && lane == 0 && rank == 0) {
     // ------------------------------------------------------- MMA issuer
-    uint32_t it = 0;
+    // Descriptors as 32-bit words: the address field holds addr / 16 of a
+    // shared address below 256 KiB, so moving an operand by d bytes (a
+    // multiple of 16) adds d / 16 to the low word and leaves the high word.
+    // The lane's scalar work sits between its tcgen05 instructions, so it is
+    // kept to a few adds (building each descriptor from its address instead,
+    // with the ring position as it % 6, measured about 10 % slower overall).
+    const uint64_t op0 = operand_desc(base);
+    const uint64_t sc0 = scale_desc(base + kPairTileA + kPairTileB);
+    const uint32_t op_lo = uint32_t(op0), op_hi = uint32_t(op0 >> 32);
+    const uint32_t sc_lo = uint32_t(sc0), sc_hi = uint32_t(sc0 >> 32);
+    constexpr uint32_t kStageW = kPairStageBytes >> 4, kTileAW = kPairTileA >> 4, kSfW = kSfTile >> 4;
+    uint32_t s = 0, phase = 0;
     for (uint32_t i = 0; i < n_my; i++) {
       if (i > 0 && !mbar_wait(acc_empty, (i - 1) & 1u, kWaitNs)) {
         record_error(a.err, kErrAccumWait);
@@ -573,30 +603,31 @@ mxfp8_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_c
       }
       tc_fence_after();
       bool ok = true;
-      for (uint32_t kb = 0; kb < a.nk; kb++, it++) {
-        const int s = it % kPairStages;
-        const uint32_t phase = (it / kPairStages) & 1u;
+      for (uint32_t kb = 0; kb < a.nk; kb++) {
         if (!mbar_wait(full_bar(s), phase, kWaitNs)) {
           record_error(a.err, kErrFullWait);
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint32_t st = base + s * kPairStageBytes;
+        const uint32_t so = s * kStageW;
         const uint32_t sfa_t = tmem + 256 + kPairSfCols * s;
         const uint32_t sfb_t = sfa_t + 4u;
-        const uint32_t sf = st + kPairTileA + kPairTileB;
         // B's two tiles first: this order measured about 0.6 % faster than
         // A first (alternating rounds, every round)
-        tmem_copy_scales_pair(sfb_t, scale_desc(sf + kSfTile));
-        tmem_copy_scales_pair(sfb_t + 4u, scale_desc(sf + 2 * kSfTile));
-        tmem_copy_scales_pair(sfa_t, scale_desc(sf));
+        tmem_copy_scales_pair(sfb_t, sc_lo + so + kSfW, sc_hi);
+        tmem_copy_scales_pair(sfb_t + 4u, sc_lo + so + 2 * kSfW, sc_hi);
+        tmem_copy_scales_pair(sfa_t, sc_lo + so, sc_hi);
 #pragma unroll
         for (uint32_t k = 0; k < 4; k++) {
-          mma_mxf8_pair(tmem, operand_desc(st + 32u * k), operand_desc(st + kPairTileA + 32u * k),
-                        instr_desc_pair(k), sfa_t | (k << 30), sfb_t | (k << 30), (kb | k) != 0u);
+          mma_mxf8_pair(tmem, op_lo + so + 2 * k, op_lo + so + kTileAW + 2 * k, op_hi,
+                          instr_desc_pair(k), sfa_t | (k << 30), sfb_t | (k << 30), (kb | k) != 0u);
         }
         mma_commit_pair(empty_bar(s));
+        if (++s == kPairStages) {
+          s = 0;
+          phase ^= 1u;
+        }
       }
       if (!ok) break;
       mma_commit_pair(acc_full);

@@ -32,16 +32,21 @@ __device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
 }
 
 // Waits until the phase of parity `parity` has completed; false once
-// timeout_ns (by %globaltimer) have passed since the call, or after 2^30
-// polls.
+// timeout_ns (by %globaltimer, read every 16 polls) have passed, or after 2^30
+// polls. Each poll may suspend the thread for up to kPollSuspendNs and ends as
+// soon as the phase completes, so waiting warps do not spin: a poll that
+// returned at once cost the GEMM about 10 % of its time (waiting warps share
+// the issue slots of the MMA and producer lanes, and burn power under the cap).
+constexpr uint32_t kPollSuspendNs = 20000;
+
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint64_t timeout_ns) {
   uint64_t deadline = 0;
   for (uint32_t it = 0; it < (1u << 30); ++it) {
     uint32_t done;
     asm volatile(
-        "{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"
+        "{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3; selp.u32 %0, 1, 0, p; }"
         : "=r"(done)
-        : "r"(bar), "r"(parity)
+        : "r"(bar), "r"(parity), "n"(kPollSuspendNs)
         : "memory");
     if (done) return true;
     if ((it & 15u) == 15u) {
