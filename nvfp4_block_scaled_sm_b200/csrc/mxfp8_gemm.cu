@@ -621,7 +621,7 @@ mxfp8_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_c
 #pragma unroll
         for (uint32_t k = 0; k < 4; k++) {
           mma_mxf8_pair(tmem, op_lo + so + 2 * k, op_lo + so + kTileAW + 2 * k, op_hi,
-                          instr_desc_pair(k), sfa_t | (k << 30), sfb_t | (k << 30), (kb | k) != 0u);
+                        instr_desc_pair(k), sfa_t | (k << 30), sfb_t | (k << 30), (kb | k) != 0u);
         }
         mma_commit_pair(empty_bar(s));
         if (++s == kPairStages) {
