@@ -60,6 +60,19 @@ def test_cpu_baseline_chunks_equal_one_call():
     assert np.array_equal(z[:256 * 8], oracle.swizzle_scales(so)[:256 * 8])
 
 
+@pytest.mark.parametrize("M", [1, 127, 300, 512, 1000, 4096, 16384, 16385])
+def test_e2e_chunks_cover_the_rows(M):
+    """The end-to-end pipeline's chunks tile [0, M) in order, each starting on
+    a 128-row boundary (so its swizzled scales are one slice of the full
+    layout), the first at most 512 rows and none above 2048."""
+    b = bench.e2e_chunks(M)
+    assert b[0] == 0 and b[-1] == M
+    sizes = [r1 - r0 for r0, r1 in zip(b[:-1], b[1:])]
+    assert all(n > 0 for n in sizes)
+    assert all(r0 % 128 == 0 for r0 in b[:-1])
+    assert sizes[0] <= 512 and max(sizes) <= 2048
+
+
 def test_sample_rows():
     import numpy as np
     r = bench.sample_rows(8192, 100, 5)
