@@ -162,26 +162,53 @@ __device__ __forceinline__ void load_expert_rows(const int64_t* __restrict__ g_o
 // the padding writer the padded width 4 ceil(S/4).
 constexpr uint32_t kMaxSwizzleTileCols = 1u << 25;
 
+// Staging tile of the aligned path of mx_swizzle_experts_kernel: 128 rows x
+// 32 words (128 scale columns), row pitch 33 words plus 8 more words per
+// 32-row quarter. A warp that writes one row's 32 words, and a warp that reads
+// one word from each of the 32 rows {b .. b+7} + {0, 32, 64, 96} (one swizzled
+// output line), then touches 32 different banks.
+constexpr uint32_t kSwzChunkWords = 32;
+constexpr uint32_t kSwzPitch = kSwzChunkWords + 1;
+__device__ __forceinline__ uint32_t swz_tile_index(uint32_t r, uint32_t c) {
+  return r * kSwzPitch + (r >> 5) * 8 + c;
+}
+
 // Per-expert swizzled scales of a stacked tensor, gathered from its compact
 // scales [M, S] (written by the quantize launch just before, in stream
 // order): output block i (128 padded rows x Sp = 4 ceil(S/4) columns, at
 // byte 128 i Sp) belongs to the expert e with pb[e] <= 128 i < pb[e + 1] and
 // holds that expert's rows off[e] + 128 i - pb[e] .. +127; rows past the
 // expert's end and columns past S are 0x00. Persistent CTAs build the row
-// table once, then write whole blocks in output order, one 4-byte word (four
-// scale columns of one row) per thread and step. No byte at or past `cap` is
-// written, whatever the offsets hold.
-__global__ void __launch_bounds__(kThreads)
+// table once, then write whole blocks in output order. No byte at or past
+// `cap` is written, whatever the offsets hold.
+//  - words_aligned (S % 4 == 0, 4-byte aligned scales): a block goes through
+//    shared memory in chunks of 32 words (128 columns) per row: each warp
+//    reads whole row segments (coalesced), then each thread writes one output
+//    word (four scale columns of one row) of the swizzled lines.
+//  - otherwise each thread gathers its output words byte by byte from the
+//    compact rows.
+__global__ void __launch_bounds__(kThreads, 4)
 mx_swizzle_experts_kernel(const uint8_t* __restrict__ scale, uint8_t* __restrict__ swz,
                           const int64_t* __restrict__ offs, int32_t E, int64_t M, uint32_t S,
                           uint32_t Sp4, uint64_t cap, bool words_aligned) {
   pdl_enter();
   extern __shared__ int64_t s_rows[];
+  __shared__ uint32_t tile[128 * kSwzPitch + 3 * 8];
   int64_t* off = s_rows;
   int64_t* pb = s_rows + (E + 1);
   load_expert_rows(offs, E, M, off, pb);
   const uint64_t blocks = uint64_t(pb[E]) >> 7;
   const uint32_t words = 128 * Sp4;  // 4-byte words per output block
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  auto store_word = [&](uint64_t o, uint32_t v) {
+    if (o + 4 <= cap) {
+      st_u32(swz + o, v);
+    } else {
+#pragma unroll
+      for (uint32_t k = 0; k < 4; k++)
+        if (o + k < cap) st_u8(swz + o + k, (v >> (8 * k)) & 0xffu);
+    }
+  };
   for (uint64_t i = blockIdx.x; i < blocks; i += gridDim.x) {
     const int64_t prow = int64_t(i) << 7;
     int lo = 0, hi = E;  // invariant: pb[lo] <= prow < pb[hi]
@@ -191,7 +218,43 @@ mx_swizzle_experts_kernel(const uint8_t* __restrict__ scale, uint8_t* __restrict
     }
     const int64_t r0 = off[lo] + (prow - pb[lo]);  // first source row of the block
     const int64_t rend = off[lo + 1];
-    constexpr int kU = 8;  // words per thread and round, all loaded before any is stored
+    if (words_aligned) {
+      // rows r0 .. r0 + nrows - 1 exist (1 <= nrows <= 128: the block lies in
+      // expert lo's padded rows, which start on its first row)
+      const int64_t left = rend - r0;
+      const uint32_t nrows = left < 128 ? uint32_t(left < 0 ? 0 : left) : 128u;
+      const uint32_t* src = reinterpret_cast<const uint32_t*>(scale);  // S / 4 = Sp4 words a row
+      for (uint32_t c0 = 0; c0 < Sp4; c0 += kSwzChunkWords) {
+        const uint32_t cw = Sp4 - c0 < kSwzChunkWords ? Sp4 - c0 : kSwzChunkWords;
+        // a warp takes rows warp, warp + 8, ..., eight loads in flight a lane
+        constexpr uint32_t kWarps = kThreads / 32, kBatch = 8;
+        const uint32_t* row_src = src + uint64_t(r0) * Sp4 + c0 + uint32_t(lane);
+#pragma unroll
+        for (uint32_t b = 0; b < 128 / (kWarps * kBatch); b++) {
+          uint32_t v[kBatch];
+#pragma unroll
+          for (uint32_t k = 0; k < kBatch; k++) {
+            const uint32_t r = uint32_t(warp) + (b * kBatch + k) * kWarps;
+            v[k] = (r < nrows && uint32_t(lane) < cw) ? row_src[r * Sp4] : 0u;  // < 2^32: Sp4 <= 2^25
+          }
+#pragma unroll
+          for (uint32_t k = 0; k < kBatch; k++)
+            tile[swz_tile_index(uint32_t(warp) + (b * kBatch + k) * kWarps, uint32_t(lane))] = v[k];
+        }
+        __syncthreads();
+        // output words of the chunk's tiles c0 .. c0 + cw - 1, in output order:
+        // word wi of tile j holds row (wi % 4) 32 + wi / 4, columns 4 j .. 4 j + 3
+        const uint64_t o0 = (i * words + uint64_t(c0) * 128) * 4;
+        for (uint32_t w = threadIdx.x; w < cw * 128; w += kThreads) {
+          const uint32_t jj = w >> 7, wi = w & 127;
+          const uint32_t r = (wi & 3) * 32 + (wi >> 2);
+          store_word(o0 + 4 * w, tile[swz_tile_index(r, jj)]);
+        }
+        __syncthreads();
+      }
+      continue;
+    }
+    constexpr int kU = 4;  // words per thread and round, all loaded before any is stored
     for (uint32_t w0 = threadIdx.x; w0 < words; w0 += kThreads * kU) {
       uint32_t v[kU];
 #pragma unroll
@@ -202,27 +265,15 @@ mx_swizzle_experts_kernel(const uint8_t* __restrict__ scale, uint8_t* __restrict
         v[u] = 0;
         if (w < words && row < rend) {
           const uint8_t* src = scale + uint64_t(row) * S + 4 * j;
-          if (words_aligned) {
-            v[u] = *reinterpret_cast<const uint32_t*>(src);
-          } else {
 #pragma unroll
-            for (uint32_t k = 0; k < 4; k++)
-              if (4 * j + k < S) v[u] |= uint32_t(src[k]) << (8 * k);
-          }
+          for (uint32_t k = 0; k < 4; k++)
+            if (4 * j + k < S) v[u] |= uint32_t(src[k]) << (8 * k);
         }
       }
 #pragma unroll
       for (int u = 0; u < kU; u++) {
         const uint32_t w = w0 + u * kThreads;
-        if (w >= words) continue;
-        const uint64_t o = (i * words + w) * 4;
-        if (o + 4 <= cap) {
-          st_u32(swz + o, v[u]);
-        } else {
-#pragma unroll
-          for (uint32_t k = 0; k < 4; k++)
-            if (o + k < cap) st_u8(swz + o + k, (v[u] >> (8 * k)) & 0xffu);
-        }
+        if (w < words) store_word((i * words + w) * 4, v[u]);
       }
     }
   }
