@@ -82,6 +82,26 @@ def test_stacked_fp32_and_odd_scale_columns():
     assert_same(host(z), zo, "fp32 per-expert swizzled scales")
 
 
+@pytest.mark.parametrize("S", [132, 256, 4])
+def test_stacked_swizzle_through_the_staged_tile(S):
+    """Scale widths with S % 4 == 0 go through the gather's shared-memory tile
+    in chunks of 128 columns: S = 132 gives a full chunk and a 4-column
+    remainder, S = 256 two full chunks, S = 4 one 4-column chunk. Ragged
+    experts (one empty, partial 128-row blocks) and the single-tensor form of
+    the same gather on the whole stack."""
+    rows = [130, 0, 1, 255, 128, 3]
+    N = 32 * S
+    parts = [W.linear_weight(seed=300 + i, M=max(r, 1), N=N)[:r] for i, r in enumerate(rows)]
+    x = np.concatenate(parts, 0)
+    offs = np.concatenate([[0], np.cumsum(rows)]).tolist()
+    q, s, z = mxq.mxfp8_quantize_grouped(dev(x), row_offsets=offs, swizzled=True)
+    qo, so, zo = oracle.mxfp8_quantize_grouped(parts, swizzled=True)
+    assert_same(host(q), qo, f"S={S} stacked codes")
+    assert_same(host(s), so, f"S={S} stacked scales")
+    assert_same(host(z), zo, f"S={S} per-expert swizzled scales")
+    assert_same(host(mxq.swizzle_scales(s)), oracle.swizzle_scales(so), f"S={S} whole-stack swizzle")
+
+
 def _stacked_swizzled_raw():
     f = ctypes.CDLL(mxq.library_path).mxfp8_quantize_grouped_swizzled
     vp, i64, i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
