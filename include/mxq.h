@@ -315,6 +315,22 @@ mxq_status mxfp8_gemm(const uint8_t* qa, const uint8_t* sa_swz, const uint8_t* q
                       const uint8_t* sb_swz, int64_t M, int64_t N, int64_t K, void* d,
                       int out_dt, int32_t* error_flag, mxq_stream_t stream);
 
+/* Self-check of the bounded barrier wait that lets mxfp8_gemm give up
+ * instead of hanging (the wait behind error_flag), run on the device in one
+ * single-thread launch: first a wait, limited to timeout_ns, on a
+ * shared-memory barrier that nothing arrives on; then a wait on a barrier
+ * whose phase the thread has just completed. Writes the device array result
+ * (4 int64, 8-byte aligned):
+ *   result[0]  1 if the first wait gave up, else 0 (expected 1);
+ *   result[1]  1 if the second wait saw its phase complete, else 0 (1);
+ *   result[2]  nanoseconds the first wait took, by %globaltimer;
+ *   result[3]  0.
+ * The wait polls with a 20 us suspend hint and reads %globaltimer every 16
+ * polls, so the first wait ends within about timeout_ns + 0.7 ms.
+ * 1000 <= timeout_ns <= 1000000000, else MXQ_ERR_ARG; result NULL ->
+ * MXQ_ERR_NULL; result not 8-byte aligned -> MXQ_ERR_ALIGN. */
+mxq_status mxq_check_bounded_wait(int64_t timeout_ns, int64_t* result, mxq_stream_t stream);
+
 /* ------------------------------------------------------------------ NVFP4 */
 
 /* Workspace bytes nvfp4_quantize / nvfp4_amax need (per-CTA partial maxima of

@@ -78,6 +78,7 @@ def _load() -> ctypes.CDLL:
     L.mxfp4_quantize_grouped_ptrs.argtypes = [i32, vp, vp, i64, i32, vp, vp, vp]
     L.mx_fake_quantize.argtypes = [i32, vp, i32, i64, i64, i64, vp, i32, vp]
     L.mxfp8_gemm.argtypes = [vp, vp, vp, vp, i64, i64, i64, vp, i32, vp, vp]
+    L.mxq_check_bounded_wait.argtypes = [i64, vp, vp]
     L.nvfp4_amax.argtypes = [vp, i32, i64, i64, i64, vp, vp, sz, vp]
     L.nvfp4_quantize.argtypes = [vp, i32, i64, i64, i64, vp, vp, vp, vp, u32, vp, sz, vp]
     L.nvfp4_dequantize.argtypes = [vp, vp, vp, i64, i64, vp, i32, vp]
@@ -90,7 +91,8 @@ def _load() -> ctypes.CDLL:
               "mxfp8_quantize_grouped_swizzled", "mxfp8_quantize_grouped_ptrs",
               "mxfp8_quantize_columnwise", "mxfp4_quantize", "mxfp4_dequantize",
               "mxfp4_quantize_grouped", "mxfp4_quantize_grouped_swizzled",
-              "mxfp4_quantize_grouped_ptrs", "mx_fake_quantize", "mxq_swizzle_scales", "mxfp8_gemm", "nvfp4_amax",
+              "mxfp4_quantize_grouped_ptrs", "mx_fake_quantize", "mxq_swizzle_scales", "mxfp8_gemm",
+              "mxq_check_bounded_wait", "nvfp4_amax",
               "nvfp4_quantize_sliced", "nvfp4_amax_sliced",
               "nvfp4_quantize", "nvfp4_dequantize"):
         getattr(L, f).restype = i32
@@ -449,6 +451,20 @@ def mxfp8_gemm(qa: torch.Tensor, sa_swizzled: torch.Tensor, qb: torch.Tensor,
                                         M, N, K, _ptr(d), _dtype_code(dtype), _ptr(error_flag),
                                         _stream(qa)))
     return d
+
+
+def check_bounded_wait(timeout_ns: int = 2_000_000, device=None) -> dict:
+    """Runs the self-check of the GEMM's bounded barrier wait on a CUDA device
+    (``mxq_check_bounded_wait``): a wait on a barrier that nothing arrives on
+    must give up after ``timeout_ns``, and a wait on a completed phase must
+    return. Returns ``{"gave_up": bool, "completed": bool, "waited_ns": int}``
+    after synchronizing the stream."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    result = torch.full((4,), -1, dtype=torch.int64, device=dev)
+    _check("mxq_check_bounded_wait",
+           lib.mxq_check_bounded_wait(int(timeout_ns), _ptr(result), _stream(result)))
+    r = result.cpu().tolist()
+    return {"gave_up": r[0] == 1, "completed": r[1] == 1, "waited_ns": r[2]}
 
 
 # ------------------------------------------------------------------ NVFP4

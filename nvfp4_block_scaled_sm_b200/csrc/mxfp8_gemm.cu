@@ -722,6 +722,28 @@ mxfp8_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_c
   }
 }
 
+// The GEMM's bounded wait, both ways (see mxq_check_bounded_wait): a barrier
+// that nothing arrives on must make mbar_wait give up after timeout_ns, and
+// one whose phase has completed must let it return at once. One thread; no
+// asynchronous operation refers to either barrier, so the CTA may exit with
+// the first one's phase still open.
+__global__ void bounded_wait_check_kernel(uint64_t timeout_ns, int64_t* result) {
+  __shared__ alignas(8) uint64_t bars[2];
+  if (threadIdx.x != 0) return;
+  const uint32_t never = smem_u32(&bars[0]), done = smem_u32(&bars[1]);
+  mbar_init(never, 1);
+  mbar_init(done, 1);
+  const uint64_t t0 = globaltimer();
+  const bool first = mbar_wait(never, 0, timeout_ns);
+  const uint64_t t1 = globaltimer();
+  mbar_arrive(done);
+  const bool second = mbar_wait(done, 0, timeout_ns);
+  result[0] = first ? 0 : 1;
+  result[1] = second ? 1 : 0;
+  result[2] = int64_t(t1 - t0);
+  result[3] = 0;
+}
+
 // ------------------------------------------------------------------ host
 
 // [rows, K] bytes, row stride K, boxes of box_rows rows x 128 bytes,
@@ -871,4 +893,15 @@ extern "C" mxq_status mxfp8_gemm(const uint8_t* qa, const uint8_t* sa_swz, const
   if (out_dt == MXQ_BF16)
     return wide ? launch_gemm<uint16_t, 256>(ta, tb, args, s) : launch_gemm<uint16_t, 128>(ta, tb, args, s);
   return wide ? launch_gemm<float, 256>(ta, tb, args, s) : launch_gemm<float, 128>(ta, tb, args, s);
+}
+
+extern "C" mxq_status mxq_check_bounded_wait(int64_t timeout_ns, int64_t* result,
+                                             mxq_stream_t stream) {
+  using namespace mxq;
+  if (timeout_ns < 1000 || timeout_ns > 1000000000) return MXQ_ERR_ARG;
+  if (!result) return MXQ_ERR_NULL;
+  if (reinterpret_cast<uintptr_t>(result) & 7u) return MXQ_ERR_ALIGN;
+  bounded_wait_check_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      uint64_t(timeout_ns), result);
+  return launched(cudaGetLastError());
 }

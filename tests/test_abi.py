@@ -44,6 +44,18 @@ def test_library_exports_every_declared_symbol():
     assert not missing, missing
 
 
+def test_bounded_wait_check_validation():
+    """The bounded-wait self-check rejects limits outside [1 us, 1 s] and a
+    NULL or misaligned result array before any launch."""
+    f = mxq.lib.mxq_check_bounded_wait
+    fake = ctypes.c_void_p(1 << 20)                  # never dereferenced: rejected first
+    assert f(999, fake, None) == 7                   # MXQ_ERR_ARG
+    assert f(10**9 + 1, fake, None) == 7
+    assert f(-5, fake, None) == 7
+    assert f(2_000_000, None, None) == 1             # MXQ_ERR_NULL
+    assert f(2_000_000, ctypes.c_void_p((1 << 20) + 4), None) == 4   # MXQ_ERR_ALIGN
+
+
 def test_version_and_strings():
     assert mxq.lib.mxq_abi_version() == 2
     for s in range(8):
