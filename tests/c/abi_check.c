@@ -63,6 +63,11 @@ int main(void) {
   /* GEMM */
   expect("gemm K % 32", mxfp8_gemm(B, B, B, B, 128, 128, 48, A, MXQ_BF16, NULL, s), MXQ_ERR_SHAPE);
   expect("gemm NULL output", mxfp8_gemm(B, B, B, B, 128, 128, 64, NULL, MXQ_BF16, NULL, s), MXQ_ERR_NULL);
+  expect("bounded wait limit below 1 us", mxq_check_bounded_wait(999, (int64_t*)A, s), MXQ_ERR_ARG);
+  expect("bounded wait limit above 1 s", mxq_check_bounded_wait(1000000001, (int64_t*)A, s), MXQ_ERR_ARG);
+  expect("bounded wait NULL result", mxq_check_bounded_wait(2000000, NULL, s), MXQ_ERR_NULL);
+  expect("bounded wait misaligned result", mxq_check_bounded_wait(2000000, (int64_t*)(B + 4), s),
+         MXQ_ERR_ALIGN);
 
   /* NVFP4 */
   float* g = (float*)A;
