@@ -36,7 +36,7 @@ __device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
 // polls. Each poll may suspend the thread for up to kPollSuspendNs and ends as
 // soon as the phase completes, so waiting warps do not spin: a poll that
 // returned at once cost the GEMM about 10 % of its time (waiting warps share
-// the issue slots of the MMA and producer lanes, and burn power under the cap).
+// the issue slots of the MMA and producer warps, and burn power under the cap).
 constexpr uint32_t kPollSuspendNs = 20000;
 
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint64_t timeout_ns) {
