@@ -110,7 +110,7 @@ int64_t mxq_swizzled_scale_bytes(int64_t M, int64_t S);
  *           tensor-core MMA (tile (i, j) = rows 128i.., scale columns 4j..,
  *           at byte (i*ceil(S/4) + j)*512; entry (r, c) inside it at
  *           (r%32)*16 + ((r%128)/32)*4 + c%4; padding bytes are 0x00);
- *           N/32 > 2^27 with scale_swz is rejected (MXQ_ERR_SHAPE).
+ *           N/32 > 2^27 - 4 with scale_swz is rejected (MXQ_ERR_SHAPE).
  * Per group: amax = max |x| over non-NaN elements; byte = 127 if amax == 0,
  * 254 if amax is infinite, else clamp(floor(log2 amax) - 8 + 127, 0, 254);
  * q = E4M3(x * 2^(127 - byte)) rounded to nearest even, |.| > 448 saturating
@@ -164,7 +164,7 @@ mxq_status mxfp8_quantize_grouped(const void* x, int dt, int32_t E, const int64_
  * expert's compact scales into its swizzled block, which reads row_offsets on
  * the device. Offsets that break the rules above are clamped into a
  * non-decreasing sequence from 0 to M_total, and no byte at or past
- * scale_swz + swz_bytes is written, whatever the offsets. N/32 > 2^27 is
+ * scale_swz + swz_bytes is written, whatever the offsets. N/32 > 2^27 - 4 is
  * rejected (MXQ_ERR_SHAPE). */
 mxq_status mxfp8_quantize_grouped_swizzled(const void* x, int dt, int32_t E,
                                            const int64_t* row_offsets, int64_t M_total, int64_t N,
@@ -179,7 +179,7 @@ mxq_status mxfp8_quantize_grouped_swizzled(const void* x, int dt, int32_t E,
  * such step; it lays out what the quantizers wrote.)
  *  scale      device [M, S] bytes, row-major, compact.
  *  scale_swz  device, 16-byte aligned, mxq_swizzled_scale_bytes(M, S) bytes.
- * M == 0 or S == 0 writes nothing; S > 2^27 is rejected (MXQ_ERR_SHAPE).
+ * M == 0 or S == 0 writes nothing; S > 2^27 - 4 is rejected (MXQ_ERR_SHAPE).
  * One launch. */
 mxq_status mxq_swizzle_scales(const uint8_t* scale, int64_t M, int64_t S, uint8_t* scale_swz,
                               mxq_stream_t stream);

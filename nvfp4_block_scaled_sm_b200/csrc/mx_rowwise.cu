@@ -157,10 +157,11 @@ __device__ __forceinline__ void load_expert_rows(const int64_t* __restrict__ g_o
   __syncthreads();
 }
 
-// Swizzled scales are limited to S <= 2^27 columns (2^25 four-column tiles):
-// the gather counts the 4-byte words of a 128-row output block in 32 bits, and
+// Swizzled scales are limited to S <= 2^27 - 4 columns (2^25 - 1 four-column
+// tiles): the gather counts the 4-byte words of a 128-row output block,
+// 128 ceil(S/4), in 32 bits (2^25 tiles would make that count wrap to 0), and
 // the padding writer the padded width 4 ceil(S/4).
-constexpr uint32_t kMaxSwizzleTileCols = 1u << 25;
+constexpr uint32_t kMaxSwizzleTileCols = (1u << 25) - 1;
 
 // Staging tile of the aligned path of mx_swizzle_experts_kernel: 128 rows x
 // 32 words (128 scale columns), row pitch 33 words plus 8 more words per

@@ -83,7 +83,7 @@ def test_mxfp8_quantize_validation():
     assert L.mxfp8_quantize(A + 2, 0, 4, 64, 64, A, A, None, None) == ALIGN
     assert L.mxfp8_quantize(A, 0, 4, 64, 68, A, A, None, None) == ALIGN
     assert L.mxfp8_quantize(A, 0, 4, 64, 64, A + 8, A, None, None) == ALIGN
-    big = 32 * ((1 << 27) + 1)        # swizzled scales take at most 2^27 columns
+    big = 32 * ((1 << 27) - 3)        # swizzled scales take at most 2^27 - 4 columns
     assert L.mxfp8_quantize(A, 0, 1, big, big, A, A, A, None) == SHAPE
     assert L.mxfp4_quantize(A, 0, 1, big, big, A, A, A, None) == SHAPE
     # empty inputs succeed without touching any pointer
@@ -193,7 +193,7 @@ def test_grouped_stacked_validation():
         assert G(A, 0, 4, O, 64, 64, A, A, A, -1, None) == SHAPE
         assert G(A, 0, 4, None, 64, 64, A, A, A, 4096, None) == NULL
         assert G(A, 0, 4, O, 64, 64, A, A, A + 8, 4096, None) == ALIGN
-        assert G(A, 0, 4, O, 1, 32 * ((1 << 27) + 1), A, A, A, 1 << 40, None) == SHAPE
+        assert G(A, 0, 4, O, 1, 32 * ((1 << 27) - 3), A, A, A, 1 << 40, None) == SHAPE
         assert G(None, 0, 4, O, 0, 64, None, None, A, 0, None) == OK
 
 
@@ -204,7 +204,9 @@ def test_swizzle_scales_validation():
     assert Z(None, 4, 4, A, None) == NULL
     assert Z(A, 4, 4, None, None) == NULL
     assert Z(A, 4, 4, A + 4, None) == ALIGN
-    assert Z(A, 4, (1 << 27) + 1, A, None) == SHAPE
+    assert Z(A, 4, (1 << 27) - 3, A, None) == SHAPE
+    assert Z(A, 4, 1 << 27, A, None) == SHAPE     # 2^25 tiles: the word count would wrap
+    assert Z(A, 4, (1 << 27) - 4, A, None) == CUDA  # the widest accepted: validation passes, the launch fails here
     assert Z(None, 0, 4, None, None) == OK
     assert Z(None, 4, 0, None, None) == OK
 
